@@ -1,0 +1,254 @@
+"""Plain fp64 CPU oracle for SQuad-Attention.
+
+TEST INFRASTRUCTURE ONLY. Nothing in the product path imports, calls or executes this module: only
+``tests/``, ``__graft_entry__.smoke()`` and ``bench.py`` (its ``cpu_baseline`` leg and ``--impl
+reference``) may use it. It shares no code with the CUDA library; both sides are fed from the seeded
+generator in ``sub_quadratic_two_squad_b200/inputs.py``, which holds no attention arithmetic.
+
+Sources ("SQuad: Sub-Quadratic Attention Distillation for Efficient Video Generation", as printed on
+the paperpeel page, the agihunt digest and the romaanj.github.io review):
+
+* Full softmax self-attention softmax(Q K^T / sqrt(d)) V per head -- paper §3.1 (eq. 5).
+* SQuad-Attention is two ordinary softmax attentions run one after the other; between them there is
+  only re-indexing, the attended axis becomes the sequence and the other axis is folded into the
+  batch/head dimension -- agihunt digest, paragraph "SQuad-Attention composes two ordinary softmax
+  attentions"; paper §4.3 ("two passes are ordinary softmax attentions separated by pure
+  re-indexing").
+* Local pass: each token attends inside its window; the window spans the full temporal extent and
+  tiles space (e.g. 21x2x4 = 168 tokens at n = 18480) -- agihunt digest, "The window size carries the
+  whole argument"; review, "Method".
+* Global pass: tokens at the same position (slot) inside their windows attend across all windows, and
+  the local output is its value stream -- paper appendix "Reachability" (two-hop path (c',j') ->
+  (c',j) -> (c,j)); gist.science technical summary, "Composição".
+* Order: local->global is the paper's default, global->local the ablated reverse; for G->L the
+  effective weight is beta_{j->j'}^{c} alpha_{c->c'}^{j'} -- paper appendix "On the ordering".
+* Cost: 4hd(n w + n^2 / w) for the two passes and 4hdn^2 for full attention -- paper appendix
+  "Conformance to the theoretical curves is quantitative".
+
+Readings where the pages are silent (equations 7-9 were lost in extraction):
+
+* Pass 2 takes the same Q and K, rearranged to the slot view; its values are the pass-1 output.
+* Both passes use the eq. 5 scale 1/sqrt(d) unless the caller passes another.
+* Tokens are flattened (t, y, x) row-major: token = (t*H + y)*W + x. Window c = (wy, wx) runs
+  row-major over (H/hw, W/ww); slot j = (t, dy, dx) runs row-major over (tw, hw, ww). The result does
+  not depend on these orders (softmax sums are permutation invariant; outputs go back to token order).
+* The backward pass is the chain rule through both passes; the pages do not print it.
+
+Every array here is float64. Pins: tests/test_oracle_pins.py.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+
+# ----------------------------------------------------------------------------------------------
+# Re-indexing (the "local" and "global" token views)
+# ----------------------------------------------------------------------------------------------
+
+def window_partition(T: int, H: int, W: int, tw: int, hw: int, ww: int) -> np.ndarray:
+    """Token index of slot j inside window c, as an int array [N_w, w].
+
+    Row c lists the w = tw*hw*ww tokens of window c (the local pass attends along a row); column j
+    lists the N_w tokens that occupy slot j in every window (the global pass attends along a column).
+    """
+    if tw != T:
+        raise ValueError("the window spans the full temporal extent: tw must equal T")
+    if H % hw or W % ww:
+        raise ValueError("window must tile the H x W grid exactly")
+    nwy, nwx = H // hw, W // ww
+    table = np.empty((nwy * nwx, tw * hw * ww), dtype=np.int64)
+    for wy in range(nwy):
+        for wx in range(nwx):
+            c = wy * nwx + wx
+            for t in range(tw):
+                for dy in range(hw):
+                    for dx in range(ww):
+                        j = (t * hw + dy) * ww + dx
+                        y = wy * hw + dy
+                        x = wx * ww + dx
+                        table[c, j] = (t * H + y) * W + x
+    return table
+
+
+# ----------------------------------------------------------------------------------------------
+# One softmax attention over a batch of sequences (eq. 5)
+# ----------------------------------------------------------------------------------------------
+
+def softmax_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float):
+    """softmax(q k^T * scale) v over the last-but-one axis; returns (out, lse).
+
+    q: [..., s, d], k: [..., s, d], v: [..., s, dv]. lse is the natural-log log-sum-exp of the scaled
+    scores per query row, [..., s]. The softmax subtracts the row maximum (exact in real arithmetic).
+    """
+    s = np.matmul(q, np.swapaxes(k, -1, -2)) * scale
+    m = s.max(axis=-1, keepdims=True)
+    p = np.exp(s - m)
+    l = p.sum(axis=-1, keepdims=True)
+    out = np.matmul(p / l, v)
+    lse = (m + np.log(l))[..., 0]
+    return out, lse
+
+
+def softmax_attention_bwd(q, k, v, dout, scale: float):
+    """Gradients (dq, dk, dv) of <dout, softmax(q k^T * scale) v> by the chain rule.
+
+    P = softmax(S), S = scale q k^T, out = P v:
+      dv = P^T dout;  dP = dout v^T;  dS = P * (dP - rowsum(dP * P));  dq = scale dS k;  dk = scale dS^T q.
+    """
+    s = np.matmul(q, np.swapaxes(k, -1, -2)) * scale
+    s = s - s.max(axis=-1, keepdims=True)
+    p = np.exp(s)
+    p = p / p.sum(axis=-1, keepdims=True)
+    dv = np.matmul(np.swapaxes(p, -1, -2), dout)
+    dp = np.matmul(dout, np.swapaxes(v, -1, -2))
+    ds = p * (dp - (dp * p).sum(axis=-1, keepdims=True))
+    dq = np.matmul(ds, k) * scale
+    dk = np.matmul(np.swapaxes(ds, -1, -2), q) * scale
+    return dq, dk, dv
+
+
+# ----------------------------------------------------------------------------------------------
+# The two passes
+# ----------------------------------------------------------------------------------------------
+
+def _scale(d: int, scale):
+    return 1.0 / np.sqrt(d) if scale is None else float(scale)
+
+
+def _pass(Q, K, V, groups: np.ndarray, scale: float):
+    """Attention inside every group of tokens (a row of ``groups`` is one sequence), per (b, head).
+
+    Q, K: [B, h, n, d]; V: [B, h, n, dv]; groups: [G, s] token indices. Returns (out [B,h,n,dv],
+    lse [B,h,n]). Heads are independent, so they are processed one at a time to bound memory.
+    """
+    B, h, n, _ = Q.shape
+    out = np.empty(V.shape, dtype=np.float64)
+    lse = np.empty((B, h, n), dtype=np.float64)
+    for b in range(B):
+        for hh in range(h):
+            qg = Q[b, hh][groups]          # [G, s, d]
+            kg = K[b, hh][groups]
+            vg = V[b, hh][groups]          # [G, s, dv]
+            o, l = softmax_attention(qg, kg, vg, scale)
+            out[b, hh][groups] = o
+            lse[b, hh][groups] = l
+    return out, lse
+
+
+def local_pass(Q, K, V, grid, window, scale=None):
+    """Attn_L: full softmax attention inside each window of tw x hw x ww tokens (tw = T)."""
+    table = window_partition(*grid, *window)
+    return _pass(_f64(Q), _f64(K), _f64(V), table, _scale(Q.shape[-1], scale))
+
+
+def global_pass(Q, K, V, grid, window, scale=None):
+    """Attn_G: for every slot j, the tokens at slot j of all n/w windows attend to one another."""
+    table = window_partition(*grid, *window)
+    return _pass(_f64(Q), _f64(K), _f64(V), np.ascontiguousarray(table.T), _scale(Q.shape[-1], scale))
+
+
+def _f64(x):
+    return np.asarray(x, dtype=np.float64)
+
+
+LOCAL_THEN_GLOBAL = "local_then_global"
+GLOBAL_THEN_LOCAL = "global_then_local"
+
+
+def squad_attn_fwd(Q, K, V, grid, window, order=LOCAL_THEN_GLOBAL, scale=None, return_aux=False):
+    """SQuad-Attention forward: the two passes composed, pass 2 taking pass 1's output as values.
+
+    grid = (T, H, W); window = (tw, hw, ww). Q, K: [B, h, n, d], V: [B, h, n, dv] with n = T*H*W.
+    With return_aux, also returns dict(o1=..., lse1=..., lse2=...) (pass-1 output and both passes'
+    log-sum-exp).
+    """
+    if order not in (LOCAL_THEN_GLOBAL, GLOBAL_THEN_LOCAL):
+        raise ValueError(order)
+    first, second = (local_pass, global_pass) if order == LOCAL_THEN_GLOBAL else (global_pass, local_pass)
+    o1, lse1 = first(Q, K, V, grid, window, scale)
+    o, lse2 = second(Q, K, o1, grid, window, scale)
+    if return_aux:
+        return o, dict(o1=o1, lse1=lse1, lse2=lse2)
+    return o
+
+
+def squad_attn_bwd(Q, K, V, dO, grid, window, order=LOCAL_THEN_GLOBAL, scale=None):
+    """Gradients (dQ, dK, dV) of <dO, squad_attn_fwd(Q, K, V)>.
+
+    Reverse of the two passes: pass 2's backward (values = pass-1 output) gives its share of dQ and dK
+    and the gradient dO1 of the pass-1 output; pass 1's backward with upstream dO1 gives the rest of dQ
+    and dK, and dV. Q and K are used by both passes, so each receives the sum of two terms.
+    """
+    Q, K, V, dO = _f64(Q), _f64(K), _f64(V), _f64(dO)
+    sc = _scale(Q.shape[-1], scale)
+    table = window_partition(*grid, *window)
+    local_groups, global_groups = table, np.ascontiguousarray(table.T)
+    g1, g2 = (local_groups, global_groups) if order == LOCAL_THEN_GLOBAL else (global_groups, local_groups)
+    o1, _ = _pass(Q, K, V, g1, sc)
+
+    dQ = np.zeros_like(Q)
+    dK = np.zeros_like(K)
+    dV = np.empty_like(V)
+    B, h = Q.shape[:2]
+    for b in range(B):
+        for hh in range(h):
+            q, k, v, do, x1 = Q[b, hh], K[b, hh], V[b, hh], dO[b, hh], o1[b, hh]
+            dq2, dk2, do1 = softmax_attention_bwd(q[g2], k[g2], x1[g2], do[g2], sc)
+            d_o1 = np.empty_like(x1)
+            d_o1[g2] = do1
+            dq1, dk1, dv1 = softmax_attention_bwd(q[g1], k[g1], v[g1], d_o1[g1], sc)
+            dq = np.zeros_like(q)
+            dk = np.zeros_like(k)
+            dq[g2] += dq2
+            dk[g2] += dk2
+            dq[g1] += dq1
+            dk[g1] += dk1
+            dQ[b, hh] = dq
+            dK[b, hh] = dk
+            dV[b, hh][g1] = dv1
+    return dQ, dK, dV
+
+
+# ----------------------------------------------------------------------------------------------
+# Full attention, the composed weight matrix, and the cost model
+# ----------------------------------------------------------------------------------------------
+
+def full_attn_fwd(Q, K, V, scale=None, rows=None):
+    """softmax(Q K^T * scale) V over all n tokens per head (eq. 5); optionally only query ``rows``.
+
+    Returns (out [B,h,r,dv], lse [B,h,r]) with r = n or len(rows).
+    """
+    Q, K, V = _f64(Q), _f64(K), _f64(V)
+    sc = _scale(Q.shape[-1], scale)
+    if rows is not None:
+        Q = Q[:, :, np.asarray(rows), :]
+    B, h = Q.shape[:2]
+    out = np.empty(Q.shape[:3] + (V.shape[-1],))
+    lse = np.empty(Q.shape[:3])
+    for b in range(B):
+        for hh in range(h):
+            out[b, hh], lse[b, hh] = softmax_attention(Q[b, hh], K[b, hh], V[b, hh], sc)
+    return out, lse
+
+
+def composed_matrix(Q, K, grid, window, order=LOCAL_THEN_GLOBAL, scale=None):
+    """The n x n matrix M with squad_attn_fwd(Q, K, V) = M V, per (b, head).
+
+    Obtained by pushing the n one-hot value vectors through both passes (V = identity, dv = n). Entry
+    M[u, v] is the effective weight gamma from source token v to target token u (paper appendix
+    "Reachability": a product of two softmax weights).
+    """
+    B, h, n, _ = Q.shape
+    eye = np.broadcast_to(np.eye(n), (B, h, n, n))
+    return squad_attn_fwd(Q, K, eye, grid, window, order, scale)
+
+
+def squad_flops(B: int, h: int, d: int, n: int, w: int) -> float:
+    """4 B h d (n w + n^2 / w): QK^T and PV of the local pass (n/w windows of w tokens) plus those of
+    the global pass (w slots of n/w tokens); each GEMM of an s-token sequence costs 2 s^2 d FLOPs."""
+    return 4.0 * B * h * d * (n * w + n * n / w)
+
+
+def full_flops(B: int, h: int, d: int, n: int) -> float:
+    """4 B h d n^2: QK^T and PV of full attention."""
+    return 4.0 * B * h * d * n * n

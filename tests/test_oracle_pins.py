@@ -1,0 +1,293 @@
+"""Pins for the fp64 oracle, against what the pages and the mathematics fix (no GPU).
+
+Each test checks the oracle against something other than itself: a library routine (torch SDPA and
+autograd in float64), a dense masked-attention construction built from token coordinates (not from
+the oracle's window table), closed forms, finite differences, invariants, or the pages' printed
+numbers (tests/golden/pages_flop_counts.json).
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import squad_oracle as orc
+from sub_quadratic_two_squad_b200.inputs import make_inputs
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+ORDERS = [orc.LOCAL_THEN_GLOBAL, orc.GLOBAL_THEN_LOCAL]
+
+
+def _coords(T, H, W):
+    return np.unravel_index(np.arange(T * H * W), (T, H, W))
+
+
+def _rand(shape, seed):
+    return np.random.default_rng(seed).standard_normal(shape)
+
+
+def _sdpa(q, k, v, scale=None):
+    """torch's scaled_dot_product_attention in float64 on the CPU (library reference)."""
+    tq, tk, tv = (torch.from_numpy(np.ascontiguousarray(x, dtype=np.float64)) for x in (q, k, v))
+    return torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, scale=scale).numpy()
+
+
+def _dense_masked_softmax(q, k, mask, scale):
+    s = q @ k.T * scale
+    s = np.where(mask, s, -np.inf)
+    s = s - s.max(axis=1, keepdims=True)
+    p = np.exp(s)
+    return p / p.sum(axis=1, keepdims=True)
+
+
+def _masks(T, H, W, hw, ww):
+    """Same-window and same-slot masks from token coordinates alone (the pages' description: a window
+    is an hw x ww spatial block over all T frames; a slot is a position (t, y mod hw, x mod ww))."""
+    t, y, x = _coords(T, H, W)
+    same_window = ((y // hw)[:, None] == (y // hw)[None, :]) & ((x // ww)[:, None] == (x // ww)[None, :])
+    same_slot = ((t[:, None] == t[None, :]) & ((y % hw)[:, None] == (y % hw)[None, :])
+                 & ((x % ww)[:, None] == (x % ww)[None, :]))
+    return same_window, same_slot
+
+
+# ------------------------------------------------------------------------------------------------
+# the re-indexing
+# ------------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("grid,window", [((3, 4, 6), (3, 2, 3)), ((5, 8, 8), (5, 2, 2)), ((2, 6, 4), (2, 3, 1))])
+def test_partition_is_window_and_slot_view(grid, window):
+    T, H, W = grid
+    _, hw, ww = window
+    table = orc.window_partition(*grid, *window)
+    t, y, x = _coords(T, H, W)
+    assert table.shape == ((H // hw) * (W // ww), T * hw * ww)
+    assert sorted(table.ravel().tolist()) == list(range(T * H * W))
+    for row in table:  # one spatial block, every frame
+        assert len(set(zip((y[row] // hw).tolist(), (x[row] // ww).tolist()))) == 1
+        assert set(t[row].tolist()) == set(range(T))
+    for col in table.T:  # one slot position, every window
+        assert len(set(zip(t[col].tolist(), (y[col] % hw).tolist(), (x[col] % ww).tolist()))) == 1
+        assert len(set(zip((y[col] // hw).tolist(), (x[col] // ww).tolist()))) == len(table)
+
+
+def test_partition_rejects_what_the_method_excludes():
+    with pytest.raises(ValueError):
+        orc.window_partition(5, 8, 8, 4, 2, 2)     # window must span all T frames
+    with pytest.raises(ValueError):
+        orc.window_partition(5, 8, 8, 5, 3, 2)     # must tile H
+
+
+# ------------------------------------------------------------------------------------------------
+# (a) special cases that reduce to full attention (torch SDPA, float64)
+# ------------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("order", ORDERS)
+def test_single_window_is_full_attention(order):
+    """w = n: the local pass is full attention and every global group has one token."""
+    x = make_inputs(1, 4, 320, 64, dtype="fp32")
+    grid = (5, 8, 8)
+    out = orc.squad_attn_fwd(x["q"], x["k"], x["v"], grid, grid, order)
+    ref = _sdpa(x["q"], x["k"], x["v"])
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
+    full, _ = orc.full_attn_fwd(x["q"], x["k"], x["v"])
+    np.testing.assert_allclose(full, ref, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("order", ORDERS)
+def test_unit_window_is_full_attention(order):
+    """w = 1 (T = 1, window 1x1x1): the local pass is the identity and the global pass is full attention."""
+    x = make_inputs(1, 2, 30, 16, dtype="fp32")
+    out = orc.squad_attn_fwd(x["q"], x["k"], x["v"], (1, 6, 5), (1, 1, 1), order)
+    np.testing.assert_allclose(out, _sdpa(x["q"], x["k"], x["v"]), rtol=0, atol=1e-12)
+
+
+def test_full_attention_rows_and_scale():
+    x = make_inputs(2, 2, 50, 8, dtype="fp32")
+    rows = np.array([0, 7, 49])
+    out, lse = orc.full_attn_fwd(x["q"], x["k"], x["v"], scale=0.3, rows=rows)
+    ref = _sdpa(x["q"][:, :, rows], x["k"], x["v"], scale=0.3)
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
+    s = np.einsum("bhid,bhjd->bhij", x["q"][:, :, rows].astype(np.float64), x["k"].astype(np.float64)) * 0.3
+    np.testing.assert_allclose(lse, np.log(np.exp(s).sum(-1)), rtol=1e-13)
+
+
+# ------------------------------------------------------------------------------------------------
+# (b) constant values come back unchanged (both passes are convex combinations)
+# ------------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("order", ORDERS)
+def test_constant_values_returned(order):
+    x = make_inputs(1, 4, 320, 64, dtype="fp32")
+    c = _rand((1, 4, 1, 64), 3)
+    v = np.broadcast_to(c, (1, 4, 320, 64))
+    out = orc.squad_attn_fwd(x["q"], x["k"], v, (5, 8, 8), (5, 2, 2), order)
+    np.testing.assert_allclose(out, np.broadcast_to(c, out.shape), rtol=0, atol=1e-13)
+
+
+# ------------------------------------------------------------------------------------------------
+# (c) the composed n x n weight matrix: brute force from dense masked attention, rows sum to one,
+#     no structural zeros (paper appendix "Reachability"), orders differ ("On the ordering")
+# ------------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("grid,window,d", [((2, 4, 4), (2, 2, 2), 16), ((5, 8, 8), (5, 2, 2), 64)])
+def test_composed_matrix_brute_force(grid, window, d):
+    T, H, W = grid
+    _, hw, ww = window
+    n = T * H * W
+    q, k = _rand((1, 2, n, d), 1), _rand((1, 2, n, d), 2)
+    same_window, same_slot = _masks(T, H, W, hw, ww)
+    scale = 1 / np.sqrt(d)
+    ms = {}
+    for order in ORDERS:
+        m = orc.composed_matrix(q, k, grid, window, order)
+        ms[order] = m
+        for hh in range(2):
+            a_l = _dense_masked_softmax(q[0, hh], k[0, hh], same_window, scale)
+            a_g = _dense_masked_softmax(q[0, hh], k[0, hh], same_slot, scale)
+            brute = a_g @ a_l if order == orc.LOCAL_THEN_GLOBAL else a_l @ a_g
+            np.testing.assert_allclose(m[0, hh], brute, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(m.sum(-1), 1.0, rtol=0, atol=1e-12)
+        assert (m > 0).all(), "full receptive field: every source reaches every target"
+    assert np.abs(ms[ORDERS[0]] - ms[ORDERS[1]]).max() > 1e-3
+
+
+def test_composed_weight_is_two_hop_product():
+    """gamma_{(c,j)<-(c',j')} = alpha_G(j; c->c') * alpha_L(c'; j->j') for L->G (appendix "Reachability")."""
+    grid, window, d = (2, 4, 4), (2, 2, 2), 8
+    n = 32
+    q, k = _rand((1, 1, n, d), 5), _rand((1, 1, n, d), 6)
+    m = orc.composed_matrix(q, k, grid, window)[0, 0]
+    table = orc.window_partition(*grid, *window)
+    scale = 1 / np.sqrt(d)
+
+    def weights(tokens, query):
+        s = np.array([q[0, 0, query] @ k[0, 0, t] for t in tokens]) * scale
+        e = np.exp(s - s.max())
+        return e / e.sum()
+
+    rng = np.random.default_rng(0)
+    for _ in range(20):
+        c, j, c2, j2 = rng.integers(4), rng.integers(8), rng.integers(4), rng.integers(8)
+        target, source = table[c, j], table[c2, j2]
+        alpha_g = weights(table[:, j], target)[c2]         # hop 2: (c2, j) -> (c, j)
+        alpha_l = weights(table[c2], table[c2, j])[j2]     # hop 1: (c2, j2) -> (c2, j)
+        assert m[target, source] == pytest.approx(alpha_g * alpha_l, rel=1e-12)
+
+
+# ------------------------------------------------------------------------------------------------
+# locality of each pass and independence from the within-window / within-slot orderings
+# ------------------------------------------------------------------------------------------------
+
+def test_pass_locality():
+    grid, window = (3, 4, 6), (3, 2, 3)
+    T, H, W = grid
+    n, d = T * H * W, 8
+    q, k, v = (_rand((1, 1, n, d), s) for s in (7, 8, 9))
+    same_window, same_slot = _masks(T, H, W, 2, 3)
+    for pass_fn, mask in ((orc.local_pass, same_window), (orc.global_pass, same_slot)):
+        base, _ = pass_fn(q, k, v, grid, window)
+        for u in (0, 17, n - 1):
+            v2 = v.copy()
+            v2[0, 0, u] += 1.0
+            moved = np.abs(pass_fn(q, k, v2, grid, window)[0] - base)[0, 0].max(-1) > 0
+            np.testing.assert_array_equal(moved, mask[:, u])
+
+
+@pytest.mark.parametrize("order", ORDERS)
+def test_ordering_conventions_do_not_matter(order):
+    """Relabel slots (same permutation in every window) and windows: the output relabels likewise."""
+    grid, window = (3, 4, 6), (3, 2, 3)
+    n, d = 72, 8
+    q, k, v = (_rand((1, 2, n, d), s) for s in (10, 11, 12))
+    table = orc.window_partition(*grid, *window)
+    rng = np.random.default_rng(1)
+    pj, pc = rng.permutation(table.shape[1]), rng.permutation(table.shape[0])
+    relabel = np.empty(n, dtype=np.int64)
+    relabel[table] = table[pc][:, pj]       # token (c, j) takes the data of token (pc[c], pj[j])
+    out = orc.squad_attn_fwd(q, k, v, grid, window, order)
+    out2 = orc.squad_attn_fwd(q[:, :, relabel], k[:, :, relabel], v[:, :, relabel], grid, window, order)
+    np.testing.assert_allclose(out2, out[:, :, relabel], rtol=0, atol=1e-13)
+
+
+# ------------------------------------------------------------------------------------------------
+# backward: per-sequence against torch autograd; the composed operator against finite differences
+# ------------------------------------------------------------------------------------------------
+
+def test_single_attention_backward_matches_autograd():
+    q, k, v, do = (_rand((3, 20, 16), s) for s in (20, 21, 22, 23))
+    dq, dk, dv = orc.softmax_attention_bwd(q, k, v, do, 0.25)
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+    out = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, scale=0.25)
+    out.backward(torch.from_numpy(do))
+    for mine, ref in ((dq, tq.grad), (dk, tk.grad), (dv, tv.grad)):
+        np.testing.assert_allclose(mine, ref.numpy(), rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("order", ORDERS)
+def test_backward_matches_finite_differences(order):
+    grid, window = (2, 4, 4), (2, 2, 2)
+    n, d = 32, 8
+    q, k, v, do = (_rand((1, 2, n, d), s) for s in (30, 31, 32, 33))
+    grads = orc.squad_attn_bwd(q, k, v, do, grid, window, order)
+
+    def loss(qq, kk, vv):
+        return float((do * orc.squad_attn_fwd(qq, kk, vv, grid, window, order)).sum())
+
+    eps = 1e-6
+    rng = np.random.default_rng(2)
+    for which in range(3):
+        base = [q, k, v]
+        for _ in range(3):  # random directional derivatives
+            u = rng.standard_normal(q.shape)
+            plus = [x + eps * u if i == which else x for i, x in enumerate(base)]
+            minus = [x - eps * u if i == which else x for i, x in enumerate(base)]
+            fd = (loss(*plus) - loss(*minus)) / (2 * eps)
+            an = float((grads[which] * u).sum())
+            assert abs(fd - an) <= 1e-6 * max(1.0, abs(an))
+        gmax = np.abs(grads[which]).max()
+        for _ in range(200 // 3 + 1):  # random coordinates
+            idx = tuple(int(rng.integers(s)) for s in q.shape)
+            plus = [x.copy() for x in base]
+            minus = [x.copy() for x in base]
+            plus[which][idx] += eps
+            minus[which][idx] -= eps
+            fd = (loss(*plus) - loss(*minus)) / (2 * eps)
+            assert abs(fd - grads[which][idx]) <= 1e-6 * gmax
+
+
+# ------------------------------------------------------------------------------------------------
+# (d) the cost model against the pages' printed numbers and against the oracle's own structure
+# ------------------------------------------------------------------------------------------------
+
+def test_flops_match_printed_numbers():
+    with open(os.path.join(GOLDEN, "pages_flop_counts.json")) as f:
+        g = json.load(f)
+    for case in g["cases"]:
+        h, d, n, w = case["h"], case["d"], case["n"], case["w"]
+        squad = orc.squad_flops(1, h, d, n, w) / 1e12
+        full = orc.full_flops(1, h, d, n) / 1e12
+        ndig = len(str(case["squad_tflops"]).split(".")[1])
+        assert round(squad, ndig) == case["squad_tflops"], (case["name"], squad)
+        assert abs(full - case["full_tflops"]) <= g["full_attention_conformance"] * case["full_tflops"] + \
+            0.5 * 10 ** -len(str(case["full_tflops"]).split(".")[1]), (case["name"], full)
+
+
+def test_flops_optimum_is_n_to_the_1p5():
+    """At w = sqrt(n): hd(n w + n^2/w) = 2 h d n^1.5 (agihunt digest) and the 4x FLOP count is 8 h d n^1.5."""
+    h, d, n = 3, 16, 64
+    assert orc.squad_flops(1, h, d, n, 8) == pytest.approx(8 * h * d * n ** 1.5, rel=1e-15)
+    assert orc.squad_flops(1, h, d, n, 8) / 4 == pytest.approx(2 * h * d * n ** 1.5, rel=1e-15)
+    assert orc.full_flops(1, h, d, n) == 4 * h * d * n * n
+
+
+@pytest.mark.parametrize("grid,window", [((21, 22, 40), (21, 2, 4)), ((21, 44, 80), (21, 4, 4)), ((5, 8, 8), (5, 2, 2))])
+def test_flops_equal_the_oracles_gemm_shapes(grid, window):
+    """Counting 2 s^2 d FLOPs per GEMM over the sequences the oracle actually forms gives the closed form."""
+    table = orc.window_partition(*grid, *window)
+    n_seq_l, s_l = table.shape
+    n_seq_g, s_g = table.T.shape
+    d = 128
+    counted = 2 * (n_seq_l * 2 * s_l * s_l * d + n_seq_g * 2 * s_g * s_g * d)
+    n = int(np.prod(grid))
+    assert counted == pytest.approx(orc.squad_flops(1, 1, d, n, s_l), rel=1e-12)
