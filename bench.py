@@ -1,0 +1,338 @@
+"""Benchmark: SQuad-Attention forward on the Wan-2.2-5B-shaped block (one GPU per rank).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one squad_attn_fwd call (local pass then global pass) over one DiT block's attention:
+B=1, h=24, d=128, grid 21x22x40 (n=18480), window 21x2x4 (w=168), bf16, seeded synthetic inputs.
+Prints one JSON line (rank 0). With N > 1 (torchrun), every rank runs an independent replica (the
+operator has no cross-GPU exchange); timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = dict(B=1, h=24, d=128, grid=(21, 22, 40), window=(21, 2, 4), order="local_then_global")
+WORKLOAD_NAME = ("Wan-2.2-5B-shaped SQuad attention block: B=1 h=24 d=128, grid 21x22x40 (n=18480), "
+                 "window 21x2x4 (w=168, 110 windows), local->global, bf16")
+METRIC = "SQuad-attn fwd ms/block & TFLOP/s at n=18480,h=24,d=128 bf16; % of roofline"
+PAGES_MS = 4.27   # pages' SQuad attention latency per block for this workload (1x H100, bf16): context
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 6650.0, 1590.0, "fallback"
+
+
+def n_tokens(w=WORKLOAD):
+    T, H, W = w["grid"]
+    return T * H * W
+
+
+def flops(w=WORKLOAD):
+    n = n_tokens(w)
+    win = w["window"][0] * w["window"][1] * w["window"][2]
+    return 4.0 * w["B"] * w["h"] * w["d"] * (n * win + n * n / win)
+
+
+def alg_bytes(w=WORKLOAD):
+    """Q, K, V read once and O written once (bf16): the roofline's algorithmic traffic of one step."""
+    return 4 * w["B"] * w["h"] * n_tokens(w) * w["d"] * 2
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        import torch
+
+        # nvidia-smi numbers GPUs differently from CUDA under CUDA_VISIBLE_DEVICES: address it by UUID.
+        try:
+            self.dev = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+        except Exception:
+            self.dev = str(device_index)
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.15)
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            time.sleep(0.1)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in (self.out or "").splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, f[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def cpu_baseline(budget_s=12.0):
+    """The fp64 oracle timed on the host cores, on whole heads of the same workload."""
+    import numpy as np
+    from threadpoolctl import threadpool_info
+
+    from oracle import squad_oracle as orc
+    from sub_quadratic_two_squad_b200.inputs import make_inputs
+
+    w = WORKLOAD
+    n = n_tokens(w)
+    x = make_inputs(1, 1, n, w["d"], dtype="bf16", heavy_tail=True)
+    done, t0 = 0, time.perf_counter()
+    while True:
+        orc.squad_attn_fwd(x["q"], x["k"], x["v"], w["grid"], w["window"])
+        done += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or done >= w["h"]:
+            break
+    per_head_flops = flops(dict(w, h=1))
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    return {"value": per_head_flops * done / el / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": f"{done} of 24 heads of the same block (fp64 numpy oracle, {el:.1f} s)",
+            "ms_per_block_extrapolated": el / done * w["h"] * 1e3}
+
+
+def run_reference(args, rank, world):
+    """--impl reference: the fp64 oracle on the host cores, one bounded sample per step."""
+    if rank != 0:
+        return
+    from threadpoolctl import threadpool_info
+
+    from oracle import squad_oracle as orc
+    from sub_quadratic_two_squad_b200.inputs import make_inputs
+
+    w = WORKLOAD
+    n = n_tokens(w)
+    x = make_inputs(1, 1, n, w["d"], dtype="bf16", heavy_tail=True)
+    t0 = time.perf_counter()
+    orc.squad_attn_fwd(x["q"], x["k"], x["v"], w["grid"], w["window"])
+    t_head = time.perf_counter() - t0
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    heads = max(1, min(w["h"], int(budget / max(t_head, 1e-6))))
+    xs = make_inputs(1, heads, n, w["d"], dtype="bf16", heavy_tail=True)
+    for _ in range(args.warmup):
+        orc.squad_attn_fwd(xs["q"], xs["k"], xs["v"], w["grid"], w["window"])
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        orc.squad_attn_fwd(xs["q"], xs["k"], xs["v"], w["grid"], w["window"])
+    el = time.perf_counter() - t0
+    value = flops(dict(w, h=heads)) * args.steps / el / 1e12
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD_NAME, "sample_heads": heads},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                             "sample": f"{heads} of 24 heads per step"},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from sub_quadratic_two_squad_b200 import HostRunner, full_attn_fwd, squad_attn_fwd, squad_attn_fwd_status
+    from sub_quadratic_two_squad_b200.inputs import make_inputs
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = WORKLOAD
+    n = n_tokens(w)
+    shape = (w["B"], w["h"], n, w["d"])
+    x = make_inputs(w["B"], w["h"], n, w["d"], dtype="bf16", heavy_tail=True)
+    host = {k: torch.from_numpy(v).to(torch.bfloat16) for k, v in x.items()}
+    # Rotating buffer sets: each set is 5 x 114 MB (> the 126 MB L2), consecutive steps use different sets.
+    n_sets = 3
+    sets = []
+    for _ in range(n_sets):
+        q, k, v = (host[s].to(dev) for s in "qkv")
+        o = torch.empty(shape, dtype=torch.bfloat16, device=dev)
+        _, ws = squad_attn_fwd(q, k, v, w["grid"], w["window"], w["order"], out=o)
+        sets.append((q, k, v, o, ws))
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        q, k, v, o, ws = sets[i % n_sets]
+        squad_attn_fwd(q, k, v, w["grid"], w["window"], w["order"], out=o, workspace=ws, stream=stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        torch.cuda.synchronize()
+        t_start.record(stream)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            step(i)
+            ev[i][1].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    total_ms = t_start.elapsed_time(t_end)
+    per_launch_ms = [a.elapsed_time(b) for a, b in ev]
+    ms = torch.tensor([total_ms], device=dev)
+    if world > 1:
+        dist.all_reduce(ms, op=dist.ReduceOp.MAX)
+    total_ms = float(ms.item())
+    ms_per_step = total_ms / args.steps
+    status_ok = all(squad_attn_fwd_status(s[4], s[0], w["grid"], w["window"], w["order"]) == 0 for s in sets)
+
+    # End to end through the public API from pinned host buffers (copies inside the timed region).
+    runner = HostRunner(w["B"], w["h"], w["d"], w["grid"], w["window"], w["order"], device=dev)
+    hq, hk, hv = (host[s].pin_memory() for s in "qkv")
+    ho = torch.empty(shape, dtype=torch.bfloat16).pin_memory()
+    e2e_steps = max(3, min(args.steps, 30))
+    for _ in range(2):
+        runner(hq, hk, hv, ho)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(runner.stream)
+    for _ in range(e2e_steps):
+        runner(hq, hk, hv, ho)
+    b.record(runner.stream)
+    torch.cuda.synchronize()
+    e2e_ms = a.elapsed_time(b) / e2e_steps
+    e2 = torch.tensor([e2e_ms], device=dev)
+    if world > 1:
+        dist.all_reduce(e2, op=dist.ReduceOp.MAX)
+    e2e_ms = float(e2.item())
+
+    # Full attention at the same n, beside SQuad (a few calls: ~4.2 TFLOP each).
+    q, k, v, o, _ = sets[0]
+    full_attn_fwd(q, k, v, grid=w["grid"], out=o)
+    torch.cuda.synchronize()
+    fa, fb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = 5
+    fa.record(stream)
+    for _ in range(reps):
+        full_attn_fwd(q, k, v, grid=w["grid"], out=o)
+    fb.record(stream)
+    torch.cuda.synchronize()
+    full_ms = fa.elapsed_time(fb) / reps
+    n_full = 4.0 * w["B"] * w["h"] * w["d"] * n * n
+
+    if rank != 0:
+        return
+    hbm, tf_peak, peak_kind = peaks()
+    f = flops()
+    mean_launch = statistics.mean(per_launch_ms)
+    achieved = alg_bytes() / (mean_launch * 1e-3) / 1e9
+    line = {
+        "metric": METRIC,
+        "value": world * f / (ms_per_step * 1e-3) / 1e12,
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": PAGES_MS / ms_per_step,
+        "vs_baseline_ref": "pages' 4.27 ms per block on 1x H100 80GB bf16 (context, other hardware)",
+        "dtype": "bf16",
+        "data": "synthetic: seeded N(0,1) Q,K,V rounded to bf16, 2% of key tokens x4 per head",
+        "config": {"workload": WORKLOAD_NAME, "global_batch": w["B"], "seq_len": n, "heads": w["h"],
+                   "head_dim": w["d"], "window": "21x2x4", "parallelism": f"replicas x{world}" if world > 1 else "1 gpu",
+                   "l2": f"{n_sets} rotating buffer sets of ~570 MB each (> 126 MB L2); no reuse between steps"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                     "traffic": None, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)",
+                     "kernel": "squad_attn_fwd step (tc_pass_kernel local + global)",
+                     "alg_bytes_per_launch": alg_bytes(), "mean_launch_ms": mean_launch,
+                     "tensor_frac": f / (mean_launch * 1e-3) / 1e12 / tf_peak},
+        "e2e": {"value": world * f / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": runner.h2d_bytes(), "d2h_bytes_per_step": runner.d2h_bytes(),
+                "steps": e2e_steps, "api": "sub_quadratic_two_squad_b200.HostRunner (pinned host buffers)"},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clk.summary(),
+        "device_status_ok": status_ok,
+        "full_attn": {"ms_per_block": full_ms, "tflops": n_full / (full_ms * 1e-3) / 1e12,
+                      "flop_ratio": n_full / f, "latency_ratio": full_ms / ms_per_step},
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline()
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

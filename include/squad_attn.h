@@ -1,0 +1,129 @@
+/*
+ * squad_attn.h -- C ABI of the SQuad-Attention CUDA library (sm_100a, one GPU).
+ *
+ * SQuad-Attention ("SQuad: Sub-Quadratic Attention Distillation for Efficient Video Generation")
+ * replaces full softmax self-attention over a T x H x W latent token grid by two ordinary softmax
+ * attentions run one after the other (paper §3.2; agihunt digest, "SQuad-Attention composes two
+ * ordinary softmax attentions"):
+ *
+ *   local pass  Attn_L: every token attends to the w = tw*hw*ww tokens of its window. A window spans
+ *                       the full temporal extent (tw = T) and an hw x ww block of space (agihunt
+ *                       digest, "The window size carries the whole argument": 21x2x4 = 168).
+ *   global pass Attn_G: the n/w tokens that occupy the same slot (t, y mod hw, x mod ww) in every
+ *                       window attend to one another; the pass-1 output is its value stream (paper
+ *                       appendix "Reachability": the two-hop path (c',j') -> (c',j) -> (c,j)).
+ *
+ * Between the passes there is only re-indexing (paper §4.3); this library never materialises a
+ * permuted copy: both views are strided boxes of the caller's [B, h, n, d] tensors.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Layout:     every tensor is contiguous [B, h, n, d] (d fastest), n = T*H*W tokens ordered
+ *             (t, y, x) row-major: token = (t*H + y)*W + x. LSE buffers are contiguous [B, h, n] fp32.
+ * Dtypes:     SQUAD_BF16: q, k, v, o, dout, dq, dk, dv are bfloat16; accumulation and softmax in
+ *             fp32 (tcgen05 tensor cores). SQUAD_FP32: all of them are float32, computed with fp32
+ *             FMA on the CUDA cores (exact fp32 path).
+ * Pointers:   device pointers, 16-byte aligned, caller-owned. The library allocates no device
+ *             memory; scratch comes from the caller's workspace (size from the *_workspace_bytes
+ *             query). Workspace pointers must be 256-byte aligned.
+ * Streams:    every call is asynchronous on `stream` (0 = legacy default stream); buffers must stay
+ *             valid until the stream reaches the call.
+ * Errors:     argument errors are detected on the host before anything is launched and returned
+ *             synchronously (SQUAD_ERR_INVALID_ARG / SQUAD_ERR_UNSUPPORTED); a failed launch returns
+ *             SQUAD_ERR_CUDA. Device-side waits are bounded: a wait that gives up records
+ *             SQUAD_ERR_TIMEOUT in the workspace status word, which squad_attn_fwd_status() reads.
+ *             No C++ exception crosses this interface.
+ */
+#ifndef SQUAD_ATTN_H
+#define SQUAD_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SQUAD_API __attribute__((visibility("default")))
+#else
+#define SQUAD_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA runtime stream (cudaStream_t); declared opaquely so this header needs no CUDA headers. */
+typedef struct CUstream_st* squad_stream_t;
+
+typedef enum {
+  SQUAD_OK = 0,
+  SQUAD_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad size, n != T*H*W, ...            */
+  SQUAD_ERR_UNSUPPORTED = 2,  /* well-formed but outside what the kernels implement           */
+  SQUAD_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed (launch, tensor map, ...)   */
+  SQUAD_ERR_TIMEOUT = 4       /* a bounded device-side wait gave up (read via *_status)        */
+} squad_status_t;
+
+typedef enum { SQUAD_BF16 = 0, SQUAD_FP32 = 1 } squad_dtype_t;
+
+/* Pass order. LOCAL_THEN_GLOBAL is the paper's chosen order; GLOBAL_THEN_LOCAL the ablated reverse
+ * (paper §4.4 "The need for and the order of the two passes"; appendix "On the ordering"). */
+typedef enum { SQUAD_LOCAL_THEN_GLOBAL = 0, SQUAD_GLOBAL_THEN_LOCAL = 1 } squad_order_t;
+
+typedef struct {
+  int B, h, d;      /* batch, heads, head dim (d in {64, 128}; bf16 tensor-core path: d == 128)  */
+  int T, H, W;      /* latent grid; n = T*H*W                                                     */
+  int tw, hw, ww;   /* window; tw must equal T (the window spans all frames), H % hw == W % ww == 0 */
+  int order;        /* squad_order_t                                                              */
+  int dtype;        /* squad_dtype_t                                                              */
+  float scale;      /* softmax scale; 0 selects 1/sqrt(d) (paper eq. 5)                           */
+} squad_params_t;
+
+/* Bytes of forward workspace: the pass-1 output O1 ([B,h,n,d] in the tensor dtype), both passes'
+ * LSE ([B,h,n] fp32 each) and a small control block. Keep the workspace unchanged between
+ * squad_attn_fwd and squad_attn_bwd: the backward reads O1 and the LSEs from it. Returns 0 for
+ * invalid parameters. */
+SQUAD_API size_t squad_attn_fwd_workspace_bytes(const squad_params_t* p);
+
+/* SQuad-Attention forward: o = pass2(q, k, pass1(q, k, v)) with the passes in `order`.
+ * q, k, v: inputs [B,h,n,d]; o: output [B,h,n,d]; workspace: >= squad_attn_fwd_workspace_bytes. */
+SQUAD_API squad_status_t squad_attn_fwd(const squad_params_t* p, const void* q, const void* k, const void* v,
+                              void* o, void* workspace, squad_stream_t stream);
+
+/* Device status recorded by the last forward/backward call on `workspace`: SQUAD_OK or
+ * SQUAD_ERR_TIMEOUT. Synchronises `stream` first. */
+SQUAD_API squad_status_t squad_attn_fwd_status(const squad_params_t* p, const void* workspace,
+                                     squad_stream_t stream);
+
+/* Bytes of backward workspace: fp32 partial dQ and dK, the fp32 gradient of the pass-1 output, the
+ * per-row softmax-Jacobian terms of each pass, and a control block. Returns 0 for invalid params. */
+SQUAD_API size_t squad_attn_bwd_workspace_bytes(const squad_params_t* p);
+
+/* SQuad-Attention backward (the pages print no formula; it is the chain rule through both passes).
+ * Gradients of <dout, o> with respect to q, k, v. Inputs: q, k, v and o as given to / returned by
+ * squad_attn_fwd, dout [B,h,n,d], and fwd_workspace as left by that forward call. Outputs dq, dk,
+ * dv [B,h,n,d] (overwritten). q and k are used by both passes, so dq and dk sum two terms. */
+SQUAD_API squad_status_t squad_attn_bwd(const squad_params_t* p, const void* q, const void* k, const void* v,
+                              const void* o, const void* dout, const void* fwd_workspace,
+                              void* dq, void* dk, void* dv, void* bwd_workspace,
+                              squad_stream_t stream);
+
+/* Full softmax self-attention softmax(q k^T * scale) v over all n tokens per head (paper eq. 5),
+ * the operator SQuad replaces. The window fields and `order` of *p are ignored (grid still gives n).
+ * lse_or_null: optional [B,h,n] fp32 output of the natural-log log-sum-exp per query. */
+SQUAD_API squad_status_t full_attn_fwd(const squad_params_t* p, const void* q, const void* k, const void* v,
+                             void* o, float* lse_or_null, squad_stream_t stream);
+
+/* FLOPs of one call, from the paper's cost model (appendix "Conformance to the theoretical curves
+ * is quantitative"): 4 B h d (n w + n^2/w) for SQuad, 4 B h d n^2 for full attention. */
+SQUAD_API double squad_attn_flops(const squad_params_t* p);
+SQUAD_API double full_attn_flops(const squad_params_t* p);
+
+/* Static string for a status code (never NULL). */
+SQUAD_API const char* squad_status_string(squad_status_t s);
+
+/* Library ABI version (incremented on any incompatible change of this header). */
+SQUAD_API int squad_attn_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SQUAD_ATTN_H */

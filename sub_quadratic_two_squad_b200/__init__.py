@@ -1,0 +1,18 @@
+"""SQuad-Attention for B200 (sm_100a): a C-ABI CUDA library (include/squad_attn.h) and its binding.
+
+The local pass attends inside windows that span all frames; the global pass attends, per slot,
+across all windows with the local output as values (SQuad paper §3.2, appendix "Reachability").
+"""
+from .api import (  # noqa: F401
+    HostRunner,
+    SquadError,
+    full_attn_flops,
+    full_attn_fwd,
+    make_params,
+    squad_attn_bwd,
+    squad_attn_bwd_workspace_bytes,
+    squad_attn_flops,
+    squad_attn_fwd,
+    squad_attn_fwd_status,
+    squad_attn_fwd_workspace_bytes,
+)

@@ -1,0 +1,54 @@
+"""ctypes view of include/squad_attn.h. Loads the in-tree libsquad_attn.so and fails loudly without it."""
+from __future__ import annotations
+
+import ctypes
+import os
+
+PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG_DIR, "libsquad_attn.so")
+
+SQUAD_OK, SQUAD_ERR_INVALID_ARG, SQUAD_ERR_UNSUPPORTED, SQUAD_ERR_CUDA, SQUAD_ERR_TIMEOUT = range(5)
+SQUAD_BF16, SQUAD_FP32 = 0, 1
+SQUAD_LOCAL_THEN_GLOBAL, SQUAD_GLOBAL_THEN_LOCAL = 0, 1
+
+# Every symbol include/squad_attn.h declares, with (restype, argtypes).
+_VP = ctypes.c_void_p
+
+
+class SquadParams(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("h", ctypes.c_int), ("d", ctypes.c_int),
+                ("T", ctypes.c_int), ("H", ctypes.c_int), ("W", ctypes.c_int),
+                ("tw", ctypes.c_int), ("hw", ctypes.c_int), ("ww", ctypes.c_int),
+                ("order", ctypes.c_int), ("dtype", ctypes.c_int), ("scale", ctypes.c_float)]
+
+
+_PP = ctypes.POINTER(SquadParams)
+SIGNATURES = {
+    "squad_attn_fwd_workspace_bytes": (ctypes.c_size_t, [_PP]),
+    "squad_attn_fwd": (ctypes.c_int, [_PP, _VP, _VP, _VP, _VP, _VP, _VP]),
+    "squad_attn_fwd_status": (ctypes.c_int, [_PP, _VP, _VP]),
+    "squad_attn_bwd_workspace_bytes": (ctypes.c_size_t, [_PP]),
+    "squad_attn_bwd": (ctypes.c_int, [_PP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
+    "full_attn_fwd": (ctypes.c_int, [_PP, _VP, _VP, _VP, _VP, _VP, _VP]),
+    "squad_attn_flops": (ctypes.c_double, [_PP]),
+    "full_attn_flops": (ctypes.c_double, [_PP]),
+    "squad_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "squad_attn_abi_version": (ctypes.c_int, []),
+}
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """The loaded library (built in-tree by ``python -m sub_quadratic_two_squad_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with `python -m sub_quadratic_two_squad_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib

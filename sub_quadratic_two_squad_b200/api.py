@@ -1,0 +1,164 @@
+"""Python binding of the SQuad-Attention C ABI, with the C names.
+
+Argument marshalling only: every step of the computation runs in the CUDA library. Tensors are torch
+CUDA tensors (PyTorch provides device memory and streams); shapes are [B, h, n, d] contiguous with
+n = T*H*W in (t, y, x) row-major order.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _lib
+
+ORDERS = {"local_then_global": _lib.SQUAD_LOCAL_THEN_GLOBAL, "global_then_local": _lib.SQUAD_GLOBAL_THEN_LOCAL}
+_DTYPES = {torch.bfloat16: _lib.SQUAD_BF16, torch.float32: _lib.SQUAD_FP32}
+
+
+class SquadError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        msg = _lib.load().squad_status_string(status).decode()
+        super().__init__(f"{what}: {msg} (status {status})")
+
+
+def make_params(B, h, d, grid, window=(1, 1, 1), order="local_then_global", dtype=torch.bfloat16, scale=None):
+    T, H, W = grid
+    tw, hw, ww = window
+    o = ORDERS[order] if isinstance(order, str) else int(order)
+    dt = _DTYPES[dtype] if isinstance(dtype, torch.dtype) else int(dtype)
+    return _lib.SquadParams(B, h, d, T, H, W, tw, hw, ww, o, dt, 0.0 if scale is None else float(scale))
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check_qkv(*ts):
+    q = ts[0]
+    for t in ts:
+        if not t.is_cuda or not t.is_contiguous() or t.dtype != q.dtype or t.shape != q.shape:
+            raise ValueError("q, k, v (and o, dout) must be contiguous CUDA tensors of one dtype and shape [B,h,n,d]")
+    if q.dim() != 4:
+        raise ValueError("expected [B, h, n, d]")
+
+
+def _params_for(q, grid, window, order, scale):
+    B, h, n, d = q.shape
+    if n != grid[0] * grid[1] * grid[2]:
+        raise ValueError(f"n = {n} but T*H*W = {grid[0] * grid[1] * grid[2]}")
+    return make_params(B, h, d, grid, window, order, q.dtype, scale)
+
+
+def squad_attn_fwd_workspace_bytes(params) -> int:
+    return int(_lib.load().squad_attn_fwd_workspace_bytes(ctypes.byref(params)))
+
+
+def squad_attn_bwd_workspace_bytes(params) -> int:
+    return int(_lib.load().squad_attn_bwd_workspace_bytes(ctypes.byref(params)))
+
+
+def squad_attn_fwd(q, k, v, grid, window, order="local_then_global", scale=None, out=None, workspace=None,
+                   stream=None):
+    """SQuad-Attention forward. Returns (out, workspace); keep the workspace for squad_attn_bwd."""
+    _check_qkv(q, k, v)
+    prm = _params_for(q, grid, window, order, scale)
+    lib = _lib.load()
+    nbytes = lib.squad_attn_fwd_workspace_bytes(ctypes.byref(prm))
+    if nbytes == 0:
+        raise SquadError(_lib.SQUAD_ERR_INVALID_ARG, "squad_attn_fwd_workspace_bytes")
+    out = torch.empty_like(q) if out is None else out
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    elif workspace.numel() * workspace.element_size() < nbytes:
+        raise ValueError(f"workspace needs {nbytes} bytes")
+    st = lib.squad_attn_fwd(ctypes.byref(prm), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(workspace), _stream(stream))
+    if st != _lib.SQUAD_OK:
+        raise SquadError(st, "squad_attn_fwd")
+    return out, workspace
+
+
+def squad_attn_fwd_status(workspace, q, grid, window, order="local_then_global", scale=None, stream=None) -> int:
+    """Device status of the last call on `workspace` (synchronises the stream): 0 ok, 4 timeout."""
+    prm = _params_for(q, grid, window, order, scale)
+    return int(_lib.load().squad_attn_fwd_status(ctypes.byref(prm), _ptr(workspace), _stream(stream)))
+
+
+def squad_attn_bwd(q, k, v, o, dout, fwd_workspace, grid, window, order="local_then_global", scale=None,
+                   dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """Gradients (dq, dk, dv) of <dout, o>; `fwd_workspace` as left by squad_attn_fwd."""
+    _check_qkv(q, k, v, o, dout)
+    prm = _params_for(q, grid, window, order, scale)
+    lib = _lib.load()
+    nbytes = lib.squad_attn_bwd_workspace_bytes(ctypes.byref(prm))
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    st = lib.squad_attn_bwd(ctypes.byref(prm), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(fwd_workspace),
+                            _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace), _stream(stream))
+    if st != _lib.SQUAD_OK:
+        raise SquadError(st, "squad_attn_bwd")
+    return dq, dk, dv
+
+
+def full_attn_fwd(q, k, v, grid=None, scale=None, out=None, lse=None, stream=None):
+    """softmax(q k^T * scale) v over all n tokens per head. Returns out (and fills `lse` if given)."""
+    _check_qkv(q, k, v)
+    B, h, n, d = q.shape
+    grid = (1, 1, n) if grid is None else grid
+    prm = _params_for(q, grid, (1, 1, 1), "local_then_global", scale)
+    out = torch.empty_like(q) if out is None else out
+    st = _lib.load().full_attn_fwd(ctypes.byref(prm), _ptr(q), _ptr(k), _ptr(v), _ptr(out),
+                                   _ptr(lse), _stream(stream))
+    if st != _lib.SQUAD_OK:
+        raise SquadError(st, "full_attn_fwd")
+    return out
+
+
+def squad_attn_flops(B, h, d, grid, window) -> float:
+    return float(_lib.load().squad_attn_flops(ctypes.byref(make_params(B, h, d, grid, window))))
+
+
+def full_attn_flops(B, h, d, grid) -> float:
+    return float(_lib.load().full_attn_flops(ctypes.byref(make_params(B, h, d, grid))))
+
+
+class HostRunner:
+    """End-to-end forward from host buffers: pinned host -> device copies, squad_attn_fwd, device -> host.
+
+    Device buffers are allocated once; every call() copies the inputs in and the output back on the
+    runner's stream, so the copies are part of what a caller holding host data pays.
+    """
+
+    def __init__(self, B, h, d, grid, window, order="local_then_global", dtype=torch.bfloat16, device="cuda"):
+        n = grid[0] * grid[1] * grid[2]
+        self.shape = (B, h, n, d)
+        self.grid, self.window, self.order = grid, window, order
+        self.dev = [torch.empty(self.shape, dtype=dtype, device=device) for _ in range(4)]
+        prm = make_params(B, h, d, grid, window, order, dtype)
+        self.ws = torch.empty(squad_attn_fwd_workspace_bytes(prm), dtype=torch.uint8, device=device)
+        self.stream = torch.cuda.Stream(device=device)
+
+    def h2d_bytes(self):
+        return 3 * self.dev[0].numel() * self.dev[0].element_size()
+
+    def d2h_bytes(self):
+        return self.dev[3].numel() * self.dev[3].element_size()
+
+    def __call__(self, q_host, k_host, v_host, o_host):
+        q, k, v, o = self.dev
+        with torch.cuda.stream(self.stream):
+            q.copy_(q_host, non_blocking=True)
+            k.copy_(k_host, non_blocking=True)
+            v.copy_(v_host, non_blocking=True)
+            squad_attn_fwd(q, k, v, self.grid, self.window, self.order, out=o, workspace=self.ws, stream=self.stream)
+            o_host.copy_(o, non_blocking=True)
+        return o_host

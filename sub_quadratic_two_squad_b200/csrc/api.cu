@@ -1,0 +1,391 @@
+// C ABI of the SQuad-Attention library (include/squad_attn.h): argument validation, TMA tensor maps
+// for the window and slot views, and the launch sequence of the two passes.
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include "squad_attn.h"
+#include "geometry.cuh"
+#include "simt_pass.h"
+#include "tc_pass.h"
+
+using namespace squad;
+
+namespace {
+
+constexpr int kAbiVersion = 1;
+constexpr size_t kCtrlBytes = 256;               // status word + reserved
+constexpr unsigned long long kWaitTimeoutNs = 1000000000ull;   // 1 s per device-side wait
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+bool aligned(const void* p, size_t a) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Validates the parameters and fills the grid description. `windowed` = SQuad call (window fields
+// and order are used); false = full attention (only B, h, d, T, H, W, dtype, scale).
+squad_status_t validate(const squad_params_t* p, bool windowed, Grid* g, float* scale) {
+  if (p == nullptr) return SQUAD_ERR_INVALID_ARG;
+  if (p->B < 1 || p->h < 1 || p->T < 1 || p->H < 1 || p->W < 1) return SQUAD_ERR_INVALID_ARG;
+  if (p->dtype != SQUAD_BF16 && p->dtype != SQUAD_FP32) return SQUAD_ERR_INVALID_ARG;
+  if (p->d < 1) return SQUAD_ERR_INVALID_ARG;
+  if (p->d != 64 && p->d != 128) return SQUAD_ERR_UNSUPPORTED;
+  if (!(p->scale >= 0.f) || !std::isfinite(p->scale)) return SQUAD_ERR_INVALID_ARG;
+  const long long n = static_cast<long long>(p->T) * p->H * p->W;
+  if (n > (1ll << 30)) return SQUAD_ERR_UNSUPPORTED;
+  const long long bhn = static_cast<long long>(p->B) * p->h * n;
+  if (bhn > (1ll << 31) - 1) return SQUAD_ERR_UNSUPPORTED;
+  Grid gg{};
+  gg.B = p->B;
+  gg.h = p->h;
+  gg.d = p->d;
+  gg.T = p->T;
+  gg.H = p->H;
+  gg.W = p->W;
+  gg.n = static_cast<int>(n);
+  if (windowed) {
+    if (p->order != SQUAD_LOCAL_THEN_GLOBAL && p->order != SQUAD_GLOBAL_THEN_LOCAL) return SQUAD_ERR_INVALID_ARG;
+    if (p->tw < 1 || p->hw < 1 || p->ww < 1) return SQUAD_ERR_INVALID_ARG;
+    if (p->tw > p->T || p->hw > p->H || p->ww > p->W) return SQUAD_ERR_INVALID_ARG;
+    // The window spans the full temporal extent and tiles space exactly; other windows (tw < T,
+    // grids that need reflect padding) are outside what this library implements.
+    if (p->tw != p->T) return SQUAD_ERR_UNSUPPORTED;
+    if (p->H % p->hw != 0 || p->W % p->ww != 0) return SQUAD_ERR_UNSUPPORTED;
+    gg.hw = p->hw;
+    gg.ww = p->ww;
+    gg.nwy = p->H / p->hw;
+    gg.nwx = p->W / p->ww;
+  } else {
+    gg.hw = 1;
+    gg.ww = 1;
+    gg.nwy = p->H;
+    gg.nwx = p->W;
+  }
+  *g = gg;
+  *scale = p->scale > 0.f ? p->scale : 1.0f / std::sqrt(static_cast<float>(p->d));
+  return SQUAD_OK;
+}
+
+size_t elem_bytes(const squad_params_t* p) { return p->dtype == SQUAD_BF16 ? 2 : 4; }
+
+struct FwdWorkspace {
+  uint32_t* status;
+  void* o1;
+  float* lse1;
+  float* lse2;
+};
+
+size_t fwd_ws_bytes(const Grid& g, size_t eb) {
+  const size_t bhn = static_cast<size_t>(g.B) * g.h * g.n;
+  return kCtrlBytes + align256(bhn * g.d * eb) + 2 * align256(bhn * 4);
+}
+
+FwdWorkspace carve_fwd(void* ws, const Grid& g, size_t eb) {
+  uint8_t* b = static_cast<uint8_t*>(ws);
+  const size_t bhn = static_cast<size_t>(g.B) * g.h * g.n;
+  FwdWorkspace w;
+  w.status = reinterpret_cast<uint32_t*>(b);
+  b += kCtrlBytes;
+  w.o1 = b;
+  b += align256(bhn * g.d * eb);
+  w.lse1 = reinterpret_cast<float*>(b);
+  b += align256(bhn * 4);
+  w.lse2 = reinterpret_cast<float*>(b);
+  return w;
+}
+
+struct BwdWorkspace {
+  uint32_t* status;
+  float* dq_acc;
+  float* dk_acc;
+  float* do1;
+  float* drow;
+};
+
+size_t bwd_ws_bytes(const Grid& g) {
+  const size_t bhn = static_cast<size_t>(g.B) * g.h * g.n;
+  return kCtrlBytes + 3 * align256(bhn * g.d * 4) + align256(bhn * 4);
+}
+
+BwdWorkspace carve_bwd(void* ws, const Grid& g) {
+  uint8_t* b = static_cast<uint8_t*>(ws);
+  const size_t bhn = static_cast<size_t>(g.B) * g.h * g.n;
+  BwdWorkspace w;
+  w.status = reinterpret_cast<uint32_t*>(b);
+  b += kCtrlBytes;
+  w.dq_acc = reinterpret_cast<float*>(b);
+  b += align256(bhn * g.d * 4);
+  w.dk_acc = reinterpret_cast<float*>(b);
+  b += align256(bhn * g.d * 4);
+  w.do1 = reinterpret_cast<float*>(b);
+  b += align256(bhn * g.d * 4);
+  w.drow = reinterpret_cast<float*>(b);
+  return w;
+}
+
+// ------------------------------------------------------------------------------------------------
+// TMA tensor maps: each pass's sequences are boxes of the caller's [B, h, n, d] tensor
+// ------------------------------------------------------------------------------------------------
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// Slot-box encoding for the GLOBAL pass. 0: element-strided box over the natural view (the slot's
+// tokens are every ww-th x and every hw-th y). 1: a view with dims (d, wx, wy, dx, (bh*T+t)*H+dy)
+// whose box has unit strides. Both describe the same tokens.
+int slot_box_variant() {
+  static int v = [] {
+    const char* e = std::getenv("SQUAD_SLOT_BOX");
+    return (e != nullptr && e[0] == '1') ? 1 : 0;
+  }();
+  return v;
+}
+
+bool encode_pass_map(CUtensorMap* m, const void* base, const Grid& g, const PassGeom& p, int variant) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  const MapDesc d = describe_pass_map(g, p, variant, 2);
+  for (int i = 0; i < 5; ++i)
+    if (d.box[i] < 1 || d.box[i] > 256 || d.es[i] < 1 || d.es[i] > 8) return false;
+  cuuint64_t dims[5], strides[4];
+  cuuint32_t box[5], es[5];
+  for (int i = 0; i < 5; ++i) {
+    dims[i] = d.dims[i];
+    box[i] = d.box[i];
+    es[i] = d.es[i];
+  }
+  for (int i = 0; i < 4; ++i) strides[i] = d.strides[i];
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, es,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// The tensor-core kernel handles bf16, d = 128, and chunks of whole lines of at most 128 rows.
+bool tc_eligible(const squad_params_t* prm, const Grid& g, const PassGeom& p) {
+  if (prm->dtype != SQUAD_BF16 || g.d != 128) return false;
+  if (p.line_len > 128 || p.chunk_rows < 1 || p.chunk_rows > 128) return false;
+  if (p.kind == kGlobal && (g.W > 256 || p.lines_per_chunk * g.hw > 256)) return false;
+  return true;
+}
+
+int num_sms_current() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  static int cache[64] = {0};
+  if (dev >= 0 && dev < 64 && cache[dev] > 0) return cache[dev];
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  if (dev >= 0 && dev < 64) cache[dev] = sms;
+  return sms;
+}
+
+// One attention pass: out = softmax(scale q k^T) v over the sequences of `kind`.
+squad_status_t run_pass(const squad_params_t* prm, const Grid& g, int kind, float scale, const void* q,
+                        const void* k, const void* v, bool v_bf16, void* out, float* lse, uint32_t* status,
+                        cudaStream_t stream) {
+  const PassGeom p = make_geom(g, kind);
+  if (tc_eligible(prm, g, p) && v_bf16) {
+    TcPassArgs a;
+    std::memset(&a, 0, sizeof(a));
+    const int variant = kind == kGlobal ? slot_box_variant() : 0;
+    if (!encode_pass_map(&a.tm_q, q, g, p, variant) || !encode_pass_map(&a.tm_k, k, g, p, variant) ||
+        !encode_pass_map(&a.tm_v, v, g, p, variant))
+      return SQUAD_ERR_CUDA;
+    a.g = g;
+    a.p = p;
+    a.global_variant = variant;
+    a.out = static_cast<__nv_bfloat16*>(out);
+    a.lse = lse;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    a.status = status;
+    a.timeout_ns = kWaitTimeoutNs;
+    const int sms = num_sms_current();
+    if (sms <= 0) return SQUAD_ERR_CUDA;
+    return launch_tc_pass(a, sms, stream) == cudaSuccess ? SQUAD_OK : SQUAD_ERR_CUDA;
+  }
+  SimtFwdArgs a;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.out = out;
+  a.lse = lse;
+  a.g = g;
+  a.p = p;
+  a.scale = scale;
+  a.in_bf16 = prm->dtype == SQUAD_BF16;
+  a.v_bf16 = v_bf16;
+  a.out_bf16 = prm->dtype == SQUAD_BF16;
+  return launch_simt_fwd(a, stream) == cudaSuccess ? SQUAD_OK : SQUAD_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int squad_attn_abi_version(void) { return kAbiVersion; }
+
+const char* squad_status_string(squad_status_t s) {
+  switch (s) {
+    case SQUAD_OK: return "ok";
+    case SQUAD_ERR_INVALID_ARG: return "invalid argument";
+    case SQUAD_ERR_UNSUPPORTED: return "unsupported configuration";
+    case SQUAD_ERR_CUDA: return "CUDA error";
+    case SQUAD_ERR_TIMEOUT: return "device-side wait timed out";
+  }
+  return "unknown status";
+}
+
+double squad_attn_flops(const squad_params_t* p) {
+  Grid g;
+  float sc;
+  if (validate(p, true, &g, &sc) != SQUAD_OK) return 0.0;
+  const double w = static_cast<double>(p->tw) * p->hw * p->ww;
+  const double n = g.n;
+  return 4.0 * p->B * p->h * p->d * (n * w + n * n / w);
+}
+
+double full_attn_flops(const squad_params_t* p) {
+  Grid g;
+  float sc;
+  if (validate(p, false, &g, &sc) != SQUAD_OK) return 0.0;
+  const double n = g.n;
+  return 4.0 * p->B * p->h * p->d * n * n;
+}
+
+size_t squad_attn_fwd_workspace_bytes(const squad_params_t* p) {
+  Grid g;
+  float sc;
+  if (validate(p, true, &g, &sc) != SQUAD_OK) return 0;
+  return fwd_ws_bytes(g, elem_bytes(p));
+}
+
+size_t squad_attn_bwd_workspace_bytes(const squad_params_t* p) {
+  Grid g;
+  float sc;
+  if (validate(p, true, &g, &sc) != SQUAD_OK) return 0;
+  return bwd_ws_bytes(g);
+}
+
+squad_status_t squad_attn_fwd(const squad_params_t* p, const void* q, const void* k, const void* v, void* o,
+                              void* workspace, squad_stream_t stream_) {
+  Grid g;
+  float scale;
+  squad_status_t st = validate(p, true, &g, &scale);
+  if (st != SQUAD_OK) return st;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(workspace, 256))
+    return SQUAD_ERR_INVALID_ARG;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  const size_t eb = elem_bytes(p);
+  FwdWorkspace ws = carve_fwd(workspace, g, eb);
+  if (cudaMemsetAsync(ws.status, 0, kCtrlBytes, stream) != cudaSuccess) return SQUAD_ERR_CUDA;
+  const bool bf16 = p->dtype == SQUAD_BF16;
+  const int first = p->order == SQUAD_LOCAL_THEN_GLOBAL ? kLocal : kGlobal;
+  const int second = p->order == SQUAD_LOCAL_THEN_GLOBAL ? kGlobal : kLocal;
+  st = run_pass(p, g, first, scale, q, k, v, bf16, ws.o1, ws.lse1, ws.status, stream);
+  if (st != SQUAD_OK) return st;
+  return run_pass(p, g, second, scale, q, k, ws.o1, bf16, o, ws.lse2, ws.status, stream);
+}
+
+squad_status_t squad_attn_fwd_status(const squad_params_t* p, const void* workspace, squad_stream_t stream_) {
+  Grid g;
+  float scale;
+  squad_status_t st = validate(p, true, &g, &scale);
+  if (st != SQUAD_OK) return st;
+  if (!aligned(workspace, 256)) return SQUAD_ERR_INVALID_ARG;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  uint32_t word = 0;
+  if (cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+    return SQUAD_ERR_CUDA;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return SQUAD_ERR_CUDA;
+  return word == 0 ? SQUAD_OK : SQUAD_ERR_TIMEOUT;
+}
+
+squad_status_t squad_attn_bwd(const squad_params_t* p, const void* q, const void* k, const void* v, const void* o,
+                              const void* dout, const void* fwd_workspace, void* dq, void* dk, void* dv,
+                              void* bwd_workspace, squad_stream_t stream_) {
+  Grid g;
+  float scale;
+  squad_status_t st = validate(p, true, &g, &scale);
+  if (st != SQUAD_OK) return st;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(dout, 16) ||
+      !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(fwd_workspace, 256) ||
+      !aligned(bwd_workspace, 256))
+    return SQUAD_ERR_INVALID_ARG;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  const size_t eb = elem_bytes(p);
+  const bool bf16 = p->dtype == SQUAD_BF16;
+  FwdWorkspace fw = carve_fwd(const_cast<void*>(fwd_workspace), g, eb);
+  BwdWorkspace bw = carve_bwd(bwd_workspace, g);
+  if (cudaMemsetAsync(bw.status, 0, kCtrlBytes, stream) != cudaSuccess) return SQUAD_ERR_CUDA;
+  const int first = p->order == SQUAD_LOCAL_THEN_GLOBAL ? kLocal : kGlobal;
+  const int second = p->order == SQUAD_LOCAL_THEN_GLOBAL ? kGlobal : kLocal;
+
+  // Pass 2 backward: values = O1 (pass-1 output), upstream = dout. Gives dQ, dK shares and dO1.
+  SimtBwdArgs a{};
+  a.q = q;
+  a.k = k;
+  a.v = fw.o1;
+  a.dout = dout;
+  a.lse = fw.lse2;
+  a.Drow = bw.drow;
+  a.dq_acc = bw.dq_acc;
+  a.dk_acc = bw.dk_acc;
+  a.dq_out = dq;
+  a.dk_out = dk;
+  a.dv_out = bw.do1;
+  a.g = g;
+  a.p = make_geom(g, second);
+  a.scale = scale;
+  a.in_bf16 = bf16;
+  a.v_bf16 = bf16;
+  a.dout_bf16 = bf16;
+  a.grad_bf16 = bf16;
+  a.dv_bf16 = 0;
+  a.accumulate = 0;
+  a.final_out = 0;
+  if (launch_simt_bwd(a, stream) != cudaSuccess) return SQUAD_ERR_CUDA;
+
+  // Pass 1 backward: values = v, upstream = dO1. Adds its dQ, dK shares and gives dV.
+  a.v = v;
+  a.dout = bw.do1;
+  a.lse = fw.lse1;
+  a.dv_out = dv;
+  a.p = make_geom(g, first);
+  a.dout_bf16 = 0;
+  a.dv_bf16 = bf16;
+  a.accumulate = 1;
+  a.final_out = 1;
+  if (launch_simt_bwd(a, stream) != cudaSuccess) return SQUAD_ERR_CUDA;
+  return SQUAD_OK;
+}
+
+squad_status_t full_attn_fwd(const squad_params_t* p, const void* q, const void* k, const void* v, void* o,
+                             float* lse_or_null, squad_stream_t stream_) {
+  Grid g;
+  float scale;
+  squad_status_t st = validate(p, false, &g, &scale);
+  if (st != SQUAD_OK) return st;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16)) return SQUAD_ERR_INVALID_ARG;
+  if (lse_or_null != nullptr && !aligned(lse_or_null, 4)) return SQUAD_ERR_INVALID_ARG;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  const bool bf16 = p->dtype == SQUAD_BF16;
+  return run_pass(p, g, kFull, scale, q, k, v, bf16, o, lse_or_null, nullptr, stream);
+}
+
+}  // extern "C"

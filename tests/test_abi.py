@@ -1,0 +1,110 @@
+"""The C-ABI library without a GPU: it loads, exports every symbol include/squad_attn.h declares, and
+rejects bad arguments on the host before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from oracle import squad_oracle as orc
+from sub_quadratic_two_squad_b200 import _lib, make_params
+from sub_quadratic_two_squad_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return _lib.load()
+
+
+def declared_symbols():
+    names = set()
+    for f in os.listdir(os.path.join(ROOT, "include")):
+        if f.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", f)).read()
+            names |= set(re.findall(r"^SQUAD_API[^;(]*?(\w+)\s*\(", text, flags=re.M))
+    return names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_symbols()
+    assert {"squad_attn_fwd", "squad_attn_bwd", "full_attn_fwd"} <= names
+    for name in names:
+        assert hasattr(lib, name), name
+    assert set(_lib.SIGNATURES) == names
+
+
+def test_status_strings(lib):
+    for s in range(5):
+        assert lib.squad_status_string(s)
+    assert lib.squad_status_string(99) == b"unknown status"
+    assert lib.squad_attn_abi_version() >= 1
+
+
+P5B = dict(B=1, h=24, d=128, grid=(21, 22, 40), window=(21, 2, 4))
+
+
+def _p(**kw):
+    a = dict(P5B)
+    a.update(kw)
+    return make_params(a["B"], a["h"], a["d"], a["grid"], a["window"], a.get("order", "local_then_global"),
+                       a.get("dtype", 0), a.get("scale"))
+
+
+def _fwd(lib, prm, ptr=16):
+    p = ctypes.c_void_p(ptr)
+    return lib.squad_attn_fwd(ctypes.byref(prm), p, p, p, p, ctypes.c_void_p(ptr * 16), None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(window=(20, 2, 4)), _lib.SQUAD_ERR_UNSUPPORTED),      # window must span all frames
+    (dict(window=(21, 3, 4)), _lib.SQUAD_ERR_UNSUPPORTED),      # H % hw != 0 (would need reflect padding)
+    (dict(window=(21, 2, 3)), _lib.SQUAD_ERR_UNSUPPORTED),      # W % ww != 0
+    (dict(window=(21, 0, 4)), _lib.SQUAD_ERR_INVALID_ARG),
+    (dict(window=(22, 2, 4)), _lib.SQUAD_ERR_INVALID_ARG),      # larger than the grid
+    (dict(d=96), _lib.SQUAD_ERR_UNSUPPORTED),
+    (dict(d=0), _lib.SQUAD_ERR_INVALID_ARG),
+    (dict(B=0), _lib.SQUAD_ERR_INVALID_ARG),
+    (dict(order=7), _lib.SQUAD_ERR_INVALID_ARG),
+    (dict(dtype=5), _lib.SQUAD_ERR_INVALID_ARG),
+    (dict(scale=-1.0), _lib.SQUAD_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), _lib.SQUAD_ERR_INVALID_ARG),
+])
+def test_bad_params_rejected_before_launch(lib, kw, status):
+    assert _fwd(lib, _p(**kw)) == status
+    assert lib.squad_attn_fwd_workspace_bytes(ctypes.byref(_p(**kw))) == 0
+
+
+def test_bad_pointers_rejected(lib):
+    prm = _p()
+    assert lib.squad_attn_fwd(ctypes.byref(prm), None, None, None, None, None, None) == _lib.SQUAD_ERR_INVALID_ARG
+    assert _fwd(lib, prm, ptr=8) == _lib.SQUAD_ERR_INVALID_ARG           # 16-byte alignment
+    p16 = ctypes.c_void_p(16)
+    assert lib.squad_attn_fwd(ctypes.byref(prm), p16, p16, p16, p16, ctypes.c_void_p(128), None) == \
+        _lib.SQUAD_ERR_INVALID_ARG                                          # workspace 256-byte alignment
+    assert lib.full_attn_fwd(ctypes.byref(prm), None, p16, p16, p16, None, None) == _lib.SQUAD_ERR_INVALID_ARG
+    args = [p16] * 5 + [ctypes.c_void_p(256)] + [p16] * 3 + [ctypes.c_void_p(256), None]
+    args[4] = None
+    assert lib.squad_attn_bwd(ctypes.byref(prm), *args) == _lib.SQUAD_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("cfg", [
+    (1, 24, 128, (21, 22, 40), (21, 2, 4)), (1, 12, 128, (21, 30, 52), (21, 2, 4)),
+    (1, 24, 128, (21, 44, 80), (21, 4, 4)), (1, 4, 64, (5, 8, 8), (5, 2, 2))])
+def test_flops_match_the_oracle_cost_model(lib, cfg):
+    B, h, d, grid, window = cfg
+    prm = make_params(B, h, d, grid, window)
+    n, w = grid[0] * grid[1] * grid[2], window[0] * window[1] * window[2]
+    assert lib.squad_attn_flops(ctypes.byref(prm)) == pytest.approx(orc.squad_flops(B, h, d, n, w), rel=1e-12)
+    assert lib.full_attn_flops(ctypes.byref(prm)) == pytest.approx(orc.full_flops(B, h, d, n), rel=1e-12)
+
+
+def test_workspace_sizes(lib):
+    prm = _p()
+    n = 21 * 22 * 40
+    fwd = lib.squad_attn_fwd_workspace_bytes(ctypes.byref(prm))
+    assert fwd >= 24 * n * 128 * 2 + 2 * 24 * n * 4
+    bwd = lib.squad_attn_bwd_workspace_bytes(ctypes.byref(prm))
+    assert bwd >= 3 * 24 * n * 128 * 4 + 24 * n * 4
