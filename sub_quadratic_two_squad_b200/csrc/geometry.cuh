@@ -65,9 +65,10 @@ __host__ __device__ inline PassGeom make_geom(const Grid& g, int kind) {
   return p;
 }
 
-// Token index (within one (b, head)) of row `r` of chunk `q` of sequence `sigma`; -1 when the row lies
-// past the end of the sequence.
+// Token index (within one (b, head)) of row `r` (0..127) of chunk `q` of sequence `sigma`; -1 when the
+// row is padding: past the chunk's box, or past the end of the sequence.
 __host__ __device__ inline int token_of(const Grid& g, const PassGeom& p, int sigma, int q, int r) {
+  if (r >= p.chunk_rows) return -1;
   const int line = q * p.lines_per_chunk + r / p.line_len;
   if (line >= p.n_lines) return -1;
   const int pos = r - (r / p.line_len) * p.line_len;

@@ -67,6 +67,12 @@ static int check_pass(const Grid& g, int kind, int variant, bool print) {
                 ++seen[static_cast<size_t>(bh) * g.n + got];
                 if (print && bh == 0) std::printf(" %lld", got);
               }
+        // Tile rows past the box (the kernel's 128-row tiles) are padding and must map to no token.
+        for (int r = p.chunk_rows; r < 128; ++r)
+          if (token_of(g, p, sigma, q, r) != -1) {
+            ++errors;
+            if (errors < 10) std::printf("tile row %d past the box maps to a token (kind %d q %d)\n", r, kind, q);
+          }
       }
       if (print && bh == 0) std::printf("\n");
     }
