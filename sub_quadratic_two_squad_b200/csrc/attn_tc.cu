@@ -5,15 +5,19 @@
 // caller's [B, h, n, d] tensors through TMA boxes (geometry.cuh): no permuted copy is made.
 //
 // CTA organisation (persistent, one CTA per SM, 384 threads):
-//   warp 0      TMA producer: Q tiles and a 3-stage ring of K/V blocks (128 keys x 128 dims, bf16).
-//   warp 1      TMEM allocator and MMA issuer (one thread): S = Q K^T and O += P V as tcgen05.mma.
+//   warp 0      TMA producer: double-buffered Q tiles per warpgroup and a 3-stage ring of K/V blocks
+//               (128 keys x 128 dims, bf16, 128-byte swizzle).
+//   warp 1      TMEM allocator and MMA issuer (one thread).
 //   warps 4-7   softmax warpgroup 0 (TMEM lanes 0-127 of S0 / O0)
 //   warps 8-11  softmax warpgroup 1 (S1 / O1).
-// A work unit is a pair of 128-row query tiles, one per softmax warpgroup. When both tiles belong to
-// the same sequence they share every K/V block. Scores S (128 fp32 columns) and the output
-// accumulator O (128 columns) of each warpgroup live in tensor memory; P goes to shared memory as
-// bf16 in the 128-byte-swizzled K-major layout that the MMA reads. Softmax is online across K/V
-// blocks, with the rescale of O skipped unless the row maximum grew by more than 2^8.
+// A work unit is a pair of 128-row query tiles, one per softmax warpgroup; when both belong to the
+// same sequence they share every K/V block. Per warpgroup, tensor memory holds the scores S (128 fp32
+// columns) and the output accumulator O (128 columns). The softmax writes P as bf16 over the first
+// half of S, and the PV product reads it from there (tcgen05.mma with A in tensor memory), so the
+// MMA issue order per warpgroup is ... S(b), [softmax], PV(b), S(b+1) ... and the in-order tensor
+// pipe finishes reading P(b) before S(b+1) overwrites it. Softmax is online across K/V blocks; the
+// rescale of O is skipped unless the row maximum grew by more than 2^8. The epilogue stages O through
+// the tile's own Q buffer (free once its last S is done) and writes it with coalesced stores.
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
@@ -29,16 +33,15 @@ constexpr int kThreads = 384;
 constexpr int kStages = 3;
 constexpr uint32_t kPanel = 16384;   // 128 rows x 128 bytes (64 bf16)
 constexpr uint32_t kTile = 2 * kPanel;
-constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffP = 2 * kTile;
-constexpr uint32_t kOffKV = 4 * kTile;
+constexpr uint32_t kOffQ = 0;                      // Q[wg][slot]: 4 tiles
+constexpr uint32_t kOffKV = 4 * kTile;             // K/V ring
 constexpr uint32_t kOffBar = kOffKV + kStages * kTile;
 constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;   // + barriers + alignment slack
 
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 struct Bars {
-  uint64_t q_full[2], q_empty[2];
+  uint64_t q_full[2][2], q_empty[2][2];
   uint64_t kv_full[kStages], kv_empty[kStages];
   uint64_t s_full[2], p_full[2], o_full[2];
   uint64_t drain;
@@ -69,13 +72,17 @@ __device__ __forceinline__ uint32_t sw_off(int row, int ch) {
   return (ch >> 3) * kPanel + row * 128 + (((ch & 7) ^ (row & 7)) << 4);
 }
 
+// Order of the K/V block loads of one unit (the producer issues them in this order, the MMA issuer
+// finds each one's ring position from it): K0, K1, V0, K2, V1, ..., K(nb-1), V(nb-2), V(nb-1).
+__device__ __forceinline__ int pos_k(int b) { return b == 0 ? 0 : 2 * b - 1; }
+__device__ __forceinline__ int pos_v(int b, int nb) { return b == nb - 1 ? 2 * nb - 1 : 2 * b + 2; }
+
 }  // namespace
 
 __global__ void __launch_bounds__(kThreads, 1) tc_pass_kernel(const __grid_constant__ TcPassArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem + kOffQ;
-  uint8_t* sP = smem + kOffP;
   uint8_t* sKV = smem + kOffKV;
   Bars* bars = reinterpret_cast<Bars*>(smem + kOffBar);
 
@@ -89,8 +96,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pass_kernel(const __grid_const
     reinterpret_cast<uint4*>(sKV)[i] = make_uint4(0, 0, 0, 0);
   if (threadIdx.x == 0) {
     for (int w = 0; w < 2; ++w) {
-      mbar_init(&bars->q_full[w], 1);
-      mbar_init(&bars->q_empty[w], 1);
+      for (int sl = 0; sl < 2; ++sl) {
+        mbar_init(&bars->q_full[w][sl], 1);
+        mbar_init(&bars->q_empty[w][sl], 4);   // one arrival per warp of the warpgroup
+      }
       mbar_init(&bars->s_full[w], 1);
       mbar_init(&bars->p_full[w], 128);
       mbar_init(&bars->o_full[w], 1);
@@ -128,22 +137,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pass_kernel(const __grid_const
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      uint32_t q_loads[2] = {0, 0};
+      uint32_t q_loads[2][2] = {{0, 0}, {0, 0}};
       uint32_t kv_loads = 0;
       bool ok = true;
-      auto load_kv = [&](const CUtensorMap* m, const TileRef& t, int chunk) -> bool {
-        const uint32_t s = kv_loads % kStages;
-        if (kv_loads >= kStages && !mbar_wait(&bars->kv_empty[s], ((kv_loads / kStages) + 1) & 1, ctl)) return false;
-        mbar_arrive_expect_tx(&bars->kv_full[s], box_bytes);
-        for (int panel = 0; panel < 2; ++panel) {
-          int c[5];
-          chunk_coords(a.g, a.p, a.global_variant, t.bh, t.sigma, chunk, panel, c);
-          tma_load_5d(sKV + s * kTile + panel * kPanel, m, &bars->kv_full[s], c[0], c[1], c[2], c[3], c[4]);
-        }
-        ++kv_loads;
-        return true;
-      };
-      for (int unit = blockIdx.x; unit < n_units && ok; unit += gridDim.x) {
+      int u_local = 0;
+      for (int unit = blockIdx.x; unit < n_units && ok; unit += gridDim.x, ++u_local) {
+        const int slot = u_local & 1;
         TileRef t[2];
         t[0] = decode_tile(p, 2 * unit);
         const bool two = 2 * unit + 1 < total_tiles;
@@ -152,20 +151,39 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pass_kernel(const __grid_const
         const int nw = two ? 2 : 1;
         const int nsrc = (two && !shared) ? 2 : 1;
         for (int w = 0; w < nw && ok; ++w) {
-          if (q_loads[w] > 0 && !mbar_wait(&bars->q_empty[w], (q_loads[w] + 1) & 1, ctl)) { ok = false; break; }
-          mbar_arrive_expect_tx(&bars->q_full[w], box_bytes);
+          uint32_t& n_ld = q_loads[w][slot];
+          if (n_ld > 0 && !mbar_wait(&bars->q_empty[w][slot], (n_ld - 1) & 1, ctl)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&bars->q_full[w][slot], box_bytes);
           for (int panel = 0; panel < 2; ++panel) {
             int c[5];
-            chunk_coords(a.g, a.p, a.global_variant, t[w].bh, t[w].sigma, t[w].q, panel, c);
-            tma_load_5d(sQ + w * kTile + panel * kPanel, &a.tm_q, &bars->q_full[w], c[0], c[1], c[2], c[3], c[4]);
+            chunk_coords(g, p, a.global_variant, t[w].bh, t[w].sigma, t[w].q, panel, c);
+            tma_load_5d(sQ + (2 * w + slot) * kTile + panel * kPanel, &a.tm_q, &bars->q_full[w][slot], c[0], c[1],
+                        c[2], c[3], c[4]);
           }
-          ++q_loads[w];
+          ++n_ld;
         }
-        for (int b = 0; b <= nb && ok; ++b) {
-          if (b < nb)
-            for (int src = 0; src < nsrc && ok; ++src) ok = load_kv(&a.tm_k, t[src], b);
-          if (b >= 1)
-            for (int src = 0; src < nsrc && ok; ++src) ok = load_kv(&a.tm_v, t[src], b - 1);
+        for (int j = 0; j < 2 * nb && ok; ++j) {
+          // position j of the load order: K(b) or V(b)
+          const bool is_k = (j == 0) || (j < 2 * nb - 1 && (j & 1));
+          const int blk = is_k ? (j + 1) / 2 : (j == 2 * nb - 1 ? nb - 1 : j / 2 - 1);
+          for (int src = 0; src < nsrc && ok; ++src) {
+            const uint32_t s = kv_loads % kStages;
+            if (kv_loads >= kStages && !mbar_wait(&bars->kv_empty[s], ((kv_loads / kStages) + 1) & 1, ctl)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&bars->kv_full[s], box_bytes);
+            for (int panel = 0; panel < 2; ++panel) {
+              int c[5];
+              chunk_coords(g, p, a.global_variant, t[src].bh, t[src].sigma, blk, panel, c);
+              tma_load_5d(sKV + s * kTile + panel * kPanel, is_k ? &a.tm_k : &a.tm_v, &bars->kv_full[s], c[0], c[1],
+                          c[2], c[3], c[4]);
+            }
+            ++kv_loads;
+          }
         }
       }
       // Let every load this thread issued land before the CTA can exit (bounded).
@@ -173,15 +191,18 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pass_kernel(const __grid_const
       for (uint32_t i = first; i < kv_loads; ++i)
         mbar_wait_drain(&bars->kv_full[i % kStages], (i / kStages) & 1, 20000000ull);
       for (int w = 0; w < 2; ++w)
-        if (q_loads[w] > 0) mbar_wait_drain(&bars->q_full[w], (q_loads[w] - 1) & 1, 20000000ull);
+        for (int sl = 0; sl < 2; ++sl)
+          if (q_loads[w][sl] > 0) mbar_wait_drain(&bars->q_full[w][sl], (q_loads[w][sl] - 1) & 1, 20000000ull);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc_pv = idesc_bf16(128, 128, true);
-      uint32_t kv_cons = 0, q_cnt[2] = {0, 0}, p_cnt[2] = {0, 0};
+      uint32_t kv_base = 0, q_cnt[2][2] = {{0, 0}, {0, 0}}, p_cnt[2] = {0, 0};
       bool ok = true;
-      for (int unit = blockIdx.x; unit < n_units && ok; unit += gridDim.x) {
+      int u_local = 0;
+      for (int unit = blockIdx.x; unit < n_units && ok; unit += gridDim.x, ++u_local) {
+        const int slot = u_local & 1;
         TileRef t[2];
         t[0] = decode_tile(p, 2 * unit);
         const bool two = 2 * unit + 1 < total_tiles;
@@ -189,72 +210,50 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pass_kernel(const __grid_const
         const bool shared = two && t[0].bh == t[1].bh && t[0].sigma == t[1].sigma;
         const int nw = two ? 2 : 1;
         const int nsrc = (two && !shared) ? 2 : 1;
-        for (int w = 0; w < nw && ok; ++w) {
-          ok = mbar_wait(&bars->q_full[w], q_cnt[w] & 1, ctl);
-          ++q_cnt[w];
-        }
-        tc_fence_after();
         for (int b = 0; b <= nb && ok; ++b) {
-          if (b < nb) {
-            uint32_t kst[2];
-            for (int src = 0; src < nsrc && ok; ++src) {
-              kst[src] = kv_cons % kStages;
-              ok = mbar_wait(&bars->kv_full[kst[src]], (kv_cons / kStages) & 1, ctl);
-              ++kv_cons;
+          for (int w = 0; w < nw && ok; ++w) {
+            const int src = shared ? 0 : w;
+            const bool last_user = !shared || w == nw - 1;
+            if (b >= 1) {
+              // O_w += P_w(b-1) V(b-1), P read from the first columns of S_w
+              ok = mbar_wait(&bars->p_full[w], p_cnt[w] & 1, ctl);
+              ++p_cnt[w];
+              const uint32_t iv = kv_base + static_cast<uint32_t>(pos_v(b - 1, nb) * nsrc + src);
+              if (ok && (w == 0 || !shared)) ok = mbar_wait(&bars->kv_full[iv % kStages], (iv / kStages) & 1, ctl);
+              if (!ok) break;
+              tc_fence_after();
+              const int nk = round16(chunk_valid_rows(p, b - 1));
+              const uint32_t va = smem_u32(sKV + (iv % kStages) * kTile);
+              for (int kk = 0; kk < nk / 16; ++kk)
+                umma_bf16_ts(tmem + 256 * w + 128, tmem + 256 * w + kk * 8, sw128_desc(va + kk * 2048, kPanel, 1024),
+                             idesc_pv, (b - 1 > 0 || kk > 0) ? 1u : 0u);
+              if (b == nb) umma_commit(&bars->o_full[w]);
+              if (last_user) umma_commit(&bars->kv_empty[iv % kStages]);
             }
-            if (!ok) break;
-            tc_fence_after();
-            const int nk = round16(chunk_valid_rows(p, b));
-            const uint32_t idesc_s = idesc_bf16(128, nk, false);
-            for (int w = 0; w < nw && ok; ++w) {
-              if (b >= 1) {
-                ok = mbar_wait(&bars->p_full[w], p_cnt[w] & 1, ctl);
-                ++p_cnt[w];
-                if (!ok) break;
-                tc_fence_after();
+            if (b < nb) {
+              // S_w = Q_w K(b)^T
+              if (b == 0) {
+                ok = mbar_wait(&bars->q_full[w][slot], q_cnt[w][slot] & 1, ctl);
+                ++q_cnt[w][slot];
               }
-              const uint32_t qa = smem_u32(sQ + w * kTile);
-              const uint32_t ka = smem_u32(sKV + kst[shared ? 0 : w] * kTile);
+              const uint32_t ik = kv_base + static_cast<uint32_t>(pos_k(b) * nsrc + src);
+              if (ok && (w == 0 || !shared)) ok = mbar_wait(&bars->kv_full[ik % kStages], (ik / kStages) & 1, ctl);
+              if (!ok) break;
+              tc_fence_after();
+              const uint32_t idesc_s = idesc_bf16(128, round16(chunk_valid_rows(p, b)), false);
+              const uint32_t qa = smem_u32(sQ + (2 * w + slot) * kTile);
+              const uint32_t ka = smem_u32(sKV + (ik % kStages) * kTile);
               for (int kk = 0; kk < 8; ++kk) {
                 const uint32_t off = (kk >> 2) * kPanel + (kk & 3) * 32;
-                umma_bf16_ss(tmem + 256 * w, sw128_desc(qa + off, 16, 1024), sw128_desc(ka + off, 16, 1024),
-                             idesc_s, kk > 0);
+                umma_bf16_ss(tmem + 256 * w, sw128_desc(qa + off, 16, 1024), sw128_desc(ka + off, 16, 1024), idesc_s,
+                             kk > 0);
               }
               umma_commit(&bars->s_full[w]);
-              if (b == nb - 1) umma_commit(&bars->q_empty[w]);
+              if (last_user) umma_commit(&bars->kv_empty[ik % kStages]);
             }
-            if (!ok) break;
-            for (int src = 0; src < nsrc; ++src) umma_commit(&bars->kv_empty[kst[src]]);
-          }
-          if (b >= 1) {
-            uint32_t vst[2];
-            for (int src = 0; src < nsrc && ok; ++src) {
-              vst[src] = kv_cons % kStages;
-              ok = mbar_wait(&bars->kv_full[vst[src]], (kv_cons / kStages) & 1, ctl);
-              ++kv_cons;
-            }
-            if (!ok) break;
-            tc_fence_after();
-            const int nk = round16(chunk_valid_rows(p, b - 1));
-            for (int w = 0; w < nw && ok; ++w) {
-              if (b == nb) {
-                ok = mbar_wait(&bars->p_full[w], p_cnt[w] & 1, ctl);
-                ++p_cnt[w];
-                if (!ok) break;
-                tc_fence_after();
-              }
-              const uint32_t pa = smem_u32(sP + w * kTile);
-              const uint32_t va = smem_u32(sKV + vst[shared ? 0 : w] * kTile);
-              for (int kk = 0; kk < nk / 16; ++kk) {
-                umma_bf16_ss(tmem + 256 * w + 128, sw128_desc(pa + (kk >> 2) * kPanel + (kk & 3) * 32, 16, 1024),
-                             sw128_desc(va + kk * 2048, kPanel, 1024), idesc_pv, (b - 1 > 0 || kk > 0) ? 1u : 0u);
-              }
-              umma_commit(&bars->o_full[w]);
-            }
-            if (!ok) break;
-            for (int src = 0; src < nsrc; ++src) umma_commit(&bars->kv_empty[vst[src]]);
           }
         }
+        kv_base += static_cast<uint32_t>(2 * nb * nsrc);
       }
       // Wait (bounded) until every MMA issued above has completed before TMEM can be released.
       umma_commit(&bars->drain);
@@ -267,41 +266,54 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pass_kernel(const __grid_const
     const int row = wq * 32 + lane;
     const uint32_t t_s = tmem + 256 * wg + (static_cast<uint32_t>(wq * 32) << 16);
     const uint32_t t_o = t_s + 128;
-    uint8_t* buf = sP + wg * kTile;
     const float sl2 = a.scale_log2;
     uint32_t s_cnt = 0, o_cnt = 0;
     bool ok = true;
-    for (int unit = blockIdx.x; unit < n_units && ok; unit += gridDim.x) {
+    int u_local = 0;
+    for (int unit = blockIdx.x; unit < n_units && ok; unit += gridDim.x, ++u_local) {
+      const int slot = u_local & 1;
       const int tile = 2 * unit + wg;
       if (tile >= total_tiles) break;
       const TileRef t = decode_tile(p, tile);
-      float m_used = -INFINITY, l = 0.f;
+      // A warp whose 32 query rows are all padding skips the arithmetic but keeps every barrier.
+      const bool active = wq * 32 < chunk_valid_rows(p, t.q);
+      const int my_tok = token_of(g, p, t.sigma, t.q, row);
+      float m_used = -INFINITY;
+      float l = 0.f;    // sum of the bf16-rounded weights: normalises O
+      float le = 0.f;   // sum of the unrounded weights: the log-sum-exp
       for (int b = 0; b < nb && ok; ++b) {
         ok = mbar_wait(&bars->s_full[wg], s_cnt & 1, ctl);
         ++s_cnt;
         if (!ok) break;
-        tc_fence_after();
+        tc_fence_after();   // S(b) is ready, and so is every earlier PV (in-order tensor pipe)
         const int valid = chunk_valid_rows(p, b);
         const int nk = round16(valid);
-        // pass 1: row maximum of the scaled scores (log2 domain)
-        float mx = -INFINITY;
         uint32_t r[32];
+        float m_new = m_used;
+        if (active) {
+          // pass 1: row maximum (4 independent partial maxima; the scale is positive, so it is applied
+          // to the maximum instead of to every score)
+          float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          if (c * 32 < nk) {
-            tmem_ld32(t_s + c * 32, r);
+          for (int c = 0; c < 4; ++c) {
+            if (c * 32 < nk) {
+              tmem_ld32(t_s + c * 32, r);
+              if (c * 32 + 32 <= valid) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (c * 32 + i < valid) mx = fmaxf(mx, __uint_as_float(r[i]) * sl2);
+                for (int i = 0; i < 32; ++i) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(r[i]));
+              } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                  if (c * 32 + i < valid) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(r[i]));
+              }
+            }
           }
+          m_new = fmaxf(m_used, fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2);
         }
-        const float m_new = fmaxf(m_used, mx);
         if (b > 0) {
-          ok = mbar_wait(&bars->o_full[wg], o_cnt & 1, ctl);
-          ++o_cnt;
-          if (!ok) break;
-          tc_fence_after();
-          const bool need = m_new > m_used + 8.f;
+          // Rescale O only when the running maximum grew by more than 2^8 (until then the unscaled
+          // exponentials stay below 256). PV(b-1) has completed: S(b) was issued after it.
+          const bool need = active && m_new > m_used + 8.f;
           if (__any_sync(0xffffffffu, need)) {
             const float f = need ? ex2_approx(m_used - m_new) : 1.f;
 #pragma unroll
@@ -313,80 +325,89 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pass_kernel(const __grid_const
             }
             if (need) {
               l *= f;
+              le *= f;
               m_used = m_new;
             }
           }
         } else {
           m_used = m_new;
         }
-        // pass 2: P = 2^(x - m), row sum, bf16 P into the swizzled K-major tile
+        if (active) {
+          // pass 2: P = 2^(x - m) rounded to bf16 on the integer pipe (add half an ulp, drop the low
+          // half) and packed two per TMEM column over the first half of S.
+          float ls[4] = {0.f, 0.f, 0.f, 0.f};
+          float lx[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          if (c * 32 < nk) {
-            tmem_ld32(t_s + c * 32, r);
+          for (int c = 0; c < 4; ++c) {
+            if (c * 32 < nk) {
+              tmem_ld32(t_s + c * 32, r);
+              const bool full = c * 32 + 32 <= valid;
+              uint32_t pk[16];
 #pragma unroll
-            for (int h8 = 0; h8 < 4; ++h8) {
-              const int col0 = c * 32 + h8 * 8;
-              if (col0 < nk) {
-                float pv[8];
+              for (int i = 0; i < 32; i += 2) {
+                uint32_t bits[2];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                  const int col = col0 + i;
-                  pv[i] = col < valid ? ex2_approx(fmaf(__uint_as_float(r[h8 * 8 + i]), sl2, -m_used)) : 0.f;
-                  l += pv[i];
+                for (int e = 0; e < 2; ++e) {
+                  float x = ex2_approx(fmaf(__uint_as_float(r[i + e]), sl2, -m_used));
+                  if (!full && c * 32 + i + e >= valid) x = 0.f;
+                  lx[(i + e) & 3] += x;
+                  bits[e] = (__float_as_uint(x) + 0x8000u) & 0xFFFF0000u;
+                  ls[(i + e) & 3] += __uint_as_float(bits[e]);
                 }
-                uint4 v;
-                v.x = pack_bf16x2(pv[0], pv[1]);
-                v.y = pack_bf16x2(pv[2], pv[3]);
-                v.z = pack_bf16x2(pv[4], pv[5]);
-                v.w = pack_bf16x2(pv[6], pv[7]);
-                *reinterpret_cast<uint4*>(buf + sw_off(row, col0 >> 3)) = v;
+                pk[i >> 1] = __byte_perm(bits[0], bits[1], 0x7632);
               }
+              tmem_st16(t_s + c * 16, pk);
             }
           }
+          l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+          le += (lx[0] + lx[1]) + (lx[2] + lx[3]);
         }
-        fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(&bars->p_full[wg]);
       }
       if (!ok) break;
-      // epilogue: O / l -> bf16 staging (this warp's 32 rows of `buf`) -> coalesced global stores
+      // epilogue: O / l -> bf16 staged in this tile's Q buffer (its S products are done) -> coalesced
+      // global stores; then the Q buffer goes back to the producer.
       ok = mbar_wait(&bars->o_full[wg], o_cnt & 1, ctl);
       ++o_cnt;
       if (!ok) break;
       tc_fence_after();
-      const float inv_l = 1.f / l;
-      uint32_t r[32];
+      uint8_t* buf = sQ + (2 * wg + slot) * kTile;
+      if (active) {
+        const float inv_l = 1.f / l;
+        uint32_t r[32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        tmem_ld32(t_o + c * 32, r);
+        for (int c = 0; c < 4; ++c) {
+          tmem_ld32(t_o + c * 32, r);
 #pragma unroll
-        for (int h8 = 0; h8 < 4; ++h8) {
-          uint4 v;
-          v.x = pack_bf16x2(__uint_as_float(r[h8 * 8 + 0]) * inv_l, __uint_as_float(r[h8 * 8 + 1]) * inv_l);
-          v.y = pack_bf16x2(__uint_as_float(r[h8 * 8 + 2]) * inv_l, __uint_as_float(r[h8 * 8 + 3]) * inv_l);
-          v.z = pack_bf16x2(__uint_as_float(r[h8 * 8 + 4]) * inv_l, __uint_as_float(r[h8 * 8 + 5]) * inv_l);
-          v.w = pack_bf16x2(__uint_as_float(r[h8 * 8 + 6]) * inv_l, __uint_as_float(r[h8 * 8 + 7]) * inv_l);
-          *reinterpret_cast<uint4*>(buf + sw_off(row, c * 4 + h8)) = v;
+          for (int h8 = 0; h8 < 4; ++h8) {
+            uint4 v;
+            v.x = pack_bf16x2(__uint_as_float(r[h8 * 8 + 0]) * inv_l, __uint_as_float(r[h8 * 8 + 1]) * inv_l);
+            v.y = pack_bf16x2(__uint_as_float(r[h8 * 8 + 2]) * inv_l, __uint_as_float(r[h8 * 8 + 3]) * inv_l);
+            v.z = pack_bf16x2(__uint_as_float(r[h8 * 8 + 4]) * inv_l, __uint_as_float(r[h8 * 8 + 5]) * inv_l);
+            v.w = pack_bf16x2(__uint_as_float(r[h8 * 8 + 6]) * inv_l, __uint_as_float(r[h8 * 8 + 7]) * inv_l);
+            *reinterpret_cast<uint4*>(buf + sw_off(row, c * 4 + h8)) = v;
+          }
         }
-      }
-      __syncwarp();
-      const size_t head_base = static_cast<size_t>(t.bh) * g.n;
+        __syncwarp();
+        const size_t head_base = static_cast<size_t>(t.bh) * g.n;
 #pragma unroll 4
-      for (int it = 0; it < 16; ++it) {
-        const int rr = wq * 32 + 2 * it + (lane >> 4);
-        const int ch = lane & 15;
-        const int tok = token_of(g, p, t.sigma, t.q, rr);
-        if (tok >= 0) {
-          const uint4 v = *reinterpret_cast<const uint4*>(buf + sw_off(rr, ch));
-          *reinterpret_cast<uint4*>(a.out + (head_base + tok) * 128 + ch * 8) = v;
+        for (int it = 0; it < 16; ++it) {
+          const int rr = 2 * it + (lane >> 4);   // row within this warp's 32
+          const int ch = lane & 15;
+          const int tok = __shfl_sync(0xffffffffu, my_tok, rr);
+          if (tok >= 0) {
+            const uint4 v = *reinterpret_cast<const uint4*>(buf + sw_off(wq * 32 + rr, ch));
+            *reinterpret_cast<uint4*>(a.out + (head_base + tok) * 128 + ch * 8) = v;
+          }
         }
+        if (a.lse != nullptr && my_tok >= 0) a.lse[head_base + my_tok] = (m_used + __log2f(le)) * 0.69314718055994531f;
       }
-      if (a.lse != nullptr) {
-        const int tok = token_of(g, p, t.sigma, t.q, row);
-        if (tok >= 0) a.lse[head_base + tok] = (m_used + __log2f(l)) * 0.69314718055994531f;
-      }
+      // The generic-proxy writes and reads of the staging area must be ordered before the next TMA
+      // load into this Q buffer.
+      fence_proxy_async_smem();
       __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->q_empty[wg][slot]);
     }
   }
 
