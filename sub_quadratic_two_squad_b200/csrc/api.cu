@@ -12,6 +12,7 @@
 
 #include "squad_attn.h"
 #include "geometry.cuh"
+#include "short_pass.h"
 #include "simt_pass.h"
 #include "tc_pass.h"
 
@@ -66,6 +67,7 @@ squad_status_t validate(const squad_params_t* p, bool windowed, Grid* g, float* 
     gg.nwy = p->H;
     gg.nwx = p->W;
   }
+  finish_grid(gg);
   *g = gg;
   *scale = p->scale > 0.f ? p->scale : 1.0f / std::sqrt(static_cast<float>(p->d));
   return SQUAD_OK;
@@ -145,16 +147,10 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// Slot-box encoding for the GLOBAL pass. 0: element-strided box over the natural view (the slot's
-// tokens are every ww-th x and every hw-th y). 1: a view with dims (d, wx, wy, dx, (bh*T+t)*H+dy)
-// whose box has unit strides. Both describe the same tokens.
-int slot_box_variant() {
-  static int v = [] {
-    const char* e = std::getenv("SQUAD_SLOT_BOX");
-    return (e != nullptr && e[0] == '1') ? 1 : 0;
-  }();
-  return v;
-}
+// Slot-box encoding for the GLOBAL pass: a view with dims (d, wx, wy, dx, (bh*T+t)*H+dy) whose box
+// has unit element strides (geometry.cuh, variant 1). Tiled TMA stores use the same maps, and they
+// are only defined for unit element strides.
+constexpr int kSlotBoxVariant = 1;
 
 bool encode_pass_map(CUtensorMap* m, const void* base, const Grid& g, const PassGeom& p, int variant) {
   auto fn = encode_fn();
@@ -195,22 +191,46 @@ int num_sms_current() {
   return sms;
 }
 
+// Sequences of at most 256 tokens run whole (one TMA box, one K/V block) in the short-sequence kernel.
+bool short_eligible(const squad_params_t* prm, const Grid& g, const PassGeom& p) {
+  return prm->dtype == SQUAD_BF16 && g.d == 128 && p.kind != kFull && p.seq_len <= 256 && p.n_chunks == 1;
+}
+
 // One attention pass: out = softmax(scale q k^T) v over the sequences of `kind`.
 squad_status_t run_pass(const squad_params_t* prm, const Grid& g, int kind, float scale, const void* q,
                         const void* k, const void* v, bool v_bf16, void* out, float* lse, uint32_t* status,
                         cudaStream_t stream) {
+  const PassGeom ps = make_geom(g, kind, 256);
+  if (short_eligible(prm, g, ps) && v_bf16) {
+    ShortPassArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.g = g;
+    a.p = ps;
+    a.global_variant = kind == kGlobal ? kSlotBoxVariant : 0;
+    if (short_pass_plan(a)) {
+      if (!encode_pass_map(&a.tm_q, q, g, ps, a.global_variant) || !encode_pass_map(&a.tm_k, k, g, ps, a.global_variant) ||
+          !encode_pass_map(&a.tm_v, v, g, ps, a.global_variant) || !encode_pass_map(&a.tm_o, out, g, ps, a.global_variant))
+        return SQUAD_ERR_CUDA;
+      a.lse = lse;
+      a.scale_log2 = scale * 1.4426950408889634f;
+      a.status = status;
+      a.timeout_ns = kWaitTimeoutNs;
+      const int sms = num_sms_current();
+      if (sms <= 0) return SQUAD_ERR_CUDA;
+      return launch_short_pass(a, sms, stream) == cudaSuccess ? SQUAD_OK : SQUAD_ERR_CUDA;
+    }
+  }
   const PassGeom p = make_geom(g, kind);
   if (tc_eligible(prm, g, p) && v_bf16) {
     TcPassArgs a;
     std::memset(&a, 0, sizeof(a));
-    const int variant = kind == kGlobal ? slot_box_variant() : 0;
+    const int variant = kind == kGlobal ? kSlotBoxVariant : 0;
     if (!encode_pass_map(&a.tm_q, q, g, p, variant) || !encode_pass_map(&a.tm_k, k, g, p, variant) ||
-        !encode_pass_map(&a.tm_v, v, g, p, variant))
+        !encode_pass_map(&a.tm_v, v, g, p, variant) || !encode_pass_map(&a.tm_o, out, g, p, variant))
       return SQUAD_ERR_CUDA;
     a.g = g;
     a.p = p;
     a.global_variant = variant;
-    a.out = static_cast<__nv_bfloat16*>(out);
     a.lse = lse;
     a.scale_log2 = scale * 1.4426950408889634f;
     a.status = status;

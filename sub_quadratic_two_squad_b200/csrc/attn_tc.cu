@@ -4,20 +4,23 @@
 // full attention (paper eq. 5) over every (b, head). Each sequence is read straight out of the
 // caller's [B, h, n, d] tensors through TMA boxes (geometry.cuh): no permuted copy is made.
 //
-// CTA organisation (persistent, one CTA per SM, 384 threads):
-//   warp 0      TMA producer: double-buffered Q tiles per warpgroup and a 3-stage ring of K/V blocks
-//               (128 keys x 128 dims, bf16, 128-byte swizzle).
-//   warp 1      TMEM allocator and MMA issuer (one thread).
-//   warps 4-7   softmax warpgroup 0 (TMEM lanes 0-127 of S0 / O0)
-//   warps 8-11  softmax warpgroup 1 (S1 / O1).
+// CTA organisation (persistent, one CTA per SM, 352 threads):
+//   warps 0-3   softmax warpgroup 0 (TMEM lanes 0-127 of S0 / O0)
+//   warps 4-7   softmax warpgroup 1 (S1 / O1)
+//   warp 8      TMA producer: double-buffered Q tiles per warpgroup and a 3-stage ring of K/V blocks
+//               (128 keys x 128 dims, bf16, 128-byte swizzle)
+//   warp 9      TMEM allocator and MMA issuer (one thread)
+//   warp 10     TMA store issuer for the outputs.
 // A work unit is a pair of 128-row query tiles, one per softmax warpgroup; when both belong to the
 // same sequence they share every K/V block. Per warpgroup, tensor memory holds the scores S (128 fp32
-// columns) and the output accumulator O (128 columns). The softmax writes P as bf16 over the first
-// half of S, and the PV product reads it from there (tcgen05.mma with A in tensor memory), so the
-// MMA issue order per warpgroup is ... S(b), [softmax], PV(b), S(b+1) ... and the in-order tensor
-// pipe finishes reading P(b) before S(b+1) overwrites it. Softmax is online across K/V blocks; the
-// rescale of O is skipped unless the row maximum grew by more than 2^8. The epilogue stages O through
-// the tile's own Q buffer (free once its last S is done) and writes it with coalesced stores.
+// columns) and the output accumulator O (128 columns). A softmax thread owns one query row: it loads
+// the row's 128 scores with one tcgen05.ld, writes P as bf16 over the first half of S, and the PV
+// product reads it from there (tcgen05.mma with A in tensor memory); the MMA issue order per
+// warpgroup is ... S(b), [softmax], PV(b), S(b+1) ..., so the in-order tensor pipe finishes reading
+// P(b) before S(b+1) overwrites it. Softmax is online across K/V blocks; the rescale of O is skipped
+// unless the row maximum grew by more than 2^8. The epilogue stages O through the tile's own Q buffer
+// (free once its last S is done); the store warp writes it back with a TMA store of the same chunk
+// box, which scatters the rows to their tokens and drops the padding rows.
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
@@ -29,7 +32,8 @@ namespace squad {
 
 namespace {
 
-constexpr int kThreads = 384;
+constexpr int kThreads = 352;
+constexpr int kWarpProducer = 8, kWarpMma = 9, kWarpStore = 10;
 constexpr int kStages = 3;
 constexpr uint32_t kPanel = 16384;   // 128 rows x 128 bytes (64 bf16)
 constexpr uint32_t kTile = 2 * kPanel;
@@ -43,7 +47,7 @@ static_assert(kSmemBytes <= 232448, "shared memory budget");
 struct Bars {
   uint64_t q_full[2][2], q_empty[2][2];
   uint64_t kv_full[kStages], kv_empty[kStages];
-  uint64_t s_full[2], p_full[2], o_full[2];
+  uint64_t s_full[2], p_full[2], o_full[2], staged[2];
   uint64_t drain;
   uint32_t tmem_base;
   uint32_t abort;
@@ -57,9 +61,9 @@ struct TileRef {
 __device__ __forceinline__ TileRef decode_tile(const PassGeom& p, int tile) {
   TileRef t;
   const int per_bh = p.n_seq * p.n_chunks;
-  t.bh = tile / per_bh;
+  t.bh = static_cast<int>(fdiv(static_cast<uint32_t>(tile), p.f_per_bh));
   const int rem = tile - t.bh * per_bh;
-  t.sigma = rem / p.n_chunks;
+  t.sigma = static_cast<int>(fdiv(static_cast<uint32_t>(rem), p.f_chunks));
   t.q = rem - t.sigma * p.n_chunks;
   return t;
 }
@@ -98,11 +102,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pass_kernel(const __grid_const
     for (int w = 0; w < 2; ++w) {
       for (int sl = 0; sl < 2; ++sl) {
         mbar_init(&bars->q_full[w][sl], 1);
-        mbar_init(&bars->q_empty[w][sl], 4);   // one arrival per warp of the warpgroup
+        mbar_init(&bars->q_empty[w][sl], 1);   // the store warp, once the tile's store has read it
       }
       mbar_init(&bars->s_full[w], 1);
       mbar_init(&bars->p_full[w], 128);
       mbar_init(&bars->o_full[w], 1);
+      mbar_init(&bars->staged[w], 4);   // one arrival per warp of the warpgroup
     }
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&bars->kv_full[s], 1);
@@ -112,12 +117,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pass_kernel(const __grid_const
     bars->abort = 0;
     fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) {
+  if (warp == kWarpProducer && lane == 0) {
     prefetch_tmap(&a.tm_q);
     prefetch_tmap(&a.tm_k);
     prefetch_tmap(&a.tm_v);
+    prefetch_tmap(&a.tm_o);
   }
-  if (warp == 1) {
+  if (warp == kWarpMma) {
     tmem_alloc(&bars->tmem_base, 512);
     tmem_relinquish();
   }
@@ -134,7 +140,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pass_kernel(const __grid_const
   const int nb = p.n_chunks;
   const uint32_t box_bytes = 2u * static_cast<uint32_t>(p.chunk_rows) * 128u;
 
-  if (warp == 0) {
+  if (warp == kWarpProducer) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       uint32_t q_loads[2][2] = {{0, 0}, {0, 0}};
@@ -194,7 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pass_kernel(const __grid_const
         for (int sl = 0; sl < 2; ++sl)
           if (q_loads[w][sl] > 0) mbar_wait_drain(&bars->q_full[w][sl], (q_loads[w][sl] - 1) & 1, 20000000ull);
     }
-  } else if (warp == 1) {
+  } else if (warp == kWarpMma) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc_pv = idesc_bf16(128, 128, true);
@@ -259,9 +265,36 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pass_kernel(const __grid_const
       umma_commit(&bars->drain);
       mbar_wait_drain(&bars->drain, 0, 20000000ull);
     }
-  } else if (warp >= 4) {
+  } else if (warp == kWarpStore) {
+    // ------------------------------------------------------------------ TMA store issuer
+    if (lane == 0) {
+      uint32_t st_cnt[2] = {0, 0};
+      bool ok = true;
+      int u_local = 0;
+      for (int unit = blockIdx.x; unit < n_units && ok; unit += gridDim.x, ++u_local) {
+        const int slot = u_local & 1;
+        for (int w = 0; w < 2 && ok; ++w) {
+          const int tile = 2 * unit + w;
+          if (tile >= total_tiles) break;
+          ok = mbar_wait(&bars->staged[w], st_cnt[w] & 1, ctl);
+          ++st_cnt[w];
+          if (!ok) break;
+          const TileRef t = decode_tile(p, tile);
+          const uint8_t* buf = sQ + (2 * w + slot) * kTile;
+          int c[5];
+          chunk_coords(g, p, a.global_variant, t.bh, t.sigma, t.q, 0, c);
+          tma_store_5d(&a.tm_o, buf, c[0], c[1], c[2], c[3], c[4]);
+          tma_store_5d(&a.tm_o, buf + kPanel, c[0] + 64, c[1], c[2], c[3], c[4]);
+          bulk_commit_group();
+          bulk_wait_read_all();   // the Q buffer may be refilled once the store has read it
+          mbar_arrive(&bars->q_empty[w][slot]);
+        }
+      }
+      bulk_wait_all();   // outputs written before the CTA exits
+    }
+  } else if (warp < 8) {
     // ------------------------------------------------------------------ softmax warpgroups
-    const int wg = (warp - 4) >> 2;
+    const int wg = warp >> 2;
     const int wq = warp & 3;
     const int row = wq * 32 + lane;
     const uint32_t t_s = tmem + 256 * wg + (static_cast<uint32_t>(wq * 32) << 16);
@@ -277,137 +310,111 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pass_kernel(const __grid_const
       const TileRef t = decode_tile(p, tile);
       // A warp whose 32 query rows are all padding skips the arithmetic but keeps every barrier.
       const bool active = wq * 32 < chunk_valid_rows(p, t.q);
-      const int my_tok = token_of(g, p, t.sigma, t.q, row);
       float m_used = -INFINITY;
-      float l = 0.f;    // sum of the bf16-rounded weights: normalises O
-      float le = 0.f;   // sum of the unrounded weights: the log-sum-exp
+      float l = 0.f;
       for (int b = 0; b < nb && ok; ++b) {
         ok = mbar_wait(&bars->s_full[wg], s_cnt & 1, ctl);
         ++s_cnt;
         if (!ok) break;
         tc_fence_after();   // S(b) is ready, and so is every earlier PV (in-order tensor pipe)
         const int valid = chunk_valid_rows(p, b);
-        const int nk = round16(valid);
-        uint32_t r[32];
+        uint32_t r[128];
         float m_new = m_used;
         if (active) {
-          // pass 1: row maximum (4 independent partial maxima; the scale is positive, so it is applied
-          // to the maximum instead of to every score)
+          tmem_ld128(t_s, r);
+          if (valid < 128)
+#pragma unroll
+            for (int i = 0; i < 128; ++i)
+              if (i >= valid) r[i] = __float_as_uint(-INFINITY);
+          // row maximum (4 independent partial maxima; the scale is positive, so it is applied to the
+          // maximum instead of to every score)
           float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            if (c * 32 < nk) {
-              tmem_ld32(t_s + c * 32, r);
-              if (c * 32 + 32 <= valid) {
-#pragma unroll
-                for (int i = 0; i < 32; ++i) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(r[i]));
-              } else {
-#pragma unroll
-                for (int i = 0; i < 32; ++i)
-                  if (c * 32 + i < valid) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(r[i]));
-              }
-            }
-          }
+          for (int i = 0; i < 128; ++i) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(r[i]));
           m_new = fmaxf(m_used, fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2);
         }
         if (b > 0) {
           // Rescale O only when the running maximum grew by more than 2^8 (until then the unscaled
-          // exponentials stay below 256). PV(b-1) has completed: S(b) was issued after it.
+          // exponentials stay below 256). PV(b-1) has completed: S(b) was issued after it. This path is
+          // rare, so it reuses the score registers for O and reloads S afterwards.
           const bool need = active && m_new > m_used + 8.f;
           if (__any_sync(0xffffffffu, need)) {
             const float f = need ? ex2_approx(m_used - m_new) : 1.f;
+            tmem_ld128(t_o, r);
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              tmem_ld32(t_o + c * 32, r);
-#pragma unroll
-              for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * f);
-              tmem_st32(t_o + c * 32, r);
-            }
+            for (int i = 0; i < 128; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * f);
+            tmem_st128(t_o, r);
             if (need) {
               l *= f;
-              le *= f;
               m_used = m_new;
+            }
+            if (active) {
+              tmem_ld128(t_s, r);
+              if (valid < 128)
+#pragma unroll
+                for (int i = 0; i < 128; ++i)
+                  if (i >= valid) r[i] = __float_as_uint(-INFINITY);
             }
           }
         } else {
           m_used = m_new;
         }
         if (active) {
-          // pass 2: P = 2^(x - m) rounded to bf16 on the integer pipe (add half an ulp, drop the low
-          // half) and packed two per TMEM column over the first half of S.
+          // P = 2^(x - m) (masked columns give 2^-inf = 0), rounded to bf16 on the integer pipe (add half
+          // an ulp, keep the high half), packed two per 32-bit word and stored 32 scores at a time over
+          // the first 64 TMEM columns of S (the scores are already in registers).
+          const float nm = -m_used;
           float ls[4] = {0.f, 0.f, 0.f, 0.f};
-          float lx[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            if (c * 32 < nk) {
-              tmem_ld32(t_s + c * 32, r);
-              const bool full = c * 32 + 32 <= valid;
-              uint32_t pk[16];
+          for (int k = 0; k < 4; ++k) {
+            uint32_t pk[16];
 #pragma unroll
-              for (int i = 0; i < 32; i += 2) {
-                uint32_t bits[2];
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                  float x = ex2_approx(fmaf(__uint_as_float(r[i + e]), sl2, -m_used));
-                  if (!full && c * 32 + i + e >= valid) x = 0.f;
-                  lx[(i + e) & 3] += x;
-                  bits[e] = (__float_as_uint(x) + 0x8000u) & 0xFFFF0000u;
-                  ls[(i + e) & 3] += __uint_as_float(bits[e]);
-                }
-                pk[i >> 1] = __byte_perm(bits[0], bits[1], 0x7632);
-              }
-              tmem_st16(t_s + c * 16, pk);
+            for (int j = 0; j < 16; ++j) {
+              const float x0 = ex2_approx(fmaf(__uint_as_float(r[32 * k + 2 * j]), sl2, nm));
+              const float x1 = ex2_approx(fmaf(__uint_as_float(r[32 * k + 2 * j + 1]), sl2, nm));
+              ls[(2 * j) & 3] += x0;
+              ls[(2 * j + 1) & 3] += x1;
+              pk[j] = __byte_perm(__float_as_uint(x0) + 0x8000u, __float_as_uint(x1) + 0x8000u, 0x7632);
             }
+            tmem_st16(t_s + 16 * k, pk);
           }
           l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-          le += (lx[0] + lx[1]) + (lx[2] + lx[3]);
         }
         tc_fence_before();
         mbar_arrive(&bars->p_full[wg]);
       }
       if (!ok) break;
-      // epilogue: O / l -> bf16 staged in this tile's Q buffer (its S products are done) -> coalesced
-      // global stores; then the Q buffer goes back to the producer.
+      // epilogue: O / l -> bf16 staged in this tile's Q buffer (its S products are done); the store
+      // warp writes it back.
       ok = mbar_wait(&bars->o_full[wg], o_cnt & 1, ctl);
       ++o_cnt;
       if (!ok) break;
       tc_fence_after();
-      uint8_t* buf = sQ + (2 * wg + slot) * kTile;
       if (active) {
+        const uint32_t row_addr = smem_u32(sQ) + (2 * wg + slot) * kTile + row * 128;
         const float inv_l = 1.f / l;
-        uint32_t r[32];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          tmem_ld32(t_o + c * 32, r);
+        for (int h = 0; h < 2; ++h) {
+          uint32_t o[64];
+          tmem_ld64(t_o + h * 64, o);
 #pragma unroll
-          for (int h8 = 0; h8 < 4; ++h8) {
-            uint4 v;
-            v.x = pack_bf16x2(__uint_as_float(r[h8 * 8 + 0]) * inv_l, __uint_as_float(r[h8 * 8 + 1]) * inv_l);
-            v.y = pack_bf16x2(__uint_as_float(r[h8 * 8 + 2]) * inv_l, __uint_as_float(r[h8 * 8 + 3]) * inv_l);
-            v.z = pack_bf16x2(__uint_as_float(r[h8 * 8 + 4]) * inv_l, __uint_as_float(r[h8 * 8 + 5]) * inv_l);
-            v.w = pack_bf16x2(__uint_as_float(r[h8 * 8 + 6]) * inv_l, __uint_as_float(r[h8 * 8 + 7]) * inv_l);
-            *reinterpret_cast<uint4*>(buf + sw_off(row, c * 4 + h8)) = v;
+          for (int c = 0; c < 8; ++c) {
+            // 16-byte chunk c of this panel's 128-byte row, at its 128-byte-swizzled position
+            st_shared_v4(row_addr + h * kPanel + ((c ^ (row & 7)) << 4),
+                         pack_bf16x2(__uint_as_float(o[c * 8 + 0]) * inv_l, __uint_as_float(o[c * 8 + 1]) * inv_l),
+                         pack_bf16x2(__uint_as_float(o[c * 8 + 2]) * inv_l, __uint_as_float(o[c * 8 + 3]) * inv_l),
+                         pack_bf16x2(__uint_as_float(o[c * 8 + 4]) * inv_l, __uint_as_float(o[c * 8 + 5]) * inv_l),
+                         pack_bf16x2(__uint_as_float(o[c * 8 + 6]) * inv_l, __uint_as_float(o[c * 8 + 7]) * inv_l));
           }
         }
-        __syncwarp();
-        const size_t head_base = static_cast<size_t>(t.bh) * g.n;
-#pragma unroll 4
-        for (int it = 0; it < 16; ++it) {
-          const int rr = 2 * it + (lane >> 4);   // row within this warp's 32
-          const int ch = lane & 15;
-          const int tok = __shfl_sync(0xffffffffu, my_tok, rr);
-          if (tok >= 0) {
-            const uint4 v = *reinterpret_cast<const uint4*>(buf + sw_off(wq * 32 + rr, ch));
-            *reinterpret_cast<uint4*>(a.out + (head_base + tok) * 128 + ch * 8) = v;
-          }
+        if (a.lse != nullptr) {
+          const int tok = token_of(g, p, t.sigma, t.q, row);
+          if (tok >= 0) a.lse[static_cast<size_t>(t.bh) * g.n + tok] = (m_used + __log2f(l)) * 0.69314718055994531f;
         }
-        if (a.lse != nullptr && my_tok >= 0) a.lse[head_base + my_tok] = (m_used + __log2f(le)) * 0.69314718055994531f;
       }
-      // The generic-proxy writes and reads of the staging area must be ordered before the next TMA
-      // load into this Q buffer.
-      fence_proxy_async_smem();
+      fence_proxy_async_smem();   // staging writes -> visible to the TMA store (async proxy)
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->q_empty[wg][slot]);
+      if (lane == 0) mbar_arrive(&bars->staged[wg]);
     }
   }
 
@@ -415,7 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pass_kernel(const __grid_const
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, 512);
+  if (warp == kWarpMma) tmem_dealloc(tmem, 512);
 }
 
 cudaError_t launch_tc_pass(const TcPassArgs& args, int num_sms, cudaStream_t stream) {

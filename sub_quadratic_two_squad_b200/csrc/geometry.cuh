@@ -10,13 +10,41 @@
 //          each line is the W/ww windows of that row.
 //   FULL   one sequence of all n tokens in order (plain softmax attention, paper eq. 5); lines are
 //          single tokens.
-// A chunk is L whole lines (L * line_len <= 128), so every chunk of a sequence is one rectangular
-// TMA box of the tensor, and lines past the end of the sequence fall outside the tensor (zero fill).
+// A chunk is L whole lines (L * line_len <= 128, or <= 256 for the short-sequence kernel), so every
+// chunk of a sequence is one rectangular TMA box of the tensor, and lines past the end of the
+// sequence fall outside the tensor (zero fill).
 #pragma once
 
 #include <cstdint>
 
 namespace squad {
+
+// Division by a divisor fixed at launch, as one high multiply and a shift: for d >= 2 with
+// L = ceil(log2 d), m = ceil(2^(31+L) / d) and s = L - 1, floor(n / d) = floor(n * m / 2^(31+L)) for
+// every 0 <= n < 2^31 (m / 2^(31+L) exceeds 1/d by less than 2^-(31+L), so n times the excess stays
+// below 2^-L <= 1/d and cannot carry floor(n/d) past the next integer). d == 1 is stored as m = 0.
+struct FastDiv {
+  uint32_t d, m, s;
+};
+
+__host__ __device__ inline FastDiv make_fastdiv(uint32_t d) {
+  FastDiv f{d, 0u, 0u};
+  if (d <= 1) return f;
+  uint32_t L = 0;
+  while ((1ull << L) < d) ++L;
+  f.m = static_cast<uint32_t>(((1ull << (31 + L)) + d - 1) / d);
+  f.s = L - 1;
+  return f;
+}
+
+__host__ __device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv& f) {
+  if (f.m == 0) return n;
+#ifdef __CUDA_ARCH__
+  return __umulhi(n, f.m) >> f.s;
+#else
+  return static_cast<uint32_t>((static_cast<unsigned long long>(n) * f.m) >> 32) >> f.s;
+#endif
+}
 
 enum PassKind : int { kLocal = 0, kGlobal = 1, kFull = 2 };
 
@@ -26,7 +54,14 @@ struct Grid {
   int hw, ww;           // window (tw == T)
   int n;                // T*H*W
   int nwy, nwx;         // H/hw, W/ww
+  FastDiv f_nwx, f_ww, f_hwww;   // divisions by nwx, ww and hw*ww
 };
+
+__host__ __device__ inline void finish_grid(Grid& g) {
+  g.f_nwx = make_fastdiv(static_cast<uint32_t>(g.nwx));
+  g.f_ww = make_fastdiv(static_cast<uint32_t>(g.ww));
+  g.f_hwww = make_fastdiv(static_cast<uint32_t>(g.hw * g.ww));
+}
 
 struct PassGeom {
   int kind;
@@ -37,9 +72,12 @@ struct PassGeom {
   int lines_per_chunk;  // L
   int n_chunks;         // ceil(n_lines / L)
   int chunk_rows;       // L * line_len  (rows of one TMA box, <= 128)
+  FastDiv f_line, f_chunks, f_per_bh;   // divisions by line_len, n_chunks and n_seq * n_chunks
 };
 
-__host__ __device__ inline PassGeom make_geom(const Grid& g, int kind) {
+// max_rows: most rows per chunk (128 for the chunked kernels; 256 makes a sequence of up to 256 tokens
+// one chunk).
+__host__ __device__ inline PassGeom make_geom(const Grid& g, int kind, int max_rows = 128) {
   PassGeom p{};
   p.kind = kind;
   if (kind == kLocal) {
@@ -58,33 +96,36 @@ __host__ __device__ inline PassGeom make_geom(const Grid& g, int kind) {
   p.seq_len = p.line_len * p.n_lines;
   // Whole lines per chunk, at most 128 rows; a line longer than 128 rows is one chunk by itself (only
   // the CUDA-core kernels accept such chunks).
-  p.lines_per_chunk = p.line_len > 128 ? 1 : 128 / p.line_len;
+  p.lines_per_chunk = p.line_len > max_rows ? 1 : max_rows / p.line_len;
   if (p.lines_per_chunk > p.n_lines) p.lines_per_chunk = p.n_lines;
   p.n_chunks = (p.n_lines + p.lines_per_chunk - 1) / p.lines_per_chunk;
   p.chunk_rows = p.lines_per_chunk * p.line_len;
+  p.f_line = make_fastdiv(static_cast<uint32_t>(p.line_len));
+  p.f_chunks = make_fastdiv(static_cast<uint32_t>(p.n_chunks));
+  p.f_per_bh = make_fastdiv(static_cast<uint32_t>(p.n_seq * p.n_chunks));
   return p;
 }
 
-// Token index (within one (b, head)) of row `r` (0..127) of chunk `q` of sequence `sigma`; -1 when the
-// row is padding: past the chunk's box, or past the end of the sequence.
+// Token index (within one (b, head)) of row `r` of chunk `q` of sequence `sigma`; -1 when the row is
+// padding: past the chunk's box, or past the end of the sequence.
 __host__ __device__ inline int token_of(const Grid& g, const PassGeom& p, int sigma, int q, int r) {
   if (r >= p.chunk_rows) return -1;
-  const int line = q * p.lines_per_chunk + r / p.line_len;
+  const int rl = static_cast<int>(fdiv(static_cast<uint32_t>(r), p.f_line));
+  const int line = q * p.lines_per_chunk + rl;
   if (line >= p.n_lines) return -1;
-  const int pos = r - (r / p.line_len) * p.line_len;
+  const int pos = r - rl * p.line_len;
   if (p.kind == kFull) return line;
   int t, y, x;
   if (p.kind == kLocal) {
-    const int wy = sigma / g.nwx, wx = sigma - (sigma / g.nwx) * g.nwx;
-    const int dy = pos / g.ww, dx = pos - (pos / g.ww) * g.ww;
+    const int wy = static_cast<int>(fdiv(static_cast<uint32_t>(sigma), g.f_nwx)), wx = sigma - wy * g.nwx;
+    const int dy = static_cast<int>(fdiv(static_cast<uint32_t>(pos), g.f_ww)), dx = pos - dy * g.ww;
     t = line;
     y = wy * g.hw + dy;
     x = wx * g.ww + dx;
   } else {
-    const int hwww = g.hw * g.ww;
-    t = sigma / hwww;
-    const int rem = sigma - t * hwww;
-    const int dy = rem / g.ww, dx = rem - (rem / g.ww) * g.ww;
+    t = static_cast<int>(fdiv(static_cast<uint32_t>(sigma), g.f_hwww));
+    const int rem = sigma - t * g.hw * g.ww;
+    const int dy = static_cast<int>(fdiv(static_cast<uint32_t>(rem), g.f_ww)), dx = rem - dy * g.ww;
     y = line * g.hw + dy;
     x = pos * g.ww + dx;
   }
@@ -147,16 +188,15 @@ __host__ __device__ inline void chunk_coords(const Grid& g, const PassGeom& p, i
                                              int chunk, int panel, int c[5]) {
   c[0] = panel * 64;
   if (p.kind == kLocal) {
-    const int wy = sigma / g.nwx, wx = sigma - (sigma / g.nwx) * g.nwx;
+    const int wy = static_cast<int>(fdiv(static_cast<uint32_t>(sigma), g.f_nwx)), wx = sigma - wy * g.nwx;
     c[1] = wx * g.ww;
     c[2] = wy * g.hw;
     c[3] = chunk * p.lines_per_chunk;
     c[4] = bh;
   } else if (p.kind == kGlobal) {
-    const int hwww = g.hw * g.ww;
-    const int tt = sigma / hwww;
-    const int rem = sigma - tt * hwww;
-    const int dy = rem / g.ww, dx = rem - (rem / g.ww) * g.ww;
+    const int tt = static_cast<int>(fdiv(static_cast<uint32_t>(sigma), g.f_hwww));
+    const int rem = sigma - tt * g.hw * g.ww;
+    const int dy = static_cast<int>(fdiv(static_cast<uint32_t>(rem), g.f_ww)), dx = rem - dy * g.ww;
     if (variant == 0) {
       c[1] = dx;
       c[2] = dy + chunk * p.lines_per_chunk * g.hw;

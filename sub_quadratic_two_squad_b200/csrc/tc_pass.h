@@ -11,10 +11,10 @@ namespace squad {
 
 struct TcPassArgs {
   CUtensorMap tm_q, tm_k, tm_v;   // bf16 tensor maps with the pass's chunk box (SWIZZLE_128B)
+  CUtensorMap tm_o;               // the same box over the output (tiled TMA stores)
   Grid g;
   PassGeom p;
   int global_variant;             // slot-box encoding used for the GLOBAL pass maps (see tmap.cpp)
-  __nv_bfloat16* out;             // [B, h, n, 128]
   float* lse;                     // [B, h, n] natural-log LSE, or null
   float scale_log2;               // softmax scale * log2(e)
   uint32_t* status;               // device status word (0 = ok, 4 = a wait timed out)

@@ -84,7 +84,33 @@ static int check_pass(const Grid& g, int kind, int variant, bool print) {
   return errors;
 }
 
+// Multiply-shift division against the hardware divide: every divisor up to 4096, numerators at the
+// boundaries and a pseudo-random sweep of [0, 2^31).
+static int check_fastdiv() {
+  int errors = 0;
+  unsigned long long x = 88172645463325252ull;
+  for (uint32_t d = 1; d <= 4096; ++d) {
+    const FastDiv f = make_fastdiv(d);
+    const uint32_t edge[] = {0u, 1u, d - 1, d, d + 1, 2 * d - 1, 2 * d, 0x7FFFFFFFu, 0x7FFFFFFEu,
+                             0x7FFFFFFFu - (0x7FFFFFFFu % d)};
+    for (uint32_t n : edge)
+      if (n < 0x80000000u && fdiv(n, f) != n / d) ++errors;
+    for (int i = 0; i < 2000; ++i) {
+      x ^= x << 13; x ^= x >> 7; x ^= x << 17;
+      const uint32_t n = static_cast<uint32_t>(x) & 0x7FFFFFFFu;
+      if (fdiv(n, f) != n / d) ++errors;
+    }
+  }
+  if (errors) std::printf("fastdiv errors %d\n", errors);
+  return errors;
+}
+
 int main(int argc, char** argv) {
+  if (argc == 2 && argv[1][0] == 'd') {
+    const int e = check_fastdiv();
+    std::printf(e == 0 ? "ok\n" : "FAILED\n");
+    return e == 0 ? 0 : 1;
+  }
   if (argc != 8) {
     std::printf("usage: geometry_check B h T H W hw ww\n");
     return 2;
@@ -101,6 +127,7 @@ int main(int argc, char** argv) {
   g.n = g.T * g.H * g.W;
   g.nwy = g.H / g.hw;
   g.nwx = g.W / g.ww;
+  finish_grid(g);
   int errors = 0;
   errors += check_pass(g, kLocal, 0, true);
   errors += check_pass(g, kGlobal, 0, true);
@@ -109,6 +136,7 @@ int main(int argc, char** argv) {
   f.hw = f.ww = 1;
   f.nwy = f.H;
   f.nwx = f.W;
+  finish_grid(f);
   errors += check_pass(f, kFull, 0, false);
   std::printf(errors == 0 ? "ok\n" : "FAILED %d\n", errors);
   return errors == 0 ? 0 : 1;

@@ -43,3 +43,8 @@ def test_boxes_match_oracle_tables(checker, B, h, grid, win):
     ref = orc.window_partition(T, H, W, T, *win)
     np.testing.assert_array_equal(np.array(tables[0]), ref)
     np.testing.assert_array_equal(np.array(tables[1]), ref.T)
+
+
+def test_fast_division(checker):
+    r = subprocess.run([checker, "div"], capture_output=True, text=True)
+    assert r.returncode == 0 and r.stdout.strip().endswith("ok"), r.stdout[-2000:]
