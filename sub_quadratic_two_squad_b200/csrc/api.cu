@@ -21,7 +21,9 @@ using namespace squad;
 namespace {
 
 constexpr int kAbiVersion = 1;
-constexpr size_t kCtrlBytes = 256;               // status word + reserved
+// Control block at the start of a workspace (zeroed by every call): word 0 the device status, words
+// 1-3 work counters of the persistent kernels, then one counter per (b, head) for the fused passes.
+constexpr size_t kCtrlFixedWords = 4;
 constexpr unsigned long long kWaitTimeoutNs = 1000000000ull;   // 1 s per device-side wait
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -75,8 +77,12 @@ squad_status_t validate(const squad_params_t* p, bool windowed, Grid* g, float* 
 
 size_t elem_bytes(const squad_params_t* p) { return p->dtype == SQUAD_BF16 ? 2 : 4; }
 
+size_t ctrl_bytes(const Grid& g) {
+  return align256(4 * (kCtrlFixedWords + static_cast<size_t>(g.B) * g.h));
+}
+
 struct FwdWorkspace {
-  uint32_t* status;
+  uint32_t* status;   // control block (ctrl_bytes)
   void* o1;
   float* lse1;
   float* lse2;
@@ -84,7 +90,7 @@ struct FwdWorkspace {
 
 size_t fwd_ws_bytes(const Grid& g, size_t eb) {
   const size_t bhn = static_cast<size_t>(g.B) * g.h * g.n;
-  return kCtrlBytes + align256(bhn * g.d * eb) + 2 * align256(bhn * 4);
+  return ctrl_bytes(g) + align256(bhn * g.d * eb) + 2 * align256(bhn * 4);
 }
 
 FwdWorkspace carve_fwd(void* ws, const Grid& g, size_t eb) {
@@ -92,7 +98,7 @@ FwdWorkspace carve_fwd(void* ws, const Grid& g, size_t eb) {
   const size_t bhn = static_cast<size_t>(g.B) * g.h * g.n;
   FwdWorkspace w;
   w.status = reinterpret_cast<uint32_t*>(b);
-  b += kCtrlBytes;
+  b += ctrl_bytes(g);
   w.o1 = b;
   b += align256(bhn * g.d * eb);
   w.lse1 = reinterpret_cast<float*>(b);
@@ -111,7 +117,7 @@ struct BwdWorkspace {
 
 size_t bwd_ws_bytes(const Grid& g) {
   const size_t bhn = static_cast<size_t>(g.B) * g.h * g.n;
-  return kCtrlBytes + 3 * align256(bhn * g.d * 4) + align256(bhn * 4);
+  return ctrl_bytes(g) + 3 * align256(bhn * g.d * 4) + align256(bhn * 4);
 }
 
 BwdWorkspace carve_bwd(void* ws, const Grid& g) {
@@ -119,7 +125,7 @@ BwdWorkspace carve_bwd(void* ws, const Grid& g) {
   const size_t bhn = static_cast<size_t>(g.B) * g.h * g.n;
   BwdWorkspace w;
   w.status = reinterpret_cast<uint32_t*>(b);
-  b += kCtrlBytes;
+  b += ctrl_bytes(g);
   w.dq_acc = reinterpret_cast<float*>(b);
   b += align256(bhn * g.d * 4);
   w.dk_acc = reinterpret_cast<float*>(b);
@@ -196,29 +202,39 @@ bool short_eligible(const squad_params_t* prm, const Grid& g, const PassGeom& p)
   return prm->dtype == SQUAD_BF16 && g.d == 128 && p.kind != kFull && p.seq_len <= 256 && p.n_chunks == 1;
 }
 
-// One attention pass: out = softmax(scale q k^T) v over the sequences of `kind`.
+bool fill_short_pass(ShortPass& sp, const Grid& g, int kind, const void* q, const void* k, const void* v, void* out,
+                     float* lse) {
+  sp.p = make_geom(g, kind, 256);
+  sp.variant = kind == kGlobal ? kSlotBoxVariant : 0;
+  sp.lse = lse;
+  return encode_pass_map(&sp.tm_q, q, g, sp.p, sp.variant) && encode_pass_map(&sp.tm_k, k, g, sp.p, sp.variant) &&
+         encode_pass_map(&sp.tm_v, v, g, sp.p, sp.variant) && encode_pass_map(&sp.tm_o, out, g, sp.p, sp.variant);
+}
+
+squad_status_t launch_short_args(ShortArgs& a, float scale, uint32_t* status, uint32_t* work, uint32_t* done,
+                                 cudaStream_t stream) {
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.status = status;
+  a.work = work;
+  a.done = done;
+  a.timeout_ns = kWaitTimeoutNs;
+  const int sms = num_sms_current();
+  if (sms <= 0) return SQUAD_ERR_CUDA;
+  return launch_short(a, sms, stream) == cudaSuccess ? SQUAD_OK : SQUAD_ERR_CUDA;
+}
+
+// One attention pass: out = softmax(scale q k^T) v over the sequences of `kind`. `work` is a zeroed
+// counter for the persistent short-sequence kernel.
 squad_status_t run_pass(const squad_params_t* prm, const Grid& g, int kind, float scale, const void* q,
                         const void* k, const void* v, bool v_bf16, void* out, float* lse, uint32_t* status,
-                        cudaStream_t stream) {
-  const PassGeom ps = make_geom(g, kind, 256);
-  if (short_eligible(prm, g, ps) && v_bf16) {
-    ShortPassArgs a;
+                        uint32_t* work, cudaStream_t stream) {
+  if (short_eligible(prm, g, make_geom(g, kind, 256)) && v_bf16 && work != nullptr) {
+    ShortArgs a;
     std::memset(&a, 0, sizeof(a));
     a.g = g;
-    a.p = ps;
-    a.global_variant = kind == kGlobal ? kSlotBoxVariant : 0;
-    if (short_pass_plan(a)) {
-      if (!encode_pass_map(&a.tm_q, q, g, ps, a.global_variant) || !encode_pass_map(&a.tm_k, k, g, ps, a.global_variant) ||
-          !encode_pass_map(&a.tm_v, v, g, ps, a.global_variant) || !encode_pass_map(&a.tm_o, out, g, ps, a.global_variant))
-        return SQUAD_ERR_CUDA;
-      a.lse = lse;
-      a.scale_log2 = scale * 1.4426950408889634f;
-      a.status = status;
-      a.timeout_ns = kWaitTimeoutNs;
-      const int sms = num_sms_current();
-      if (sms <= 0) return SQUAD_ERR_CUDA;
-      return launch_short_pass(a, sms, stream) == cudaSuccess ? SQUAD_OK : SQUAD_ERR_CUDA;
-    }
+    a.n_passes = 1;
+    if (!fill_short_pass(a.pass[0], g, kind, q, k, v, out, lse)) return SQUAD_ERR_CUDA;
+    if (short_plan(a)) return launch_short_args(a, scale, status, work, nullptr, stream);
   }
   const PassGeom p = make_geom(g, kind);
   if (tc_eligible(prm, g, p) && v_bf16) {
@@ -313,13 +329,26 @@ squad_status_t squad_attn_fwd(const squad_params_t* p, const void* q, const void
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   const size_t eb = elem_bytes(p);
   FwdWorkspace ws = carve_fwd(workspace, g, eb);
-  if (cudaMemsetAsync(ws.status, 0, kCtrlBytes, stream) != cudaSuccess) return SQUAD_ERR_CUDA;
+  if (cudaMemsetAsync(ws.status, 0, ctrl_bytes(g), stream) != cudaSuccess) return SQUAD_ERR_CUDA;
   const bool bf16 = p->dtype == SQUAD_BF16;
   const int first = p->order == SQUAD_LOCAL_THEN_GLOBAL ? kLocal : kGlobal;
   const int second = p->order == SQUAD_LOCAL_THEN_GLOBAL ? kGlobal : kLocal;
-  st = run_pass(p, g, first, scale, q, k, v, bf16, ws.o1, ws.lse1, ws.status, stream);
+  uint32_t* ctrl = ws.status;
+  if (short_eligible(p, g, make_geom(g, first, 256)) && short_eligible(p, g, make_geom(g, second, 256))) {
+    // Both passes in one persistent launch; the second pass reads each head's first-pass output
+    // (its values) once all of that head's first-pass units are stored.
+    ShortArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.g = g;
+    a.n_passes = 2;
+    if (!fill_short_pass(a.pass[0], g, first, q, k, v, ws.o1, ws.lse1) ||
+        !fill_short_pass(a.pass[1], g, second, q, k, ws.o1, o, ws.lse2))
+      return SQUAD_ERR_CUDA;
+    if (short_plan(a)) return launch_short_args(a, scale, ctrl, ctrl + 1, ctrl + kCtrlFixedWords, stream);
+  }
+  st = run_pass(p, g, first, scale, q, k, v, bf16, ws.o1, ws.lse1, ctrl, ctrl + 2, stream);
   if (st != SQUAD_OK) return st;
-  return run_pass(p, g, second, scale, q, k, ws.o1, bf16, o, ws.lse2, ws.status, stream);
+  return run_pass(p, g, second, scale, q, k, ws.o1, bf16, o, ws.lse2, ctrl, ctrl + 3, stream);
 }
 
 squad_status_t squad_attn_fwd_status(const squad_params_t* p, const void* workspace, squad_stream_t stream_) {
@@ -352,7 +381,7 @@ squad_status_t squad_attn_bwd(const squad_params_t* p, const void* q, const void
   const bool bf16 = p->dtype == SQUAD_BF16;
   FwdWorkspace fw = carve_fwd(const_cast<void*>(fwd_workspace), g, eb);
   BwdWorkspace bw = carve_bwd(bwd_workspace, g);
-  if (cudaMemsetAsync(bw.status, 0, kCtrlBytes, stream) != cudaSuccess) return SQUAD_ERR_CUDA;
+  if (cudaMemsetAsync(bw.status, 0, ctrl_bytes(g), stream) != cudaSuccess) return SQUAD_ERR_CUDA;
   const int first = p->order == SQUAD_LOCAL_THEN_GLOBAL ? kLocal : kGlobal;
   const int second = p->order == SQUAD_LOCAL_THEN_GLOBAL ? kGlobal : kLocal;
 
@@ -405,7 +434,7 @@ squad_status_t full_attn_fwd(const squad_params_t* p, const void* q, const void*
   if (lse_or_null != nullptr && !aligned(lse_or_null, 4)) return SQUAD_ERR_INVALID_ARG;
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   const bool bf16 = p->dtype == SQUAD_BF16;
-  return run_pass(p, g, kFull, scale, q, k, v, bf16, o, lse_or_null, nullptr, stream);
+  return run_pass(p, g, kFull, scale, q, k, v, bf16, o, lse_or_null, nullptr, nullptr, stream);
 }
 
 }  // extern "C"

@@ -1,24 +1,36 @@
-// Tensor-core attention over sequences of at most 256 tokens, sm_100a: one SQuad pass (local windows
-// or global slots, paper §3.2) per launch, every sequence handled in one block.
+// Tensor-core attention over sequences of at most 256 tokens, sm_100a: one SQuad pass, or both passes
+// fused, in one persistent launch (paper §3.2: the local pass inside windows, then the global pass
+// across windows with the local output as values).
 //
-// Each of Q, K, V of a sequence arrives as one TMA box (the whole window, or the whole slot across
-// all windows) in a slot of a shared-memory ring; S = Q K^T is one tcgen05.mma per 16-deep K step
-// with N = the sequence length rounded up to 16 (<= 256), so the softmax needs no running maximum.
+// Each of Q, K, V of a sequence arrives as one TMA box (the whole window, or the whole slot across all
+// windows) in a shared-memory ring; S = Q K^T is one tcgen05.mma per 16-deep K step with N = the
+// sequence length rounded up to 16 (<= 256), so the softmax needs no running maximum.
 //
-// CTA organisation (persistent, one CTA per SM, 352 threads):
+// CTA organisation (one CTA per SM, 352 threads):
 //   warps 0-3   softmax warpgroup 0 (TMEM lanes 0-127 of its S / O)
 //   warps 4-7   softmax warpgroup 1
-//   warp 8      TMA producer       warp 9  TMEM allocator and MMA issuer     warp 10  TMA store issuer
-// A work unit is either one sequence of 129-256 tokens (its two 128-row query tiles go to the two
-// warpgroups and share K and V) or two sequences of at most 128 tokens (one per warpgroup).
-// Per unit the producer fills ring slots in the order Q, K (per tile) then V (per tile); Q and K slots
-// are released as soon as the S products that read them complete, the V slot when the output stored
-// through it has left: the softmax warps stage O (normalised, bf16) in the V slot after PV has read
-// it, and the store warp writes it back with a TMA store of the same box. So the next unit's loads
-// overlap this unit's softmax and epilogue.
+//   warp 8      scheduler + TMA producer   warp 9  TMEM allocator + MMA issuer   warp 10  TMA stores
+// Work units are claimed dynamically (an atomic counter) and handed to the other warps through a small
+// queue in shared memory. A unit is either one sequence of 129-256 tokens (its two 128-row query tiles
+// go to the two warpgroups and share K and V) or two sequences of at most 128 tokens (one per
+// warpgroup).
+//
+// Fused passes: the unit order is L(0) L(1) .. L(lag-1), then L(k) G(k-lag) for each head k, then the
+// remaining G: a head's second-pass units trail its first-pass units by `lag` heads, so the second
+// pass re-reads that head's Q, K and first-pass output from L2. Before loading the values of a
+// second-pass unit (the first pass's output), the producer waits, bounded, until every first-pass unit
+// of that head has been stored (a per-head counter the store warp increments with release semantics
+// after its TMA stores complete).
+//
+// Ring: allocations (one per Q, K or V box) get consecutive offsets in a byte ring; every warp derives
+// the same offsets from the same unit sequence. Q and K allocations are released when the S products
+// that read them complete, a V allocation when the output staged in it has been stored: the softmax
+// warps write O (normalised, bf16) into the V allocation after PV has read it, and the store warp
+// writes it back with a TMA store of the sequence's box. So the next units' loads overlap this unit's
+// softmax and epilogue.
 // Tensor memory per warpgroup (256 columns): S in [0, N), P (bf16 pairs) over [0, N/2), and O in
-// [128, 256) when N <= 128, else in [N/2, N/2 + 128) over the consumed scores; in the second case the
-// next unit's S waits until the epilogue has read O.
+// [128, 256) when N <= 128, else in [N/2, N/2 + 128) over consumed scores; a unit's S then waits until
+// the warpgroup has read the previous unit's O.
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
@@ -32,96 +44,163 @@ namespace {
 
 constexpr int kThreads = 352;
 constexpr int kWarpProducer = 8, kWarpMma = 9, kWarpStore = 10;
-constexpr int kMaxSlots = 8;
+constexpr int kND = 16;   // ring allocations in flight (full/empty barrier pairs)
+constexpr int kQ = 4;     // unit queue entries
 constexpr uint32_t kSmemLimit = 232448;
 
 struct Bars {
-  uint64_t full[kMaxSlots], empty[kMaxSlots];
+  uint64_t full[kND], empty[kND];
+  uint64_t qf[kQ], qe[kQ];
   uint64_t s_full[2], p_full[2], o_full[2], o_free[2], staged[2];
   uint64_t drain;
+  int unit_q[kQ];
   uint32_t tmem_base;
   uint32_t abort;
 };
-constexpr uint32_t kBarBytes = 256;
+constexpr uint32_t kBarBytes = 512;
 static_assert(sizeof(Bars) <= kBarBytes, "barrier block");
 
 __device__ __forceinline__ int round16(int x) { return (x + 15) & ~15; }
 
-// The sequences and ring allocations of one work unit. Allocation indices count every slot fill of
-// the launch in order; slot = index % n_slots.
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.global.acquire.gpu.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void red_release_gpu_add(uint32_t* p, uint32_t v) {
+  asm volatile("fence.acq_rel.gpu;\n\tred.relaxed.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// One work unit: its pass, head, sequences and ring allocations.
 struct Unit {
-  int nw;            // query tiles in the unit (1 or 2)
-  bool shared;       // both tiles belong to one sequence (shared K and V)
-  int bh[2], sigma[2];
-  uint32_t q[2], k[2], v[2];
-  uint32_t n_alloc;  // allocations this unit makes
+  int pass, bh, nw;
+  bool shared;       // both query tiles belong to one sequence (shared K and V)
+  int sigma[2];
+  uint32_t q[2], k[2], v[2];        // allocation indices
+  uint32_t qo[2], ko[2], vo[2];     // their byte offsets in the ring
+  uint32_t qvs[2], kvs[2], vvs[2];  // their virtual starts (producer bookkeeping)
 };
 
-__device__ __forceinline__ Unit plan_unit(const Grid& g, const PassGeom& p, int unit, uint32_t base) {
-  Unit u;
-  const int total = g.B * g.h * p.n_seq;
-  const bool two_tiles = p.seq_len > 128;
-  int seq[2];
-  if (two_tiles) {
-    u.nw = 2;
-    u.shared = true;
-    seq[0] = seq[1] = unit;
-    u.q[0] = u.q[1] = base;
-    u.k[0] = u.k[1] = base + 1;
-    u.v[0] = u.v[1] = base + 2;
-    u.n_alloc = 3;
-  } else {
-    u.shared = false;
-    seq[0] = 2 * unit;
-    seq[1] = 2 * unit + 1;
-    u.nw = seq[1] < total ? 2 : 1;
-    u.q[0] = base;
-    u.k[0] = base + 1;
-    if (u.nw == 2) {
-      u.q[1] = base + 2;
-      u.k[1] = base + 3;
-      u.v[0] = base + 4;
-      u.v[1] = base + 5;
-      u.n_alloc = 6;
-    } else {
-      u.q[1] = u.k[1] = u.v[1] = 0;
-      u.v[0] = base + 2;
-      u.n_alloc = 3;
+// Allocation cursor over the byte ring, identical in every warp.
+struct Cursor {
+  uint32_t ai = 0, vpos = 0, phys = 0;
+  __device__ __forceinline__ void take(uint32_t sz, uint32_t ring, uint32_t& idx, uint32_t& off, uint32_t& vstart) {
+    if (phys + sz > ring) {
+      vpos += ring - phys;
+      phys = 0;
     }
+    idx = ai++;
+    off = phys;
+    vstart = vpos;
+    phys += sz;
+    vpos += sz;
   }
-  for (int w = 0; w < 2; ++w) {
-    const int sq = seq[w] < total ? seq[w] : seq[0];
-    u.bh[w] = static_cast<int>(fdiv(static_cast<uint32_t>(sq), p.f_per_bh));
-    u.sigma[w] = sq - u.bh[w] * p.n_seq;
+};
+
+// Global unit index -> (pass, head, unit within head).
+__device__ __forceinline__ void decode_unit(const ShortArgs& a, int U, int& pass, int& bh, int& j) {
+  const int H = a.g.B * a.g.h;
+  const int n0 = a.pass[0].units_per_head;
+  if (a.n_passes == 1) {
+    bh = static_cast<int>(fdiv(static_cast<uint32_t>(U), a.f_u0));
+    pass = 0;
+    j = U - bh * n0;
+    return;
+  }
+  const int n1 = a.pass[1].units_per_head;
+  const int lag = a.lag;
+  const int lead = lag * n0;                 // blocks 0..lag-1: first-pass units only
+  const int mid = lead + (H - lag) * (n0 + n1);
+  if (U < lead) {
+    bh = static_cast<int>(fdiv(static_cast<uint32_t>(U), a.f_u0));
+    pass = 0;
+    j = U - bh * n0;
+  } else if (U < mid) {
+    const int r = U - lead;
+    const int k = static_cast<int>(fdiv(static_cast<uint32_t>(r), a.f_u01));
+    const int o = r - k * (n0 + n1);
+    if (o < n0) {
+      pass = 0;
+      bh = lag + k;
+      j = o;
+    } else {
+      pass = 1;
+      bh = k;
+      j = o - n0;
+    }
+  } else {
+    const int r = U - mid;
+    const int k = static_cast<int>(fdiv(static_cast<uint32_t>(r), a.f_u1));
+    pass = 1;
+    bh = H - lag + k;
+    j = r - k * n1;
+  }
+}
+
+__device__ __forceinline__ Unit plan_unit(const ShortArgs& a, int U, Cursor& cur, uint32_t ring) {
+  Unit u;
+  int j;
+  decode_unit(a, U, u.pass, u.bh, j);
+  const PassGeom& p = a.pass[u.pass].p;
+  const uint32_t sz = a.pass[u.pass].alloc_bytes;
+  u.shared = p.seq_len > 128;
+  if (u.shared) {
+    u.nw = 2;
+    u.sigma[0] = u.sigma[1] = j;
+    cur.take(sz, ring, u.q[0], u.qo[0], u.qvs[0]);
+    cur.take(sz, ring, u.k[0], u.ko[0], u.kvs[0]);
+    cur.take(sz, ring, u.v[0], u.vo[0], u.vvs[0]);
+    u.q[1] = u.q[0]; u.qo[1] = u.qo[0]; u.qvs[1] = u.qvs[0];
+    u.k[1] = u.k[0]; u.ko[1] = u.ko[0]; u.kvs[1] = u.kvs[0];
+    u.v[1] = u.v[0]; u.vo[1] = u.vo[0]; u.vvs[1] = u.vvs[0];
+  } else {
+    u.sigma[0] = 2 * j;
+    u.sigma[1] = 2 * j + 1;
+    u.nw = u.sigma[1] < p.n_seq ? 2 : 1;
+    for (int w = 0; w < u.nw; ++w) {
+      cur.take(sz, ring, u.q[w], u.qo[w], u.qvs[w]);
+      cur.take(sz, ring, u.k[w], u.ko[w], u.kvs[w]);
+    }
+    for (int w = 0; w < u.nw; ++w) cur.take(sz, ring, u.v[w], u.vo[w], u.vvs[w]);
+    if (u.nw == 1) {
+      u.sigma[1] = u.sigma[0];
+      u.q[1] = u.q[0]; u.qo[1] = u.qo[0]; u.qvs[1] = u.qvs[0];
+      u.k[1] = u.k[0]; u.ko[1] = u.ko[0]; u.kvs[1] = u.kvs[0];
+      u.v[1] = u.v[0]; u.vo[1] = u.vo[0]; u.vvs[1] = u.vvs[0];
+    }
   }
   return u;
 }
 
+__device__ __forceinline__ int total_units(const ShortArgs& a) {
+  const int H = a.g.B * a.g.h;
+  return H * (a.pass[0].units_per_head + (a.n_passes == 2 ? a.pass[1].units_per_head : 0));
+}
+
 }  // namespace
 
-__global__ void __launch_bounds__(kThreads, 1) short_pass_kernel(const __grid_constant__ ShortPassArgs a) {
+__global__ void __launch_bounds__(kThreads, 1) short_kernel(const __grid_constant__ ShortArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const uint32_t ring_bytes = static_cast<uint32_t>(a.n_slots) * a.slot_bytes;
-  Bars* bars = reinterpret_cast<Bars*>(ring + ring_bytes + a.guard_bytes);
+  const uint32_t RB = a.ring_bytes;
+  Bars* bars = reinterpret_cast<Bars*>(ring + RB + a.guard_bytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const PassGeom& p = a.p;
   const Grid& g = a.g;
-  const int NS = a.n_slots;
-  const int s_len = p.seq_len;
-  const int N = round16(s_len);
-  const bool o_overlap = N > 128;
-  const uint32_t o_off = o_overlap ? static_cast<uint32_t>(N / 2) : 128u;
+  const int n_total = total_units(a);
 
-  // Zero the ring and guard once: rows past a sequence inside a slot (and past the ring) are read by
-  // the MMAs and must hold finite values.
-  for (uint32_t i = threadIdx.x; i < (ring_bytes + a.guard_bytes) / 16; i += kThreads)
+  // Zero the ring and guard once: rows past a sequence inside an allocation (and past the ring) are
+  // read by the MMAs and must hold finite values.
+  for (uint32_t i = threadIdx.x; i < (RB + a.guard_bytes) / 16; i += kThreads)
     reinterpret_cast<uint4*>(ring)[i] = make_uint4(0, 0, 0, 0);
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kMaxSlots; ++i) {
+    for (int i = 0; i < kND; ++i) {
       mbar_init(&bars->full[i], 1);
       mbar_init(&bars->empty[i], 1);
+    }
+    for (int i = 0; i < kQ; ++i) {
+      mbar_init(&bars->qf[i], 1);
+      mbar_init(&bars->qe[i], 10);   // MMA issuer, store warp and the 8 softmax warps
     }
     for (int w = 0; w < 2; ++w) {
       mbar_init(&bars->s_full[w], 1);
@@ -135,10 +214,12 @@ __global__ void __launch_bounds__(kThreads, 1) short_pass_kernel(const __grid_co
     fence_mbar_init();
   }
   if (warp == kWarpProducer && lane == 0) {
-    prefetch_tmap(&a.tm_q);
-    prefetch_tmap(&a.tm_k);
-    prefetch_tmap(&a.tm_v);
-    prefetch_tmap(&a.tm_o);
+    for (int ps = 0; ps < a.n_passes; ++ps) {
+      prefetch_tmap(&a.pass[ps].tm_q);
+      prefetch_tmap(&a.pass[ps].tm_k);
+      prefetch_tmap(&a.pass[ps].tm_v);
+      prefetch_tmap(&a.pass[ps].tm_o);
+    }
   }
   if (warp == kWarpMma) {
     tmem_alloc(&bars->tmem_base, 512);
@@ -151,96 +232,153 @@ __global__ void __launch_bounds__(kThreads, 1) short_pass_kernel(const __grid_co
 
   const uint32_t tmem = bars->tmem_base;
   WaitCtl ctl{&bars->abort, a.status, a.timeout_ns};
-  const int total_seq = g.B * g.h * p.n_seq;
-  const int n_units = s_len > 128 ? total_seq : (total_seq + 1) / 2;
-  const uint32_t box_bytes = 2u * static_cast<uint32_t>(s_len) * 128u;
-  auto slot_ptr = [&](uint32_t alloc) { return ring + (alloc % static_cast<uint32_t>(NS)) * a.slot_bytes; };
+
+  // Next unit from the queue (consumers); returns false at the end of the work.
+  // (A failed wait counts as the end of the work.)
+  auto next_unit = [&](uint32_t& qi, int& U, bool arrive) -> bool {
+    const uint32_t e = qi % kQ;
+    U = mbar_wait(&bars->qf[e], (qi / kQ) & 1, ctl) ? *reinterpret_cast<volatile int*>(&bars->unit_q[e]) : n_total;
+    if (arrive) mbar_arrive(&bars->qe[e]);
+    ++qi;
+    return U < n_total;
+  };
 
   if (warp == kWarpProducer) {
-    // ------------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------------ scheduler + TMA producer
     if (lane == 0) {
-      uint32_t base = 0;
+      Cursor cur;
+      uint32_t tail = 0, vstart[kND];
+      uint32_t qi = 0;
       bool ok = true;
-      auto load = [&](const CUtensorMap* m, int bh, int sigma, uint32_t alloc) -> bool {
-        const uint32_t sl = alloc % static_cast<uint32_t>(NS);
-        if (alloc >= static_cast<uint32_t>(NS) &&
-            !mbar_wait(&bars->empty[sl], ((alloc / NS) + 1) & 1, ctl))
-          return false;
-        mbar_arrive_expect_tx(&bars->full[sl], box_bytes);
-        int c[5];
-        chunk_coords(g, p, a.global_variant, bh, sigma, 0, 0, c);
-        uint8_t* dst = slot_ptr(alloc);
-        tma_load_5d(dst, m, &bars->full[sl], c[0], c[1], c[2], c[3], c[4]);
-        tma_load_5d(dst + a.panel_bytes, m, &bars->full[sl], c[0] + 64, c[1], c[2], c[3], c[4]);
+      // Wait until allocation `idx`, virtual range [vs, vs + sz), may be filled. Its bytes were last used
+      // by virtual [vs - RB, vs + sz - RB): every live allocation starting before vs + sz - RB overlaps
+      // them, and live allocations start in increasing order, so release the oldest ones until the
+      // oldest starts at or after that point (or none is left). The allocation whose barriers it reuses
+      // (idx - kND) must be released too.
+      auto make_room = [&](uint32_t idx, uint32_t vs, uint32_t sz) -> bool {
+        while (tail < idx &&
+               (idx - tail >= static_cast<uint32_t>(kND) || (vs + sz > RB && vstart[tail % kND] < vs + sz - RB))) {
+          if (!mbar_wait(&bars->empty[tail % kND], (tail / kND) & 1, ctl)) return false;
+          ++tail;
+        }
+        vstart[idx % kND] = vs;
         return true;
       };
-      for (int unit = blockIdx.x; unit < n_units && ok; unit += gridDim.x) {
-        const Unit u = plan_unit(g, p, unit, base);
+      auto load = [&](const ShortPass& ps, const CUtensorMap* m, int bh, int sigma, uint32_t idx, uint32_t off,
+                      uint32_t vs) -> bool {
+        if (!make_room(idx, vs, ps.alloc_bytes)) return false;
+        uint64_t* fb = &bars->full[idx % kND];
+        mbar_arrive_expect_tx(fb, 2u * static_cast<uint32_t>(ps.p.seq_len) * 128u);
+        int c[5];
+        chunk_coords(g, ps.p, ps.variant, bh, sigma, 0, 0, c);
+        tma_load_5d(ring + off, m, fb, c[0], c[1], c[2], c[3], c[4]);
+        tma_load_5d(ring + off + ps.panel_bytes, m, fb, c[0] + 64, c[1], c[2], c[3], c[4]);
+        return true;
+      };
+      while (ok) {
+        // claim the next unit and publish it to the other warps
+        const uint32_t e = qi % kQ;
+        if (qi >= kQ && !mbar_wait(&bars->qe[e], ((qi / kQ) + 1) & 1, ctl)) break;
+        const int U = static_cast<int>(atomicAdd(a.work, 1u));
+        bars->unit_q[e] = U;
+        mbar_arrive(&bars->qf[e]);   // release: the entry is visible to the waiting warps
+        ++qi;
+        if (U >= n_total) break;
+        const Unit u = plan_unit(a, U, cur, RB);
+        const ShortPass& ps = a.pass[u.pass];
         const int nsrc = u.shared ? 1 : u.nw;
         for (int w = 0; w < nsrc && ok; ++w) {
-          ok = load(&a.tm_q, u.bh[w], u.sigma[w], u.q[w]);
-          if (ok) ok = load(&a.tm_k, u.bh[w], u.sigma[w], u.k[w]);
+          ok = load(ps, &ps.tm_q, u.bh, u.sigma[w], u.q[w], u.qo[w], u.qvs[w]);
+          if (ok) ok = load(ps, &ps.tm_k, u.bh, u.sigma[w], u.k[w], u.ko[w], u.kvs[w]);
         }
-        for (int w = 0; w < nsrc && ok; ++w) ok = load(&a.tm_v, u.bh[w], u.sigma[w], u.v[w]);
-        base += u.n_alloc;
+        if (ok && u.pass == 1) {
+          // values = the first pass's output for this head: wait until all of it is in memory
+          const uint32_t need = static_cast<uint32_t>(a.pass[0].units_per_head);
+          const uint32_t* cnt = &a.done[u.bh];
+          if (ld_acquire_gpu(cnt) < need) {
+            const uint64_t t0 = globaltimer_ns();
+            while (ld_acquire_gpu(cnt) < need) {
+              if (*ctl.abort || globaltimer_ns() - t0 > a.timeout_ns) {
+                record_timeout(ctl);
+                ok = false;
+                break;
+              }
+              __nanosleep(256);
+            }
+          }
+          fence_proxy_async_global();   // the TMA loads below must observe those stores
+        }
+        for (int w = 0; w < nsrc && ok; ++w) ok = load(ps, &ps.tm_v, u.bh, u.sigma[w], u.v[w], u.vo[w], u.vvs[w]);
+      }
+      if (!ok) {   // make sure the other warps see the end of the work
+        for (int i = 0; i < kQ; ++i) {
+          const uint32_t e = qi % kQ;
+          if (qi >= kQ) mbar_wait_drain(&bars->qe[e], ((qi / kQ) + 1) & 1, 20000000ull);
+          bars->unit_q[e] = n_total;
+          mbar_arrive(&bars->qf[e]);
+          ++qi;
+        }
       }
       // Let every load this thread issued land before the CTA can exit (bounded).
-      const uint32_t first = base > static_cast<uint32_t>(NS) ? base - NS : 0;
-      for (uint32_t i = first; i < base; ++i)
-        mbar_wait_drain(&bars->full[i % NS], (i / NS) & 1, 20000000ull);
+      const uint32_t first = cur.ai > static_cast<uint32_t>(kND) ? cur.ai - kND : 0;
+      for (uint32_t i = first; i < cur.ai; ++i) mbar_wait_drain(&bars->full[i % kND], (i / kND) & 1, 20000000ull);
     }
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc_s = idesc_bf16(128, N, false);
       const uint32_t idesc_pv = idesc_bf16(128, 128, true);
-      uint32_t base = 0, p_cnt[2] = {0, 0}, of_cnt[2] = {0, 0};
+      Cursor cur;
+      uint32_t qi = 0, p_cnt[2] = {0, 0}, wu[2] = {0, 0}, prev_ooff[2] = {0xFFFFFFFFu, 0xFFFFFFFFu};
+      int U;
       bool ok = true;
-      for (int unit = blockIdx.x; unit < n_units && ok; unit += gridDim.x) {
-        const Unit u = plan_unit(g, p, unit, base);
+      while (ok && next_unit(qi, U, true)) {
+        const Unit u = plan_unit(a, U, cur, RB);
+        const ShortPass& ps = a.pass[u.pass];
+        const int N = round16(ps.p.seq_len);
+        const uint32_t o_off = N > 128 ? static_cast<uint32_t>(N / 2) : 128u;
+        const uint32_t idesc_s = idesc_bf16(128, N, false);
         for (int w = 0; w < u.nw && ok; ++w) {
-          const bool first_user = w == 0 || !u.shared;
-          if (first_user) {
-            ok = mbar_wait(&bars->full[u.q[w] % NS], (u.q[w] / NS) & 1, ctl);
-            if (ok) ok = mbar_wait(&bars->full[u.k[w] % NS], (u.k[w] / NS) & 1, ctl);
+          if (w == 0 || !u.shared) {
+            ok = mbar_wait(&bars->full[u.q[w] % kND], (u.q[w] / kND) & 1, ctl);
+            if (ok) ok = mbar_wait(&bars->full[u.k[w] % kND], (u.k[w] / kND) & 1, ctl);
           }
-          if (ok && o_overlap && unit != static_cast<int>(blockIdx.x)) {
-            // the previous unit's epilogue must have read O, which overlaps this S
-            ok = mbar_wait(&bars->o_free[w], of_cnt[w] & 1, ctl);
-            ++of_cnt[w];
-          }
+          if (ok && prev_ooff[w] != 0xFFFFFFFFu && static_cast<uint32_t>(N) > prev_ooff[w])
+            ok = mbar_wait(&bars->o_free[w], (wu[w] - 1) & 1, ctl);   // previous O read before S overwrites it
           if (!ok) break;
           tc_fence_after();
-          const uint32_t qa = smem_u32(slot_ptr(u.q[w])) + (u.shared ? static_cast<uint32_t>(w) * 16384u : 0u);
-          const uint32_t ka = smem_u32(slot_ptr(u.k[w]));
+          const uint32_t qa = smem_u32(ring + u.qo[w]) + (u.shared ? static_cast<uint32_t>(w) * 16384u : 0u);
+          const uint32_t ka = smem_u32(ring + u.ko[w]);
           for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t off = (kk >> 2) * a.panel_bytes + (kk & 3) * 32;
+            const uint32_t off = (kk >> 2) * ps.panel_bytes + (kk & 3) * 32;
             umma_bf16_ss(tmem + 256 * w, sw128_desc(qa + off, 16, 1024), sw128_desc(ka + off, 16, 1024), idesc_s,
                          kk > 0);
           }
           umma_commit(&bars->s_full[w]);
           if (!u.shared || w == u.nw - 1) {
-            umma_commit(&bars->empty[u.q[w] % NS]);
-            umma_commit(&bars->empty[u.k[w] % NS]);
+            umma_commit(&bars->empty[u.q[w] % kND]);
+            umma_commit(&bars->empty[u.k[w] % kND]);
           }
         }
         for (int w = 0; w < u.nw && ok; ++w) {
           ok = mbar_wait(&bars->p_full[w], p_cnt[w] & 1, ctl);
           ++p_cnt[w];
-          if (ok && (w == 0 || !u.shared)) ok = mbar_wait(&bars->full[u.v[w] % NS], (u.v[w] / NS) & 1, ctl);
+          if (ok && (w == 0 || !u.shared)) ok = mbar_wait(&bars->full[u.v[w] % kND], (u.v[w] / kND) & 1, ctl);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t va = smem_u32(slot_ptr(u.v[w]));
+          const uint32_t va = smem_u32(ring + u.vo[w]);
           for (int kk = 0; kk < N / 16; ++kk)
-            umma_bf16_ts(tmem + 256 * w + o_off, tmem + 256 * w + kk * 8, sw128_desc(va + kk * 2048, a.panel_bytes, 1024),
-                         idesc_pv, kk > 0);
+            umma_bf16_ts(tmem + 256 * w + o_off, tmem + 256 * w + kk * 8,
+                         sw128_desc(va + kk * 2048, ps.panel_bytes, 1024), idesc_pv, kk > 0);
           if (!u.shared) umma_commit(&bars->o_full[w]);
         }
-        if (ok && u.shared) {   // both tiles read the one V slot: neither may overwrite it before both PVs end
+        if (ok && u.shared) {   // both tiles read the one V allocation: neither overwrites it before both PVs
           umma_commit(&bars->o_full[0]);
           umma_commit(&bars->o_full[1]);
         }
-        base += u.n_alloc;
+        for (int w = 0; w < u.nw; ++w) {
+          ++wu[w];
+          prev_ooff[w] = o_off;
+        }
       }
       umma_commit(&bars->drain);
       mbar_wait_drain(&bars->drain, 0, 20000000ull);
@@ -248,26 +386,35 @@ __global__ void __launch_bounds__(kThreads, 1) short_pass_kernel(const __grid_co
   } else if (warp == kWarpStore) {
     // ------------------------------------------------------------------ TMA store issuer
     if (lane == 0) {
-      uint32_t base = 0, st_cnt[2] = {0, 0};
+      Cursor cur;
+      uint32_t qi = 0, st_cnt[2] = {0, 0};
+      int U;
       bool ok = true;
-      for (int unit = blockIdx.x; unit < n_units && ok; unit += gridDim.x) {
-        const Unit u = plan_unit(g, p, unit, base);
+      while (ok && next_unit(qi, U, true)) {
+        const Unit u = plan_unit(a, U, cur, RB);
+        const ShortPass& ps = a.pass[u.pass];
         const int nseq = u.shared ? 1 : u.nw;
         for (int w = 0; w < u.nw && ok; ++w) {
           ok = mbar_wait(&bars->staged[w], st_cnt[w] & 1, ctl);
           ++st_cnt[w];
         }
-        for (int w = 0; w < nseq && ok; ++w) {
+        if (!ok) break;
+        for (int w = 0; w < nseq; ++w) {
           int c[5];
-          chunk_coords(g, p, a.global_variant, u.bh[w], u.sigma[w], 0, 0, c);
-          const uint8_t* src = slot_ptr(u.v[w]);
-          tma_store_5d(&a.tm_o, src, c[0], c[1], c[2], c[3], c[4]);
-          tma_store_5d(&a.tm_o, src + a.panel_bytes, c[0] + 64, c[1], c[2], c[3], c[4]);
-          bulk_commit_group();
+          chunk_coords(g, ps.p, ps.variant, u.bh, u.sigma[w], 0, 0, c);
+          const uint8_t* src = ring + u.vo[w];
+          tma_store_5d(&ps.tm_o, src, c[0], c[1], c[2], c[3], c[4]);
+          tma_store_5d(&ps.tm_o, src + ps.panel_bytes, c[0] + 64, c[1], c[2], c[3], c[4]);
         }
-        bulk_wait_read_all();   // the V slots may be refilled once their stores have read them
-        for (int w = 0; w < nseq; ++w) mbar_arrive(&bars->empty[u.v[w] % NS]);
-        base += u.n_alloc;
+        bulk_commit_group();
+        bulk_wait_read_all();   // the V allocations may be refilled once their stores have read them
+        for (int w = 0; w < nseq; ++w) mbar_arrive(&bars->empty[u.v[w] % kND]);
+        if (a.n_passes == 2 && u.pass == 0) {
+          // publish this head's progress once the output is in global memory
+          bulk_wait_all();
+          fence_proxy_async_global();
+          red_release_gpu_add(&a.done[u.bh], 1u);
+        }
       }
       bulk_wait_all();   // outputs written before the CTA exits
     }
@@ -277,20 +424,29 @@ __global__ void __launch_bounds__(kThreads, 1) short_pass_kernel(const __grid_co
     const int wq = warp & 3;
     const int row = wq * 32 + lane;
     const uint32_t t_s = tmem + 256 * wg + (static_cast<uint32_t>(wq * 32) << 16);
-    const uint32_t t_o = t_s + o_off;
     const float sl2 = a.scale_log2;
-    const int nchunk = (N + 63) / 64;
-    uint32_t s_cnt = 0, o_cnt = 0, base = 0;
+    Cursor cur;
+    uint32_t qi = 0, s_cnt = 0, o_cnt = 0;
+    int U;
     bool ok = true;
-    for (int unit = blockIdx.x; unit < n_units && ok; unit += gridDim.x) {
-      const Unit u = plan_unit(g, p, unit, base);
-      base += u.n_alloc;
-      if (wg >= u.nw) break;
-      const int row0 = u.shared ? 128 * wg : 0;           // first sequence row of this tile
+    while (ok) {
+      const bool more = next_unit(qi, U, false);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->qe[(qi - 1) % kQ]);
+      if (!more) break;
+      const Unit u = plan_unit(a, U, cur, RB);
+      if (wg >= u.nw) continue;
+      const ShortPass& ps = a.pass[u.pass];
+      const PassGeom& p = ps.p;
+      const int s_len = p.seq_len;
+      const int N = round16(s_len);
+      const uint32_t t_o = t_s + (N > 128 ? static_cast<uint32_t>(N / 2) : 128u);
+      const int nchunk = (N + 63) / 64;
+      const int row0 = u.shared ? 128 * wg : 0;   // first sequence row of this tile
       const int src = u.shared ? 0 : wg;
       int valid = s_len - row0;
       if (valid > 128) valid = 128;
-      const bool active = wq * 32 < valid;                 // warps of padding rows only keep the barriers
+      const bool active = wq * 32 < valid;        // warps of padding rows only keep the barriers
       ok = mbar_wait(&bars->s_full[wg], s_cnt & 1, ctl);
       ++s_cnt;
       if (!ok) break;
@@ -341,14 +497,14 @@ __global__ void __launch_bounds__(kThreads, 1) short_pass_kernel(const __grid_co
       tc_fence_before();
       mbar_arrive(&bars->p_full[wg]);
 
-      // epilogue: O / l -> bf16 into this tile's rows of the V slot (PV has finished reading it); the
-      // store warp writes the slot back with the sequence's box.
+      // epilogue: O / l -> bf16 into this tile's rows of the V allocation (PV has finished reading it);
+      // the store warp writes the allocation back with the sequence's box.
       ok = mbar_wait(&bars->o_full[wg], o_cnt & 1, ctl);
       ++o_cnt;
       if (!ok) break;
       tc_fence_after();
-      const int vrow = row0 + row;   // row within the V slot's panels
-      const uint32_t row_addr = smem_u32(slot_ptr(u.v[src])) + static_cast<uint32_t>(vrow) * 128u;
+      const int vrow = row0 + row;   // row within the V allocation's panels
+      const uint32_t row_addr = smem_u32(ring + u.vo[src]) + static_cast<uint32_t>(vrow) * 128u;
       const bool store_row = row < valid;
       const float inv_l = active ? 1.f / l : 0.f;
 #pragma unroll
@@ -364,16 +520,16 @@ __global__ void __launch_bounds__(kThreads, 1) short_pass_kernel(const __grid_co
         if (store_row) {
 #pragma unroll
           for (int c = 0; c < 8; ++c)
-            st_shared_v4(row_addr + h * a.panel_bytes + ((c ^ (vrow & 7)) << 4),
+            st_shared_v4(row_addr + h * ps.panel_bytes + ((c ^ (vrow & 7)) << 4),
                          pack_bf16x2(__uint_as_float(o[c * 8 + 0]) * inv_l, __uint_as_float(o[c * 8 + 1]) * inv_l),
                          pack_bf16x2(__uint_as_float(o[c * 8 + 2]) * inv_l, __uint_as_float(o[c * 8 + 3]) * inv_l),
                          pack_bf16x2(__uint_as_float(o[c * 8 + 4]) * inv_l, __uint_as_float(o[c * 8 + 5]) * inv_l),
                          pack_bf16x2(__uint_as_float(o[c * 8 + 6]) * inv_l, __uint_as_float(o[c * 8 + 7]) * inv_l));
         }
       }
-      if (a.lse != nullptr && store_row) {
+      if (ps.lse != nullptr && store_row) {
         const int tok = token_of(g, p, u.sigma[src], 0, vrow);
-        if (tok >= 0) a.lse[static_cast<size_t>(u.bh[src]) * g.n + tok] = (m + __log2f(l)) * 0.69314718055994531f;
+        if (tok >= 0) ps.lse[static_cast<size_t>(u.bh) * g.n + tok] = (m + __log2f(l)) * 0.69314718055994531f;
       }
       fence_proxy_async_smem();   // staging writes -> visible to the TMA store (async proxy)
       __syncwarp();
@@ -388,40 +544,55 @@ __global__ void __launch_bounds__(kThreads, 1) short_pass_kernel(const __grid_co
   if (warp == kWarpMma) tmem_dealloc(tmem, 512);
 }
 
-bool short_pass_plan(ShortPassArgs& a) {
-  const int s = a.p.seq_len;
-  if (s < 1 || s > 256 || a.p.n_chunks != 1 || a.g.d != 128) return false;
-  const uint32_t rows8 = static_cast<uint32_t>((s + 7) & ~7);
-  a.panel_bytes = rows8 * 128u;
-  a.slot_bytes = 2u * a.panel_bytes;
-  // Past a slot's end the MMAs read at most: the second 128-row query tile of a 256-row tile pair
-  // (or the only 128-row tile), and the K/V rows up to the sequence length rounded to 16.
-  const uint32_t tile_span = s > 128 ? 32768u : 16384u;
-  uint32_t guard = tile_span > a.panel_bytes ? tile_span - a.panel_bytes : 0u;
-  if (guard < 2048u) guard = 2048u;
+bool short_plan(ShortArgs& a) {
+  if (a.n_passes < 1 || a.n_passes > 2 || a.g.d != 128) return false;
+  uint32_t guard = 2048u, max_alloc = 0u;
+  for (int i = 0; i < a.n_passes; ++i) {
+    ShortPass& ps = a.pass[i];
+    const int s = ps.p.seq_len;
+    if (s < 1 || s > 256 || ps.p.n_chunks != 1) return false;
+    const uint32_t rows8 = static_cast<uint32_t>((s + 7) & ~7);
+    ps.panel_bytes = rows8 * 128u;
+    ps.alloc_bytes = 2u * ps.panel_bytes;
+    ps.units_per_head = s > 128 ? ps.p.n_seq : (ps.p.n_seq + 1) / 2;
+    // Past an allocation's end the MMAs read at most the second 128-row query tile of a 256-row pair
+    // (or the only 128-row tile), and K/V rows up to the sequence length rounded to 16.
+    const uint32_t tile_span = s > 128 ? 32768u : 16384u;
+    const uint32_t over = tile_span > ps.panel_bytes ? tile_span - ps.panel_bytes : 0u;
+    if (over > guard) guard = over;
+    if (ps.alloc_bytes > max_alloc) max_alloc = ps.alloc_bytes;
+  }
   a.guard_bytes = (guard + 1023u) & ~1023u;
   const uint32_t fixed = 1024u + a.guard_bytes + kBarBytes;
-  int n = static_cast<int>((kSmemLimit - fixed) / a.slot_bytes);
-  if (n > kMaxSlots) n = kMaxSlots;
-  const int need = s > 128 ? 3 : 6;   // slots one unit holds at once
-  if (n < need) return false;
-  a.n_slots = n;
-  a.smem_bytes = fixed + static_cast<uint32_t>(n) * a.slot_bytes;
+  a.ring_bytes = ((kSmemLimit - fixed) / 1024u) * 1024u;
+  // One unit holds up to 6 allocations (or 3 for a shared pair) at once.
+  for (int i = 0; i < a.n_passes; ++i) {
+    const uint32_t need = (a.pass[i].p.seq_len > 128 ? 3u : 6u) * a.pass[i].alloc_bytes;
+    if (need + max_alloc > a.ring_bytes) return false;   // + max_alloc: room lost to a wrap
+  }
+  a.smem_bytes = fixed + a.ring_bytes;
+  const int H = a.g.B * a.g.h;
+  a.lag = a.n_passes == 2 ? (H < 2 ? H : 2) : 0;
+  a.f_u0 = make_fastdiv(static_cast<uint32_t>(a.pass[0].units_per_head));
+  if (a.n_passes == 2) {
+    a.f_u1 = make_fastdiv(static_cast<uint32_t>(a.pass[1].units_per_head));
+    a.f_u01 = make_fastdiv(static_cast<uint32_t>(a.pass[0].units_per_head + a.pass[1].units_per_head));
+  }
   return true;
 }
 
-cudaError_t launch_short_pass(const ShortPassArgs& args, int num_sms, cudaStream_t stream) {
+cudaError_t launch_short(const ShortArgs& args, int num_sms, cudaStream_t stream) {
   static bool configured = false;
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(short_pass_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
+    cudaError_t e = cudaFuncSetAttribute(short_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  const int total_seq = args.g.B * args.g.h * args.p.n_seq;
-  const int n_units = args.p.seq_len > 128 ? total_seq : (total_seq + 1) / 2;
+  const int H = args.g.B * args.g.h;
+  const int n_units = H * (args.pass[0].units_per_head + (args.n_passes == 2 ? args.pass[1].units_per_head : 0));
   const int grid = n_units < num_sms ? n_units : num_sms;
   if (grid < 1) return cudaSuccess;
-  short_pass_kernel<<<grid, kThreads, args.smem_bytes, stream>>>(args);
+  short_kernel<<<grid, kThreads, args.smem_bytes, stream>>>(args);
   return cudaGetLastError();
 }
 
