@@ -24,6 +24,10 @@ constexpr int kAbiVersion = 1;
 // Control block at the start of a workspace (zeroed by every call): word 0 the device status, words
 // 1-3 work counters of the persistent kernels, then one counter per (b, head) for the fused passes.
 constexpr size_t kCtrlFixedWords = 4;
+// Run both passes of a short-sequence problem in one persistent launch (second pass trailing the first
+// by two heads, reading it from L2). Off until that schedule beats two back-to-back launches: its ring
+// cannot yet hold a unit's boxes while the next unit's load, so consecutive units barely overlap.
+constexpr bool kFusePasses = false;
 constexpr unsigned long long kWaitTimeoutNs = 1000000000ull;   // 1 s per device-side wait
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -334,7 +338,7 @@ squad_status_t squad_attn_fwd(const squad_params_t* p, const void* q, const void
   const int first = p->order == SQUAD_LOCAL_THEN_GLOBAL ? kLocal : kGlobal;
   const int second = p->order == SQUAD_LOCAL_THEN_GLOBAL ? kGlobal : kLocal;
   uint32_t* ctrl = ws.status;
-  if (short_eligible(p, g, make_geom(g, first, 256)) && short_eligible(p, g, make_geom(g, second, 256))) {
+  if (kFusePasses && short_eligible(p, g, make_geom(g, first, 256)) && short_eligible(p, g, make_geom(g, second, 256))) {
     // Both passes in one persistent launch; the second pass reads each head's first-pass output
     // (its values) once all of that head's first-pass units are stored.
     ShortArgs a;
