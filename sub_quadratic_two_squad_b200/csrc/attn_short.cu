@@ -247,7 +247,7 @@ __global__ void __launch_bounds__(kThreads, 1) short_kernel(const __grid_constan
     // ------------------------------------------------------------------ scheduler + TMA producer
     if (lane == 0) {
       Cursor cur;
-      uint32_t tail = 0, vstart[kND];
+      uint32_t tail = 0, vstart[kND] = {};
       uint32_t qi = 0;
       bool ok = true;
       // Wait until allocation `idx`, virtual range [vs, vs + sz), may be filled. Its bytes were last used

@@ -70,12 +70,6 @@ __device__ __forceinline__ TileRef decode_tile(const PassGeom& p, int tile) {
 
 __device__ __forceinline__ int round16(int x) { return (x + 15) & ~15; }
 
-// Physical byte offset of the 16-byte chunk `ch` (0..15 over 128 columns) of row `row` in a 2-panel
-// 128-byte-swizzled tile: the layout TMA writes with SWIZZLE_128B and the MMA reads.
-__device__ __forceinline__ uint32_t sw_off(int row, int ch) {
-  return (ch >> 3) * kPanel + row * 128 + (((ch & 7) ^ (row & 7)) << 4);
-}
-
 // Order of the K/V block loads of one unit (the producer issues them in this order, the MMA issuer
 // finds each one's ring position from it): K0, K1, V0, K2, V1, ..., K(nb-1), V(nb-2), V(nb-1).
 __device__ __forceinline__ int pos_k(int b) { return b == 0 ? 0 : 2 * b - 1; }
