@@ -111,6 +111,29 @@ SQUAD_API squad_status_t squad_attn_bwd(const squad_params_t* p, const void* q, 
 SQUAD_API squad_status_t full_attn_fwd(const squad_params_t* p, const void* q, const void* k, const void* v,
                              void* o, float* lse_or_null, squad_stream_t stream);
 
+/* Largest workspace squad_attn_fwd_noalloc can provide: 128 MiB (one Wan-2.2-5B-shaped block,
+ * B = 1, h = 24, n = 18480, d = 128 in bf16, needs about 117 MB). */
+#define SQUAD_NOALLOC_MAX_WORKSPACE_BYTES (128u * 1024u * 1024u)
+
+/* squad_attn_fwd without a caller-provided workspace, for callers that cannot allocate device memory:
+ * code running inside a framework or engine that owns the whole device memory pool (a cudaMalloc
+ * there fails or fragments the pool), latency-critical loops where an allocation's synchronisation
+ * is not acceptable, and plugins that only receive the input and output tensors. The paper has no
+ * counterpart: this is a deployment variant of squad_attn_fwd with the same arguments minus the
+ * workspace, and the same results.
+ *
+ * The scratch is a file-scope device array of SQUAD_NOALLOC_MAX_WORKSPACE_BYTES in this library,
+ * which every GPU that loads the library holds until the process exits. It is shared by every call:
+ * calls that may overlap on the GPU (different streams, or different host threads, without ordering
+ * between them) race on it and must be serialised by the caller. Each call zeroes what must start at
+ * zero. The first call on a device looks up the array's device address (once per device, with that
+ * device current); make that first call before any stream capture on the device. The LSEs and the
+ * device status word of this entry point stay inside the scratch and are not exposed.
+ * Returns SQUAD_ERR_UNSUPPORTED, before launching anything, when squad_attn_fwd_workspace_bytes(p)
+ * exceeds SQUAD_NOALLOC_MAX_WORKSPACE_BYTES. It allocates nothing (no cudaMalloc or cudaFree). */
+SQUAD_API squad_status_t squad_attn_fwd_noalloc(const squad_params_t* p, const void* q, const void* k,
+                                                const void* v, void* o, squad_stream_t stream);
+
 /* FLOPs of one call, from the paper's cost model (appendix "Conformance to the theoretical curves
  * is quantitative"): 4 B h d (n w + n^2/w) for SQuad, 4 B h d n^2 for full attention. */
 SQUAD_API double squad_attn_flops(const squad_params_t* p);

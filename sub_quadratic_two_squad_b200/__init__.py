@@ -13,6 +13,7 @@ from .api import (  # noqa: F401
     squad_attn_bwd_workspace_bytes,
     squad_attn_flops,
     squad_attn_fwd,
+    squad_attn_fwd_noalloc,
     squad_attn_fwd_status,
     squad_attn_fwd_workspace_bytes,
 )

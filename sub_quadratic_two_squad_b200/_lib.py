@@ -10,6 +10,7 @@ LIB_PATH = os.path.join(PKG_DIR, "libsquad_attn.so")
 SQUAD_OK, SQUAD_ERR_INVALID_ARG, SQUAD_ERR_UNSUPPORTED, SQUAD_ERR_CUDA, SQUAD_ERR_TIMEOUT = range(5)
 SQUAD_BF16, SQUAD_FP32 = 0, 1
 SQUAD_LOCAL_THEN_GLOBAL, SQUAD_GLOBAL_THEN_LOCAL = 0, 1
+SQUAD_NOALLOC_MAX_WORKSPACE_BYTES = 128 * 1024 * 1024
 
 # Every symbol include/squad_attn.h declares, with (restype, argtypes).
 _VP = ctypes.c_void_p
@@ -30,6 +31,7 @@ SIGNATURES = {
     "squad_attn_bwd_workspace_bytes": (ctypes.c_size_t, [_PP]),
     "squad_attn_bwd": (ctypes.c_int, [_PP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
     "full_attn_fwd": (ctypes.c_int, [_PP, _VP, _VP, _VP, _VP, _VP, _VP]),
+    "squad_attn_fwd_noalloc": (ctypes.c_int, [_PP, _VP, _VP, _VP, _VP, _VP]),
     "squad_attn_flops": (ctypes.c_double, [_PP]),
     "full_attn_flops": (ctypes.c_double, [_PP]),
     "squad_status_string": (ctypes.c_char_p, [ctypes.c_int]),

@@ -84,6 +84,18 @@ def squad_attn_fwd(q, k, v, grid, window, order="local_then_global", scale=None,
     return out, workspace
 
 
+def squad_attn_fwd_noalloc(q, k, v, grid, window, order="local_then_global", scale=None, out=None, stream=None):
+    """SQuad-Attention forward with the library's fixed device scratch instead of a workspace (for
+    callers that cannot allocate device memory; calls that overlap on the GPU race on the scratch)."""
+    _check_qkv(q, k, v)
+    prm = _params_for(q, grid, window, order, scale)
+    out = torch.empty_like(q) if out is None else out
+    st = _lib.load().squad_attn_fwd_noalloc(ctypes.byref(prm), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _stream(stream))
+    if st != _lib.SQUAD_OK:
+        raise SquadError(st, "squad_attn_fwd_noalloc")
+    return out
+
+
 def squad_attn_fwd_status(workspace, q, grid, window, order="local_then_global", scale=None, stream=None) -> int:
     """Device status of the last call on `workspace` (synchronises the stream): 0 ok, 4 timeout."""
     prm = _params_for(q, grid, window, order, scale)
