@@ -141,9 +141,10 @@ __device__ __forceinline__ Unit plan_unit(const ShortArgs& a, int U, Cursor& cur
   Unit u;
   int j;
   decode_unit(a, U, u.pass, u.bh, j);
-  const PassGeom& p = a.pass[u.pass].p;
-  const uint32_t sz = a.pass[u.pass].alloc_bytes;
-  u.shared = p.seq_len > 128;
+  const int seq_len = u.pass ? a.pass[1].p.seq_len : a.pass[0].p.seq_len;
+  const int n_seq = u.pass ? a.pass[1].p.n_seq : a.pass[0].p.n_seq;
+  const uint32_t sz = u.pass ? a.pass[1].alloc_bytes : a.pass[0].alloc_bytes;
+  u.shared = seq_len > 128;
   if (u.shared) {
     u.nw = 2;
     u.sigma[0] = u.sigma[1] = j;
@@ -156,12 +157,15 @@ __device__ __forceinline__ Unit plan_unit(const ShortArgs& a, int U, Cursor& cur
   } else {
     u.sigma[0] = 2 * j;
     u.sigma[1] = 2 * j + 1;
-    u.nw = u.sigma[1] < p.n_seq ? 2 : 1;
-    for (int w = 0; w < u.nw; ++w) {
-      cur.take(sz, ring, u.q[w], u.qo[w], u.qvs[w]);
-      cur.take(sz, ring, u.k[w], u.ko[w], u.kvs[w]);
+    u.nw = u.sigma[1] < n_seq ? 2 : 1;
+    cur.take(sz, ring, u.q[0], u.qo[0], u.qvs[0]);
+    cur.take(sz, ring, u.k[0], u.ko[0], u.kvs[0]);
+    if (u.nw == 2) {
+      cur.take(sz, ring, u.q[1], u.qo[1], u.qvs[1]);
+      cur.take(sz, ring, u.k[1], u.ko[1], u.kvs[1]);
     }
-    for (int w = 0; w < u.nw; ++w) cur.take(sz, ring, u.v[w], u.vo[w], u.vvs[w]);
+    cur.take(sz, ring, u.v[0], u.vo[0], u.vvs[0]);
+    if (u.nw == 2) cur.take(sz, ring, u.v[1], u.vo[1], u.vvs[1]);
     if (u.nw == 1) {
       u.sigma[1] = u.sigma[0];
       u.q[1] = u.q[0]; u.qo[1] = u.qo[0]; u.qvs[1] = u.qvs[0];
@@ -170,6 +174,30 @@ __device__ __forceinline__ Unit plan_unit(const ShortArgs& a, int U, Cursor& cur
     }
   }
   return u;
+}
+
+// The fields of one pass, selected with static offsets into the kernel parameters (indexing the
+// parameter array with a run-time pass number would go through local memory).
+struct PassView {
+  const CUtensorMap *q, *k, *v, *o;
+  PassGeom p;
+  int variant;
+  float* lse;
+  uint32_t panel, alloc;
+};
+
+__device__ __forceinline__ PassView view_of(const ShortArgs& a, int pass) {
+  PassView v;
+  if (pass == 0) {
+    v.q = &a.pass[0].tm_q; v.k = &a.pass[0].tm_k; v.v = &a.pass[0].tm_v; v.o = &a.pass[0].tm_o;
+    v.p = a.pass[0].p; v.variant = a.pass[0].variant; v.lse = a.pass[0].lse;
+    v.panel = a.pass[0].panel_bytes; v.alloc = a.pass[0].alloc_bytes;
+  } else {
+    v.q = &a.pass[1].tm_q; v.k = &a.pass[1].tm_k; v.v = &a.pass[1].tm_v; v.o = &a.pass[1].tm_o;
+    v.p = a.pass[1].p; v.variant = a.pass[1].variant; v.lse = a.pass[1].lse;
+    v.panel = a.pass[1].panel_bytes; v.alloc = a.pass[1].alloc_bytes;
+  }
+  return v;
 }
 
 __device__ __forceinline__ int total_units(const ShortArgs& a) {
@@ -264,15 +292,15 @@ __global__ void __launch_bounds__(kThreads, 1) short_kernel(const __grid_constan
         vstart[idx % kND] = vs;
         return true;
       };
-      auto load = [&](const ShortPass& ps, const CUtensorMap* m, int bh, int sigma, uint32_t idx, uint32_t off,
+      auto load = [&](const PassView& ps, const CUtensorMap* m, int bh, int sigma, uint32_t idx, uint32_t off,
                       uint32_t vs) -> bool {
-        if (!make_room(idx, vs, ps.alloc_bytes)) return false;
+        if (!make_room(idx, vs, ps.alloc)) return false;
         uint64_t* fb = &bars->full[idx % kND];
         mbar_arrive_expect_tx(fb, 2u * static_cast<uint32_t>(ps.p.seq_len) * 128u);
         int c[5];
         chunk_coords(g, ps.p, ps.variant, bh, sigma, 0, 0, c);
         tma_load_5d(ring + off, m, fb, c[0], c[1], c[2], c[3], c[4]);
-        tma_load_5d(ring + off + ps.panel_bytes, m, fb, c[0] + 64, c[1], c[2], c[3], c[4]);
+        tma_load_5d(ring + off + ps.panel, m, fb, c[0] + 64, c[1], c[2], c[3], c[4]);
         return true;
       };
       while (ok) {
@@ -285,11 +313,14 @@ __global__ void __launch_bounds__(kThreads, 1) short_kernel(const __grid_constan
         ++qi;
         if (U >= n_total) break;
         const Unit u = plan_unit(a, U, cur, RB);
-        const ShortPass& ps = a.pass[u.pass];
+        const PassView ps = view_of(a, u.pass);
         const int nsrc = u.shared ? 1 : u.nw;
-        for (int w = 0; w < nsrc && ok; ++w) {
-          ok = load(ps, &ps.tm_q, u.bh, u.sigma[w], u.q[w], u.qo[w], u.qvs[w]);
-          if (ok) ok = load(ps, &ps.tm_k, u.bh, u.sigma[w], u.k[w], u.ko[w], u.kvs[w]);
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+          if (w < nsrc && ok) {
+            ok = load(ps, ps.q, u.bh, u.sigma[w], u.q[w], u.qo[w], u.qvs[w]);
+            if (ok) ok = load(ps, ps.k, u.bh, u.sigma[w], u.k[w], u.ko[w], u.kvs[w]);
+          }
         }
         if (ok && u.pass == 1) {
           // values = the first pass's output for this head: wait until all of it is in memory
@@ -308,7 +339,9 @@ __global__ void __launch_bounds__(kThreads, 1) short_kernel(const __grid_constan
           }
           fence_proxy_async_global();   // the TMA loads below must observe those stores
         }
-        for (int w = 0; w < nsrc && ok; ++w) ok = load(ps, &ps.tm_v, u.bh, u.sigma[w], u.v[w], u.vo[w], u.vvs[w]);
+#pragma unroll
+        for (int w = 0; w < 2; ++w)
+          if (w < nsrc && ok) ok = load(ps, ps.v, u.bh, u.sigma[w], u.v[w], u.vo[w], u.vvs[w]);
       }
       if (!ok) {   // make sure the other warps see the end of the work
         for (int i = 0; i < kQ; ++i) {
@@ -333,11 +366,13 @@ __global__ void __launch_bounds__(kThreads, 1) short_kernel(const __grid_constan
       bool ok = true;
       while (ok && next_unit(qi, U, true)) {
         const Unit u = plan_unit(a, U, cur, RB);
-        const ShortPass& ps = a.pass[u.pass];
-        const int N = round16(ps.p.seq_len);
+        const uint32_t panel = u.pass ? a.pass[1].panel_bytes : a.pass[0].panel_bytes;
+        const int N = round16(u.pass ? a.pass[1].p.seq_len : a.pass[0].p.seq_len);
         const uint32_t o_off = N > 128 ? static_cast<uint32_t>(N / 2) : 128u;
         const uint32_t idesc_s = idesc_bf16(128, N, false);
-        for (int w = 0; w < u.nw && ok; ++w) {
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+          if (w >= u.nw || !ok) break;
           if (w == 0 || !u.shared) {
             ok = mbar_wait(&bars->full[u.q[w] % kND], (u.q[w] / kND) & 1, ctl);
             if (ok) ok = mbar_wait(&bars->full[u.k[w] % kND], (u.k[w] / kND) & 1, ctl);
@@ -349,7 +384,7 @@ __global__ void __launch_bounds__(kThreads, 1) short_kernel(const __grid_constan
           const uint32_t qa = smem_u32(ring + u.qo[w]) + (u.shared ? static_cast<uint32_t>(w) * 16384u : 0u);
           const uint32_t ka = smem_u32(ring + u.ko[w]);
           for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t off = (kk >> 2) * ps.panel_bytes + (kk & 3) * 32;
+            const uint32_t off = (kk >> 2) * panel + (kk & 3) * 32;
             umma_bf16_ss(tmem + 256 * w, sw128_desc(qa + off, 16, 1024), sw128_desc(ka + off, 16, 1024), idesc_s,
                          kk > 0);
           }
@@ -359,7 +394,9 @@ __global__ void __launch_bounds__(kThreads, 1) short_kernel(const __grid_constan
             umma_commit(&bars->empty[u.k[w] % kND]);
           }
         }
-        for (int w = 0; w < u.nw && ok; ++w) {
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+          if (w >= u.nw || !ok) break;
           ok = mbar_wait(&bars->p_full[w], p_cnt[w] & 1, ctl);
           ++p_cnt[w];
           if (ok && (w == 0 || !u.shared)) ok = mbar_wait(&bars->full[u.v[w] % kND], (u.v[w] / kND) & 1, ctl);
@@ -368,16 +405,19 @@ __global__ void __launch_bounds__(kThreads, 1) short_kernel(const __grid_constan
           const uint32_t va = smem_u32(ring + u.vo[w]);
           for (int kk = 0; kk < N / 16; ++kk)
             umma_bf16_ts(tmem + 256 * w + o_off, tmem + 256 * w + kk * 8,
-                         sw128_desc(va + kk * 2048, ps.panel_bytes, 1024), idesc_pv, kk > 0);
+                         sw128_desc(va + kk * 2048, panel, 1024), idesc_pv, kk > 0);
           if (!u.shared) umma_commit(&bars->o_full[w]);
         }
         if (ok && u.shared) {   // both tiles read the one V allocation: neither overwrites it before both PVs
           umma_commit(&bars->o_full[0]);
           umma_commit(&bars->o_full[1]);
         }
-        for (int w = 0; w < u.nw; ++w) {
-          ++wu[w];
-          prev_ooff[w] = o_off;
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+          if (w < u.nw) {
+            ++wu[w];
+            prev_ooff[w] = o_off;
+          }
         }
       }
       umma_commit(&bars->drain);
@@ -392,23 +432,31 @@ __global__ void __launch_bounds__(kThreads, 1) short_kernel(const __grid_constan
       bool ok = true;
       while (ok && next_unit(qi, U, true)) {
         const Unit u = plan_unit(a, U, cur, RB);
-        const ShortPass& ps = a.pass[u.pass];
+        const PassView ps = view_of(a, u.pass);
         const int nseq = u.shared ? 1 : u.nw;
-        for (int w = 0; w < u.nw && ok; ++w) {
-          ok = mbar_wait(&bars->staged[w], st_cnt[w] & 1, ctl);
-          ++st_cnt[w];
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+          if (w < u.nw && ok) {
+            ok = mbar_wait(&bars->staged[w], st_cnt[w] & 1, ctl);
+            ++st_cnt[w];
+          }
         }
         if (!ok) break;
-        for (int w = 0; w < nseq; ++w) {
-          int c[5];
-          chunk_coords(g, ps.p, ps.variant, u.bh, u.sigma[w], 0, 0, c);
-          const uint8_t* src = ring + u.vo[w];
-          tma_store_5d(&ps.tm_o, src, c[0], c[1], c[2], c[3], c[4]);
-          tma_store_5d(&ps.tm_o, src + ps.panel_bytes, c[0] + 64, c[1], c[2], c[3], c[4]);
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+          if (w < nseq) {
+            int c[5];
+            chunk_coords(g, ps.p, ps.variant, u.bh, u.sigma[w], 0, 0, c);
+            const uint8_t* src = ring + u.vo[w];
+            tma_store_5d(ps.o, src, c[0], c[1], c[2], c[3], c[4]);
+            tma_store_5d(ps.o, src + ps.panel, c[0] + 64, c[1], c[2], c[3], c[4]);
+          }
         }
         bulk_commit_group();
         bulk_wait_read_all();   // the V allocations may be refilled once their stores have read them
-        for (int w = 0; w < nseq; ++w) mbar_arrive(&bars->empty[u.v[w] % kND]);
+#pragma unroll
+        for (int w = 0; w < 2; ++w)
+          if (w < nseq) mbar_arrive(&bars->empty[u.v[w] % kND]);
         if (a.n_passes == 2 && u.pass == 0) {
           // publish this head's progress once the output is in global memory
           bulk_wait_all();
@@ -436,14 +484,15 @@ __global__ void __launch_bounds__(kThreads, 1) short_kernel(const __grid_constan
       if (!more) break;
       const Unit u = plan_unit(a, U, cur, RB);
       if (wg >= u.nw) continue;
-      const ShortPass& ps = a.pass[u.pass];
-      const PassGeom& p = ps.p;
-      const int s_len = p.seq_len;
+      const int s_len = u.pass ? a.pass[1].p.seq_len : a.pass[0].p.seq_len;
+      const uint32_t panel = u.pass ? a.pass[1].panel_bytes : a.pass[0].panel_bytes;
       const int N = round16(s_len);
       const uint32_t t_o = t_s + (N > 128 ? static_cast<uint32_t>(N / 2) : 128u);
       const int nchunk = (N + 63) / 64;
       const int row0 = u.shared ? 128 * wg : 0;   // first sequence row of this tile
       const int src = u.shared ? 0 : wg;
+      const uint32_t v_off = src ? u.vo[1] : u.vo[0];
+      const int sigma = src ? u.sigma[1] : u.sigma[0];
       int valid = s_len - row0;
       if (valid > 128) valid = 128;
       const bool active = wq * 32 < valid;        // warps of padding rows only keep the barriers
@@ -504,7 +553,7 @@ __global__ void __launch_bounds__(kThreads, 1) short_kernel(const __grid_constan
       if (!ok) break;
       tc_fence_after();
       const int vrow = row0 + row;   // row within the V allocation's panels
-      const uint32_t row_addr = smem_u32(ring + u.vo[src]) + static_cast<uint32_t>(vrow) * 128u;
+      const uint32_t row_addr = smem_u32(ring + v_off) + static_cast<uint32_t>(vrow) * 128u;
       const bool store_row = row < valid;
       const float inv_l = active ? 1.f / l : 0.f;
 #pragma unroll
@@ -520,16 +569,18 @@ __global__ void __launch_bounds__(kThreads, 1) short_kernel(const __grid_constan
         if (store_row) {
 #pragma unroll
           for (int c = 0; c < 8; ++c)
-            st_shared_v4(row_addr + h * ps.panel_bytes + ((c ^ (vrow & 7)) << 4),
+            st_shared_v4(row_addr + h * panel + ((c ^ (vrow & 7)) << 4),
                          pack_bf16x2(__uint_as_float(o[c * 8 + 0]) * inv_l, __uint_as_float(o[c * 8 + 1]) * inv_l),
                          pack_bf16x2(__uint_as_float(o[c * 8 + 2]) * inv_l, __uint_as_float(o[c * 8 + 3]) * inv_l),
                          pack_bf16x2(__uint_as_float(o[c * 8 + 4]) * inv_l, __uint_as_float(o[c * 8 + 5]) * inv_l),
                          pack_bf16x2(__uint_as_float(o[c * 8 + 6]) * inv_l, __uint_as_float(o[c * 8 + 7]) * inv_l));
         }
       }
-      if (ps.lse != nullptr && store_row) {
-        const int tok = token_of(g, p, u.sigma[src], 0, vrow);
-        if (tok >= 0) ps.lse[static_cast<size_t>(u.bh) * g.n + tok] = (m + __log2f(l)) * 0.69314718055994531f;
+      float* lse = u.pass ? a.pass[1].lse : a.pass[0].lse;
+      if (lse != nullptr && store_row) {
+        const PassGeom pg = u.pass ? a.pass[1].p : a.pass[0].p;
+        const int tok = token_of(g, pg, sigma, 0, vrow);
+        if (tok >= 0) lse[static_cast<size_t>(u.bh) * g.n + tok] = (m + __log2f(l)) * 0.69314718055994531f;
       }
       fence_proxy_async_smem();   // staging writes -> visible to the TMA store (async proxy)
       __syncwarp();
