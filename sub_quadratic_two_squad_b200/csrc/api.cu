@@ -25,9 +25,8 @@ constexpr int kAbiVersion = 1;
 // 1-3 work counters of the persistent kernels, then one counter per (b, head) for the fused passes.
 constexpr size_t kCtrlFixedWords = 4;
 // Run both passes of a short-sequence problem in one persistent launch (second pass trailing the first
-// by two heads, reading it from L2). Off until that schedule beats two back-to-back launches: its ring
-// cannot yet hold a unit's boxes while the next unit's load, so consecutive units barely overlap.
-constexpr bool kFusePasses = false;
+// by two heads, reading it from L2); otherwise one launch per pass.
+constexpr bool kFusePasses = true;
 constexpr unsigned long long kWaitTimeoutNs = 1000000000ull;   // 1 s per device-side wait
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
