@@ -26,6 +26,36 @@ WORKLOAD_NAME = ("Wan-2.2-5B-shaped SQuad attention block: B=1 h=24 d=128, grid 
 METRIC = "SQuad-attn fwd ms/block & TFLOP/s at n=18480,h=24,d=128 bf16; % of roofline"
 PAGES_MS = 4.27   # pages' SQuad attention latency per block for this workload (1x H100, bf16): context
 
+# DRAM traffic of one launch of the forward kernel from the ncu capture summarised in
+# profiles/short_kernel_wan22_5b_fwd.md (dram__bytes_read.sum + dram__bytes_write.sum), valid only for
+# the kernel source it was measured on (sha1 prefix below); otherwise reported as null.
+PROFILED_TRAFFIC_BYTES = (442.92224 + 194.259456) * 1e6
+PROFILED_KERNEL_SHA1 = "02bb1d3717706da7"
+PROFILED_KERNEL_SRC = os.path.join(ROOT, "sub_quadratic_two_squad_b200", "csrc", "attn_short.cu")
+
+
+def profiled_traffic():
+    import hashlib
+
+    try:
+        with open(PROFILED_KERNEL_SRC, "rb") as f:
+            sha = hashlib.sha1(f.read()).hexdigest()
+    except OSError:
+        return None
+    return PROFILED_TRAFFIC_BYTES if sha.startswith(PROFILED_KERNEL_SHA1) else None
+
+
+def max_over_ranks(value, world, device=None):
+    """Largest `value` over all ranks (device-side timing is reported as the slowest rank)."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
 
 def peaks():
     try:
@@ -217,12 +247,8 @@ def run_ours(args, rank, world, local_rank):
             ev[i][1].record(stream)
         t_end.record(stream)
         torch.cuda.synchronize()
-    total_ms = t_start.elapsed_time(t_end)
+    total_ms = max_over_ranks(t_start.elapsed_time(t_end), world, dev)
     per_launch_ms = [a.elapsed_time(b) for a, b in ev]
-    ms = torch.tensor([total_ms], device=dev)
-    if world > 1:
-        dist.all_reduce(ms, op=dist.ReduceOp.MAX)
-    total_ms = float(ms.item())
     ms_per_step = total_ms / args.steps
     status_ok = all(squad_attn_fwd_status(s[4], s[0], w["grid"], w["window"], w["order"]) == 0 for s in sets)
 
@@ -240,11 +266,7 @@ def run_ours(args, rank, world, local_rank):
         runner(hq, hk, hv, ho)
     b.record(runner.stream)
     torch.cuda.synchronize()
-    e2e_ms = a.elapsed_time(b) / e2e_steps
-    e2 = torch.tensor([e2e_ms], device=dev)
-    if world > 1:
-        dist.all_reduce(e2, op=dist.ReduceOp.MAX)
-    e2e_ms = float(e2.item())
+    e2e_ms = max_over_ranks(a.elapsed_time(b) / e2e_steps, world, dev)
 
     # Full attention at the same n, beside SQuad (a few calls: ~4.2 TFLOP each).
     q, k, v, o, _ = sets[0]
@@ -259,6 +281,22 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     full_ms = fa.elapsed_time(fb) / reps
     n_full = 4.0 * w["B"] * w["h"] * w["d"] * n * n
+
+    # Backward at the same shape, beside the forward (a few calls).
+    from sub_quadratic_two_squad_b200 import squad_attn_bwd
+
+    q, k, v, o, ws = sets[0]
+    dout = torch.from_numpy(make_inputs(w["B"], w["h"], n, w["d"], dtype="bf16", with_dout=True)["do"]).to(dev, torch.bfloat16)
+    squad_attn_fwd(q, k, v, w["grid"], w["window"], w["order"], out=o, workspace=ws)
+    grads = squad_attn_bwd(q, k, v, o, dout, ws, w["grid"], w["window"], w["order"])
+    torch.cuda.synchronize()
+    ba, bb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ba.record(stream)
+    for _ in range(3):
+        squad_attn_bwd(q, k, v, o, dout, ws, w["grid"], w["window"], w["order"], dq=grads[0], dk=grads[1], dv=grads[2])
+    bb.record(stream)
+    torch.cuda.synchronize()
+    bwd_ms = ba.elapsed_time(bb) / 3
 
     if rank != 0:
         return
@@ -284,18 +322,19 @@ def run_ours(args, rank, world, local_rank):
                    "head_dim": w["d"], "window": "21x2x4", "parallelism": f"replicas x{world}" if world > 1 else "1 gpu",
                    "l2": f"{n_sets} rotating buffer sets of ~570 MB each (> 126 MB L2); no reuse between steps"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                     "traffic": None, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)",
-                     "kernel": "squad_attn_fwd step (tc_pass_kernel local + global)",
+                     "traffic": profiled_traffic(), "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)",
+                     "kernel": "short_kernel (both passes in one launch) + control-block memset",
                      "alg_bytes_per_launch": alg_bytes(), "mean_launch_ms": mean_launch,
                      "tensor_frac": f / (mean_launch * 1e-3) / 1e12 / tf_peak},
         "e2e": {"value": world * f / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": runner.h2d_bytes(), "d2h_bytes_per_step": runner.d2h_bytes(),
                 "steps": e2e_steps, "api": "sub_quadratic_two_squad_b200.HostRunner (pinned host buffers)"},
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": args.steps,
         "clocks": clk.summary(),
         "device_status_ok": status_ok,
         "full_attn": {"ms_per_block": full_ms, "tflops": n_full / (full_ms * 1e-3) / 1e12,
                       "flop_ratio": n_full / f, "latency_ratio": full_ms / ms_per_step},
+        "backward": {"ms_per_block": bwd_ms, "kernels": "CUDA-core row/column kernels, 2 per pass"},
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
