@@ -12,6 +12,7 @@
 
 #include "squad_attn.h"
 #include "geometry.cuh"
+#include "bwd_pass.h"
 #include "short_pass.h"
 #include "simt_pass.h"
 #include "tc_pass.h"
@@ -387,6 +388,49 @@ squad_status_t squad_attn_bwd(const squad_params_t* p, const void* q, const void
   if (cudaMemsetAsync(bw.status, 0, ctrl_bytes(g), stream) != cudaSuccess) return SQUAD_ERR_CUDA;
   const int first = p->order == SQUAD_LOCAL_THEN_GLOBAL ? kLocal : kGlobal;
   const int second = p->order == SQUAD_LOCAL_THEN_GLOBAL ? kGlobal : kLocal;
+
+  if (bf16) {
+    // Tensor-core kernels when every sequence of both passes fits one CTA: pass 2 first (values O1,
+    // upstream dout; gives the dQ, dK shares and dO1 in bf16), then pass 1 (values v, upstream dO1;
+    // completes dQ, dK and gives dV).
+    BwdTcArgs b2, b1;
+    std::memset(&b2, 0, sizeof(b2));
+    b2.g = g;
+    b2.p = make_geom(g, second, 256);
+    b1 = b2;
+    b1.p = make_geom(g, first, 256);
+    if (short_eligible(p, g, b2.p) && short_eligible(p, g, b1.p) && bwd_tc_plan(b2) && bwd_tc_plan(b1)) {
+      __nv_bfloat16* do1 = reinterpret_cast<__nv_bfloat16*>(bw.do1);
+      b2.variant = second == kGlobal ? kSlotBoxVariant : 0;
+      b1.variant = first == kGlobal ? kSlotBoxVariant : 0;
+      if (!encode_pass_map(&b2.tm_q, q, g, b2.p, b2.variant) || !encode_pass_map(&b2.tm_k, k, g, b2.p, b2.variant) ||
+          !encode_pass_map(&b2.tm_v, fw.o1, g, b2.p, b2.variant) ||
+          !encode_pass_map(&b2.tm_do, dout, g, b2.p, b2.variant) ||
+          !encode_pass_map(&b1.tm_q, q, g, b1.p, b1.variant) || !encode_pass_map(&b1.tm_k, k, g, b1.p, b1.variant) ||
+          !encode_pass_map(&b1.tm_v, v, g, b1.p, b1.variant) || !encode_pass_map(&b1.tm_do, do1, g, b1.p, b1.variant))
+        return SQUAD_ERR_CUDA;
+      for (BwdTcArgs* b : {&b2, &b1}) {
+        b->drow = bw.drow;
+        b->dq_acc = bw.dq_acc;
+        b->dk_acc = bw.dk_acc;
+        b->scale = scale;
+        b->scale_log2 = scale * 1.4426950408889634f;
+        b->status = bw.status;
+        b->timeout_ns = kWaitTimeoutNs;
+      }
+      b2.lse = fw.lse2;
+      b2.dv_out = do1;
+      b2.final_out = 0;
+      b1.lse = fw.lse1;
+      b1.dq_out = static_cast<__nv_bfloat16*>(dq);
+      b1.dk_out = static_cast<__nv_bfloat16*>(dk);
+      b1.dv_out = static_cast<__nv_bfloat16*>(dv);
+      b1.final_out = 1;
+      if (launch_bwd_tc(b2, stream) != cudaSuccess) return SQUAD_ERR_CUDA;
+      if (launch_bwd_tc(b1, stream) != cudaSuccess) return SQUAD_ERR_CUDA;
+      return SQUAD_OK;
+    }
+  }
 
   // Pass 2 backward: values = O1 (pass-1 output), upstream = dout. Gives dQ, dK shares and dO1.
   SimtBwdArgs a{};

@@ -1,0 +1,38 @@
+// Arguments and launchers of the tensor-core backward kernels (bwd_tc.cu): one SQuad pass's gradients
+// over sequences of at most 256 tokens, each sequence loaded whole (Q, K, V, dO) as TMA boxes.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "geometry.cuh"
+
+namespace squad {
+
+struct BwdTcArgs {
+  CUtensorMap tm_q, tm_k, tm_v, tm_do;   // bf16 maps whose box is one whole sequence (SWIZZLE_128B)
+  Grid g;
+  PassGeom p;                 // one chunk per sequence (make_geom(..., 256))
+  int variant;                // slot-box encoding (GLOBAL pass)
+  const float* lse;           // [B, h, n] natural-log LSE of this pass's forward
+  float* drow;                // [B, h, n] D_i = sum_j P_ij dP_ij: written by the row kernel, read by the column kernel
+  float* dq_acc;              // [B, h, n, d] fp32 share of dQ (written, or read and completed when final)
+  float* dk_acc;              // [B, h, n, d] fp32 share of dK (likewise)
+  __nv_bfloat16* dq_out;      // final dQ (final_out only)
+  __nv_bfloat16* dk_out;      // final dK (final_out only)
+  __nv_bfloat16* dv_out;      // gradient of this pass's values
+  float scale, scale_log2;
+  int final_out;              // add the other pass's share and write dq_out / dk_out
+  uint32_t panel_bytes;       // rows (rounded to 8) x 128 bytes
+  uint32_t guard_bytes, smem_bytes;
+  uint32_t* status;           // device status word (0 = ok, 4 = a wait timed out)
+  unsigned long long timeout_ns;
+};
+
+// Fills the shared-memory plan of `a` (p and g set); false if the sequences do not fit.
+bool bwd_tc_plan(BwdTcArgs& a);
+// Row kernel (dQ, D) then column kernel (dK, dV) of one pass.
+cudaError_t launch_bwd_tc(const BwdTcArgs& a, cudaStream_t stream);
+
+}  // namespace squad
