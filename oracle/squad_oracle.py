@@ -153,6 +153,11 @@ def _f64(x):
 
 LOCAL_THEN_GLOBAL = "local_then_global"
 GLOBAL_THEN_LOCAL = "global_then_local"
+# Single-pass variants: each pass alone, as the paper ablates them (SQuad paper §4.4, "The need for and
+# the order of the two passes").
+LOCAL_ONLY = "local_only"
+GLOBAL_ONLY = "global_only"
+SINGLE_PASS = (LOCAL_ONLY, GLOBAL_ONLY)
 
 
 def squad_attn_fwd(Q, K, V, grid, window, order=LOCAL_THEN_GLOBAL, scale=None, return_aux=False):
@@ -162,6 +167,9 @@ def squad_attn_fwd(Q, K, V, grid, window, order=LOCAL_THEN_GLOBAL, scale=None, r
     With return_aux, also returns dict(o1=..., lse1=..., lse2=...) (pass-1 output and both passes'
     log-sum-exp).
     """
+    if order in SINGLE_PASS:
+        o, lse = (local_pass if order == LOCAL_ONLY else global_pass)(Q, K, V, grid, window, scale)
+        return (o, dict(lse1=lse)) if return_aux else o
     if order not in (LOCAL_THEN_GLOBAL, GLOBAL_THEN_LOCAL):
         raise ValueError(order)
     first, second = (local_pass, global_pass) if order == LOCAL_THEN_GLOBAL else (global_pass, local_pass)
@@ -183,6 +191,17 @@ def squad_attn_bwd(Q, K, V, dO, grid, window, order=LOCAL_THEN_GLOBAL, scale=Non
     sc = _scale(Q.shape[-1], scale)
     table = window_partition(*grid, *window)
     local_groups, global_groups = table, np.ascontiguousarray(table.T)
+    if order in SINGLE_PASS:
+        # one softmax attention per sequence of the pass
+        g = local_groups if order == LOCAL_ONLY else global_groups
+        dQ, dK, dV = np.empty_like(Q), np.empty_like(K), np.empty_like(V)
+        for b in range(Q.shape[0]):
+            for hh in range(Q.shape[1]):
+                dq, dk, dv = softmax_attention_bwd(Q[b, hh][g], K[b, hh][g], V[b, hh][g], dO[b, hh][g], sc)
+                dQ[b, hh][g], dK[b, hh][g], dV[b, hh][g] = dq, dk, dv
+        return dQ, dK, dV
+    if order not in (LOCAL_THEN_GLOBAL, GLOBAL_THEN_LOCAL):
+        raise ValueError(order)
     g1, g2 = (local_groups, global_groups) if order == LOCAL_THEN_GLOBAL else (global_groups, local_groups)
     o1, _ = _pass(Q, K, V, g1, sc)
 

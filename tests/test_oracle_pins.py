@@ -291,3 +291,47 @@ def test_flops_equal_the_oracles_gemm_shapes(grid, window):
     counted = 2 * (n_seq_l * 2 * s_l * s_l * d + n_seq_g * 2 * s_g * s_g * d)
     n = int(np.prod(grid))
     assert counted == pytest.approx(orc.squad_flops(1, 1, d, n, s_l), rel=1e-12)
+
+
+# ------------------------------------------------------------------------------------------------
+# single-pass variants (each pass alone, as the paper ablates them)
+# ------------------------------------------------------------------------------------------------
+
+def _masked_attention_torch(q, k, v, mask, scale):
+    """Dense attention restricted by a boolean mask, torch float64 autograd-ready (library routine)."""
+    return torch.nn.functional.scaled_dot_product_attention(q, k, v, attn_mask=torch.from_numpy(mask), scale=scale)
+
+
+@pytest.mark.parametrize("order", [orc.LOCAL_ONLY, orc.GLOBAL_ONLY])
+@pytest.mark.parametrize("grid,window", [((3, 4, 6), (3, 2, 3)), ((2, 6, 4), (2, 3, 1))])
+def test_single_pass_forward_and_backward_are_masked_attention(order, grid, window):
+    """local_only = attention restricted to the same window; global_only = restricted to the same slot.
+    Forward against torch SDPA with that mask, backward against torch autograd of it (float64)."""
+    T, H, W = grid
+    n, d = T * H * W, 5
+    same_window, same_slot = _masks(T, H, W, window[1], window[2])
+    mask = same_window if order == orc.LOCAL_ONLY else same_slot
+    q, k, v, do = (_rand((1, 2, n, d), s) for s in (11, 12, 13, 14))
+    sc = 0.7
+    o = orc.squad_attn_fwd(q, k, v, grid, window, order, scale=sc)
+    tq, tk, tv = (torch.from_numpy(x).requires_grad_(True) for x in (q, k, v))
+    to = _masked_attention_torch(tq, tk, tv, mask, sc)
+    np.testing.assert_allclose(o, to.detach().numpy(), rtol=1e-12, atol=1e-12)
+    to.backward(torch.from_numpy(do))
+    dq, dk, dv = orc.squad_attn_bwd(q, k, v, do, grid, window, order, scale=sc)
+    for got, ref in ((dq, tq.grad), (dk, tk.grad), (dv, tv.grad)):
+        np.testing.assert_allclose(got, ref.numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_single_passes_compose_to_squad():
+    """Chaining the two single-pass variants (the second taking the first's output as values) is the
+    two-pass method, in either order."""
+    grid, window = (3, 4, 6), (3, 2, 3)
+    n = 72
+    q, k, v = (_rand((1, 1, n, 4), s) for s in (21, 22, 23))
+    o_l = orc.squad_attn_fwd(q, k, v, grid, window, orc.LOCAL_ONLY)
+    np.testing.assert_allclose(orc.squad_attn_fwd(q, k, o_l, grid, window, orc.GLOBAL_ONLY),
+                               orc.squad_attn_fwd(q, k, v, grid, window, orc.LOCAL_THEN_GLOBAL), rtol=1e-12, atol=1e-13)
+    o_g = orc.squad_attn_fwd(q, k, v, grid, window, orc.GLOBAL_ONLY)
+    np.testing.assert_allclose(orc.squad_attn_fwd(q, k, o_g, grid, window, orc.LOCAL_ONLY),
+                               orc.squad_attn_fwd(q, k, v, grid, window, orc.GLOBAL_THEN_LOCAL), rtol=1e-12, atol=1e-13)
