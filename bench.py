@@ -299,6 +299,23 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     bwd_ms = ba.elapsed_time(bb) / bwd_reps
 
+    # Single-pass variants (one pass alone) at the same shape, rotating the same buffer sets.
+    single = {}
+    for order in ("local_only", "global_only"):
+        q, k, v, o, ws = sets[0]
+        squad_attn_fwd(q, k, v, w["grid"], w["window"], order, out=o, workspace=ws)
+        torch.cuda.synchronize()
+        sa, sb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 30
+        sa.record(stream)
+        for i in range(reps):
+            q, k, v, o, ws = sets[i % len(sets)]
+            squad_attn_fwd(q, k, v, w["grid"], w["window"], order, out=o, workspace=ws)
+        sb.record(stream)
+        torch.cuda.synchronize()
+        ms = sa.elapsed_time(sb) / reps
+        single[order] = {"ms_per_block": ms, "hbm_frac": alg_bytes() / (ms * 1e-3) / 1e9 / peaks()[0]}
+
     if rank != 0:
         return
     hbm, tf_peak, peak_kind = peaks()
@@ -335,6 +352,7 @@ def run_ours(args, rank, world, local_rank):
         "device_status_ok": status_ok,
         "full_attn": {"ms_per_block": full_ms, "tflops": n_full / (full_ms * 1e-3) / 1e12,
                       "flop_ratio": n_full / f, "latency_ratio": full_ms / ms_per_step},
+        "single_pass": single,
         "backward": {"ms_per_block": bwd_ms,
                      "tflops_algorithmic": 2.0 * f / (bwd_ms * 1e-3) / 1e12,
                      "flops_note": "algorithmic = 2x forward (dQ, dK, dV, dP products); the kernels execute 3.5x "

@@ -64,8 +64,15 @@ typedef enum {
 typedef enum { SQUAD_BF16 = 0, SQUAD_FP32 = 1 } squad_dtype_t;
 
 /* Pass order. LOCAL_THEN_GLOBAL is the paper's chosen order; GLOBAL_THEN_LOCAL the ablated reverse
- * (paper §4.4 "The need for and the order of the two passes"; appendix "On the ordering"). */
-typedef enum { SQUAD_LOCAL_THEN_GLOBAL = 0, SQUAD_GLOBAL_THEN_LOCAL = 1 } squad_order_t;
+ * (paper §4.4 "The need for and the order of the two passes"; appendix "On the ordering").
+ * LOCAL_ONLY and GLOBAL_ONLY run one pass alone (o = pass(q, k, v)), the single-pass variants the
+ * same section ablates; chaining them reproduces either two-pass order. */
+typedef enum {
+  SQUAD_LOCAL_THEN_GLOBAL = 0,
+  SQUAD_GLOBAL_THEN_LOCAL = 1,
+  SQUAD_LOCAL_ONLY = 2,
+  SQUAD_GLOBAL_ONLY = 3
+} squad_order_t;
 
 typedef struct {
   int B, h, d;      /* batch, heads, head dim (d in {64, 128}; bf16 tensor-core path: d == 128)  */
@@ -82,7 +89,8 @@ typedef struct {
  * invalid parameters. */
 SQUAD_API size_t squad_attn_fwd_workspace_bytes(const squad_params_t* p);
 
-/* SQuad-Attention forward: o = pass2(q, k, pass1(q, k, v)) with the passes in `order`.
+/* SQuad-Attention forward: o = pass2(q, k, pass1(q, k, v)) with the passes in `order` (or one pass,
+ * o = pass(q, k, v), for the single-pass orders).
  * q, k, v: inputs [B,h,n,d]; o: output [B,h,n,d]; workspace: >= squad_attn_fwd_workspace_bytes. */
 SQUAD_API squad_status_t squad_attn_fwd(const squad_params_t* p, const void* q, const void* k, const void* v,
                               void* o, void* workspace, squad_stream_t stream);

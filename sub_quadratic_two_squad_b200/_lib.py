@@ -9,7 +9,7 @@ LIB_PATH = os.path.join(PKG_DIR, "libsquad_attn.so")
 
 SQUAD_OK, SQUAD_ERR_INVALID_ARG, SQUAD_ERR_UNSUPPORTED, SQUAD_ERR_CUDA, SQUAD_ERR_TIMEOUT = range(5)
 SQUAD_BF16, SQUAD_FP32 = 0, 1
-SQUAD_LOCAL_THEN_GLOBAL, SQUAD_GLOBAL_THEN_LOCAL = 0, 1
+SQUAD_LOCAL_THEN_GLOBAL, SQUAD_GLOBAL_THEN_LOCAL, SQUAD_LOCAL_ONLY, SQUAD_GLOBAL_ONLY = 0, 1, 2, 3
 SQUAD_NOALLOC_MAX_WORKSPACE_BYTES = 128 * 1024 * 1024
 
 # Every symbol include/squad_attn.h declares, with (restype, argtypes).

@@ -12,7 +12,8 @@ import torch
 
 from . import _lib
 
-ORDERS = {"local_then_global": _lib.SQUAD_LOCAL_THEN_GLOBAL, "global_then_local": _lib.SQUAD_GLOBAL_THEN_LOCAL}
+ORDERS = {"local_then_global": _lib.SQUAD_LOCAL_THEN_GLOBAL, "global_then_local": _lib.SQUAD_GLOBAL_THEN_LOCAL,
+          "local_only": _lib.SQUAD_LOCAL_ONLY, "global_only": _lib.SQUAD_GLOBAL_ONLY}
 _DTYPES = {torch.bfloat16: _lib.SQUAD_BF16, torch.float32: _lib.SQUAD_FP32}
 
 
@@ -135,8 +136,8 @@ def full_attn_fwd(q, k, v, grid=None, scale=None, out=None, lse=None, stream=Non
     return out
 
 
-def squad_attn_flops(B, h, d, grid, window) -> float:
-    return float(_lib.load().squad_attn_flops(ctypes.byref(make_params(B, h, d, grid, window))))
+def squad_attn_flops(B, h, d, grid, window, order="local_then_global") -> float:
+    return float(_lib.load().squad_attn_flops(ctypes.byref(make_params(B, h, d, grid, window, order))))
 
 
 def full_attn_flops(B, h, d, grid) -> float:

@@ -56,7 +56,7 @@ squad_status_t validate(const squad_params_t* p, bool windowed, Grid* g, float* 
   gg.W = p->W;
   gg.n = static_cast<int>(n);
   if (windowed) {
-    if (p->order != SQUAD_LOCAL_THEN_GLOBAL && p->order != SQUAD_GLOBAL_THEN_LOCAL) return SQUAD_ERR_INVALID_ARG;
+    if (p->order < SQUAD_LOCAL_THEN_GLOBAL || p->order > SQUAD_GLOBAL_ONLY) return SQUAD_ERR_INVALID_ARG;
     if (p->tw < 1 || p->hw < 1 || p->ww < 1) return SQUAD_ERR_INVALID_ARG;
     if (p->tw > p->T || p->hw > p->H || p->ww > p->W) return SQUAD_ERR_INVALID_ARG;
     // The window spans the full temporal extent and tiles space exactly; other windows (tw < T,
@@ -297,7 +297,9 @@ double squad_attn_flops(const squad_params_t* p) {
   if (validate(p, true, &g, &sc) != SQUAD_OK) return 0.0;
   const double w = static_cast<double>(p->tw) * p->hw * p->ww;
   const double n = g.n;
-  return 4.0 * p->B * p->h * p->d * (n * w + n * n / w);
+  const double local = n * w, global = n * n / w;   // per (b, head, d): n rows x sequence length
+  const double terms = p->order == SQUAD_LOCAL_ONLY ? local : p->order == SQUAD_GLOBAL_ONLY ? global : local + global;
+  return 4.0 * p->B * p->h * p->d * terms;
 }
 
 double full_attn_flops(const squad_params_t* p) {
@@ -335,9 +337,14 @@ squad_status_t squad_attn_fwd(const squad_params_t* p, const void* q, const void
   FwdWorkspace ws = carve_fwd(workspace, g, eb);
   if (cudaMemsetAsync(ws.status, 0, ctrl_bytes(g), stream) != cudaSuccess) return SQUAD_ERR_CUDA;
   const bool bf16 = p->dtype == SQUAD_BF16;
+  uint32_t* ctrl = ws.status;
+  if (p->order == SQUAD_LOCAL_ONLY || p->order == SQUAD_GLOBAL_ONLY) {
+    // one pass straight into o; its LSE goes where the first pass's would (the backward reads it there)
+    const int kind = p->order == SQUAD_LOCAL_ONLY ? kLocal : kGlobal;
+    return run_pass(p, g, kind, scale, q, k, v, bf16, o, ws.lse1, ctrl, ctrl + 2, stream);
+  }
   const int first = p->order == SQUAD_LOCAL_THEN_GLOBAL ? kLocal : kGlobal;
   const int second = p->order == SQUAD_LOCAL_THEN_GLOBAL ? kGlobal : kLocal;
-  uint32_t* ctrl = ws.status;
   if (kFusePasses && short_eligible(p, g, make_geom(g, first, 256)) && short_eligible(p, g, make_geom(g, second, 256))) {
     // Both passes in one persistent launch; the second pass reads each head's first-pass output
     // (its values) once all of that head's first-pass units are stored.
@@ -386,6 +393,59 @@ squad_status_t squad_attn_bwd(const squad_params_t* p, const void* q, const void
   FwdWorkspace fw = carve_fwd(const_cast<void*>(fwd_workspace), g, eb);
   BwdWorkspace bw = carve_bwd(bwd_workspace, g);
   if (cudaMemsetAsync(bw.status, 0, ctrl_bytes(g), stream) != cudaSuccess) return SQUAD_ERR_CUDA;
+  if (p->order == SQUAD_LOCAL_ONLY || p->order == SQUAD_GLOBAL_ONLY) {
+    // One pass: values v, upstream dout, the pass's LSE in the first slot; no share to add.
+    const int kind = p->order == SQUAD_LOCAL_ONLY ? kLocal : kGlobal;
+    if (bf16) {
+      BwdTcArgs b;
+      std::memset(&b, 0, sizeof(b));
+      b.g = g;
+      b.p = make_geom(g, kind, 256);
+      if (short_eligible(p, g, b.p) && bwd_tc_plan(b)) {
+        b.variant = kind == kGlobal ? kSlotBoxVariant : 0;
+        if (!encode_pass_map(&b.tm_q, q, g, b.p, b.variant) || !encode_pass_map(&b.tm_k, k, g, b.p, b.variant) ||
+            !encode_pass_map(&b.tm_v, v, g, b.p, b.variant) || !encode_pass_map(&b.tm_do, dout, g, b.p, b.variant))
+          return SQUAD_ERR_CUDA;
+        b.lse = fw.lse1;
+        b.drow = bw.drow;
+        b.dq_acc = bw.dq_acc;
+        b.dk_acc = bw.dk_acc;
+        b.dq_out = static_cast<__nv_bfloat16*>(dq);
+        b.dk_out = static_cast<__nv_bfloat16*>(dk);
+        b.dv_out = static_cast<__nv_bfloat16*>(dv);
+        b.final_out = 1;
+        b.accumulate = 0;
+        b.scale = scale;
+        b.scale_log2 = scale * 1.4426950408889634f;
+        b.status = bw.status;
+        b.timeout_ns = kWaitTimeoutNs;
+        return launch_bwd_tc(b, stream) == cudaSuccess ? SQUAD_OK : SQUAD_ERR_CUDA;
+      }
+    }
+    SimtBwdArgs a{};
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.dout = dout;
+    a.lse = fw.lse1;
+    a.Drow = bw.drow;
+    a.dq_acc = bw.dq_acc;
+    a.dk_acc = bw.dk_acc;
+    a.dq_out = dq;
+    a.dk_out = dk;
+    a.dv_out = dv;
+    a.g = g;
+    a.p = make_geom(g, kind);
+    a.scale = scale;
+    a.in_bf16 = bf16;
+    a.v_bf16 = bf16;
+    a.dout_bf16 = bf16;
+    a.grad_bf16 = bf16;
+    a.dv_bf16 = bf16;
+    a.accumulate = 0;
+    a.final_out = 1;
+    return launch_simt_bwd(a, stream) == cudaSuccess ? SQUAD_OK : SQUAD_ERR_CUDA;
+  }
   const int first = p->order == SQUAD_LOCAL_THEN_GLOBAL ? kLocal : kGlobal;
   const int second = p->order == SQUAD_LOCAL_THEN_GLOBAL ? kGlobal : kLocal;
 
@@ -426,6 +486,7 @@ squad_status_t squad_attn_bwd(const squad_params_t* p, const void* q, const void
       b1.dk_out = static_cast<__nv_bfloat16*>(dk);
       b1.dv_out = static_cast<__nv_bfloat16*>(dv);
       b1.final_out = 1;
+      b1.accumulate = 1;
       if (launch_bwd_tc(b2, stream) != cudaSuccess) return SQUAD_ERR_CUDA;
       if (launch_bwd_tc(b1, stream) != cudaSuccess) return SQUAD_ERR_CUDA;
       return SQUAD_OK;

@@ -556,20 +556,23 @@ __global__ void __launch_bounds__(kThreads, 1) short_kernel(const __grid_constan
       const uint32_t row_addr = smem_u32(ring + v_off) + static_cast<uint32_t>(vrow) * 128u;
       const bool store_row = row < valid;
       const float inv_l = active ? 1.f / l : 0.f;
+      {
+        // both halves of O into registers (the first packed to bf16 at once), then release O
+        uint32_t pk0[32], o[64];
+        if (active) tmem_ld64(t_o, o);
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t o[64];
-        if (active) tmem_ld64(t_o + 64 * h, o);
-        if (h == 1) {
-          // O has been read into registers: the next unit's S may overwrite it
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&bars->o_free[wg]);
-        }
+        for (int i = 0; i < 32; ++i) pk0[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
+        if (active) tmem_ld64(t_o + 64, o);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->o_free[wg]);
         if (store_row) {
 #pragma unroll
           for (int c = 0; c < 8; ++c)
-            st_shared_v4(row_addr + h * panel + ((c ^ (vrow & 7)) << 4),
+            st_shared_v4(row_addr + ((c ^ (vrow & 7)) << 4), pk0[4 * c], pk0[4 * c + 1], pk0[4 * c + 2], pk0[4 * c + 3]);
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            st_shared_v4(row_addr + panel + ((c ^ (vrow & 7)) << 4),
                          pack_bf16x2(__uint_as_float(o[c * 8 + 0]) * inv_l, __uint_as_float(o[c * 8 + 1]) * inv_l),
                          pack_bf16x2(__uint_as_float(o[c * 8 + 2]) * inv_l, __uint_as_float(o[c * 8 + 3]) * inv_l),
                          pack_bf16x2(__uint_as_float(o[c * 8 + 4]) * inv_l, __uint_as_float(o[c * 8 + 5]) * inv_l),
@@ -623,7 +626,7 @@ bool short_plan(ShortArgs& a) {
   }
   a.smem_bytes = fixed + a.ring_bytes;
   const int H = a.g.B * a.g.h;
-  a.lag = a.n_passes == 2 ? (H < 2 ? H : 2) : 0;
+  a.lag = a.n_passes == 2 ? (H < 4 ? H : 4) : 0;
   a.f_u0 = make_fastdiv(static_cast<uint32_t>(a.pass[0].units_per_head));
   if (a.n_passes == 2) {
     a.f_u1 = make_fastdiv(static_cast<uint32_t>(a.pass[1].units_per_head));

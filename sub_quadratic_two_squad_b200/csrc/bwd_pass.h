@@ -23,7 +23,8 @@ struct BwdTcArgs {
   __nv_bfloat16* dk_out;      // final dK (final_out only)
   __nv_bfloat16* dv_out;      // gradient of this pass's values
   float scale, scale_log2;
-  int final_out;              // add the other pass's share and write dq_out / dk_out
+  int final_out;              // write dq_out / dk_out (bf16) instead of the fp32 shares
+  int accumulate;             // with final_out: add the other pass's fp32 share first
   uint32_t panel_bytes;       // rows (rounded to 8) x 128 bytes
   uint32_t guard_bytes, smem_bytes;
   uint32_t* status;           // device status word (0 = ok, 4 = a wait timed out)

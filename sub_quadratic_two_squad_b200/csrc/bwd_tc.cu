@@ -301,7 +301,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
         {
           const size_t ro = gi * 128;
           if (a.final_out)
-            write_row(t_row + N, tok >= 0, a.scale, a.dq_acc + ro, a.dq_out + ro, nullptr);
+            write_row(t_row + N, tok >= 0, a.scale, a.accumulate ? a.dq_acc + ro : nullptr, a.dq_out + ro, nullptr);
           else
             write_row(t_row + N, tok >= 0, a.scale, nullptr, nullptr, a.dq_acc + ro);
         }
@@ -352,7 +352,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
           const size_t ro = gi * 128;
           write_row(t_row + 256, tok >= 0, 1.f, nullptr, a.dv_out + ro, nullptr);
           if (a.final_out)
-            write_row(t_row + 384, tok >= 0, a.scale, a.dk_acc + ro, a.dk_out + ro, nullptr);
+            write_row(t_row + 384, tok >= 0, a.scale, a.accumulate ? a.dk_acc + ro : nullptr, a.dk_out + ro, nullptr);
           else
             write_row(t_row + 384, tok >= 0, a.scale, nullptr, nullptr, a.dk_acc + ro);
         }

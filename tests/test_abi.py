@@ -68,6 +68,8 @@ def _fwd(lib, prm, ptr=16):
     (dict(d=0), _lib.SQUAD_ERR_INVALID_ARG),
     (dict(B=0), _lib.SQUAD_ERR_INVALID_ARG),
     (dict(order=7), _lib.SQUAD_ERR_INVALID_ARG),
+    (dict(order=4), _lib.SQUAD_ERR_INVALID_ARG),
+    (dict(order=-1), _lib.SQUAD_ERR_INVALID_ARG),
     (dict(dtype=5), _lib.SQUAD_ERR_INVALID_ARG),
     (dict(scale=-1.0), _lib.SQUAD_ERR_INVALID_ARG),
     (dict(scale=float("nan")), _lib.SQUAD_ERR_INVALID_ARG),
@@ -99,6 +101,21 @@ def test_flops_match_the_oracle_cost_model(lib, cfg):
     n, w = grid[0] * grid[1] * grid[2], window[0] * window[1] * window[2]
     assert lib.squad_attn_flops(ctypes.byref(prm)) == pytest.approx(orc.squad_flops(B, h, d, n, w), rel=1e-12)
     assert lib.full_attn_flops(ctypes.byref(prm)) == pytest.approx(orc.full_flops(B, h, d, n), rel=1e-12)
+
+
+@pytest.mark.parametrize("cfg", [(1, 24, 128, (21, 22, 40), (21, 2, 4)), (1, 4, 64, (5, 8, 8), (5, 2, 2))])
+def test_single_pass_orders_accepted_and_counted(lib, cfg):
+    """local_only / global_only: one pass each, so their FLOPs are the two terms of the two-pass count."""
+    B, h, d, grid, window = cfg
+    n, w = grid[0] * grid[1] * grid[2], window[0] * window[1] * window[2]
+    fl = {}
+    for order in ("local_only", "global_only"):
+        prm = make_params(B, h, d, grid, window, order)
+        assert lib.squad_attn_fwd_workspace_bytes(ctypes.byref(prm)) > 0
+        assert lib.squad_attn_bwd_workspace_bytes(ctypes.byref(prm)) > 0
+        fl[order] = lib.squad_attn_flops(ctypes.byref(prm))
+    assert fl["local_only"] == pytest.approx(4.0 * B * h * d * n * w, rel=1e-12)
+    assert fl["local_only"] + fl["global_only"] == pytest.approx(orc.squad_flops(B, h, d, n, w), rel=1e-12)
 
 
 def test_workspace_sizes(lib):

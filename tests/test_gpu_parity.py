@@ -18,7 +18,8 @@ from sub_quadratic_two_squad_b200.inputs import make_inputs
 pytestmark = pytest.mark.gpu
 
 LG, GL = "local_then_global", "global_then_local"
-ORC_ORDER = {LG: orc.LOCAL_THEN_GLOBAL, GL: orc.GLOBAL_THEN_LOCAL}
+LO, GO = "local_only", "global_only"
+ORC_ORDER = {LG: orc.LOCAL_THEN_GLOBAL, GL: orc.GLOBAL_THEN_LOCAL, LO: orc.LOCAL_ONLY, GO: orc.GLOBAL_ONLY}
 
 
 def _dev(x, dtype):
@@ -185,3 +186,26 @@ def test_backward_small_bf16(order):
 
 def test_backward_wan21_14b():
     run_bwd(1, 40, 128, (21, 22, 40), (21, 2, 4), LG, torch.bfloat16, heads=[0, 13, 27, 39])
+
+
+# ------------------------------------------------------------------------------------------------
+# single-pass variants (one pass alone)
+# ------------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("order", [LO, GO])
+def test_single_pass_tiny_fp32(order):
+    run_fwd(1, 4, 64, (5, 8, 8), (5, 2, 2), order, torch.float32)
+    run_bwd(1, 4, 64, (5, 8, 8), (5, 2, 2), order, torch.float32)
+
+
+@pytest.mark.parametrize("order", [LO, GO])
+def test_single_pass_small_bf16(order):
+    run_fwd(2, 2, 128, (21, 4, 8), (21, 2, 4), order, torch.bfloat16)
+    run_bwd(2, 2, 128, (21, 4, 8), (21, 2, 4), order, torch.bfloat16)
+
+
+@pytest.mark.parametrize("order", [LO, GO])
+def test_single_pass_wan22_5b_shape(order):
+    """Windows of 168 and slot sequences of 110 tokens, one pass, forward and backward (2 heads)."""
+    run_fwd(1, 24, 128, (21, 22, 40), (21, 2, 4), order, torch.bfloat16, heavy_tail=True, heads=[0, 23])
+    run_bwd(1, 2, 128, (21, 22, 40), (21, 2, 4), order, torch.bfloat16)
