@@ -33,6 +33,14 @@ Readings where the pages are silent (equations 7-9 were lost in extraction):
   row-major over (H/hw, W/ww); slot j = (t, dy, dx) runs row-major over (tw, hw, ww). The result does
   not depend on these orders (softmax sums are permutation invariant; outputs go back to token order).
 * The backward pass is the chain rule through both passes; the pages do not print it.
+* Grids the window does not divide (paper appendix, "Conformance to the theoretical curves is
+  quantitative": such a window "forces a little reflect padding", and the window is re-solved per
+  resolution with w_t = T and w_h:w_w following the grid's aspect ratio). Readings: reflect padding
+  (the edge token is not repeated) at the bottom of H and the right of W in every frame, up to the next
+  multiple of the window; both passes run on the padded grid and the output is cropped back, so the
+  gradient of an input token sums over its padded copies. The solver takes, among windows with
+  w_t = T and for each w_h the w_w whose ratio w_h:w_w is closest to H:W (log ratio), the one with the
+  least cost n'm + n'^2/m on the padded count n'.
 
 Every array here is float64. Pins: tests/test_oracle_pins.py.
 """
@@ -151,6 +159,82 @@ def _f64(x):
     return np.asarray(x, dtype=np.float64)
 
 
+# ----------------------------------------------------------------------------------------------
+# Grids the window does not divide: reflect padding, cropping, and the window solver
+# ----------------------------------------------------------------------------------------------
+
+def padded_grid(grid, window):
+    """(T, H', W'): H and W rounded up to multiples of the window's hw and ww."""
+    T, H, W = grid
+    _, hw, ww = window
+    return T, -(-H // hw) * hw, -(-W // ww) * ww
+
+
+def divides(grid, window):
+    return tuple(padded_grid(grid, window)) == tuple(grid)
+
+
+def reflect_pad_tokens(X, grid, window):
+    """[B, h, n, d] -> [B, h, n', d]: each frame reflect-padded at the bottom and right ends."""
+    T, H, W = grid
+    _, Hp, Wp = padded_grid(grid, window)
+    if Hp - H > H - 1 or Wp - W > W - 1:
+        raise ValueError("reflect padding needs a pad shorter than the extent")
+    B, h, n, d = X.shape
+    x = np.asarray(X).reshape(B, h, T, H, W, d)
+    x = np.pad(x, ((0, 0), (0, 0), (0, 0), (0, Hp - H), (0, Wp - W), (0, 0)), mode="reflect")
+    return x.reshape(B, h, T * Hp * Wp, d)
+
+
+def crop_tokens(X, grid, window):
+    """[B, h, n', d] -> [B, h, n, d]: the tokens of the original grid."""
+    T, H, W = grid
+    _, Hp, Wp = padded_grid(grid, window)
+    B, h, _, d = X.shape
+    return np.ascontiguousarray(np.asarray(X).reshape(B, h, T, Hp, Wp, d)[:, :, :, :H, :W]).reshape(B, h, T * H * W, d)
+
+
+def fold_reflect_grad(G, grid, window):
+    """Adjoint of reflect_pad_tokens: the gradient on the padded grid summed onto the source tokens."""
+    T, H, W = grid
+    _, Hp, Wp = padded_grid(grid, window)
+    B, h, _, d = G.shape
+    g = np.asarray(G).reshape(B, h, T, Hp, Wp, d)
+    src_y = np.array([i if i < H else 2 * (H - 1) - i for i in range(Hp)])
+    src_x = np.array([i if i < W else 2 * (W - 1) - i for i in range(Wp)])
+    out = np.zeros((B, h, T, H, W, d), dtype=np.float64)
+    for yp in range(Hp):
+        for xp in range(Wp):
+            out[:, :, :, src_y[yp], src_x[xp]] += g[:, :, :, yp, xp]
+    return out.reshape(B, h, T * H * W, d)
+
+
+def _aspect_ww(hw: int, H: int, W: int) -> int:
+    """The ww whose ratio hw:ww is closest to H:W (in log ratio; the lower one on a tie)."""
+    lo = max(1, int(np.floor(hw * W / H)))
+    cands = (lo, lo + 1)
+    return min(cands, key=lambda ww: (abs(np.log(hw / ww) - np.log(H / W)), ww))
+
+
+def window_solve(T: int, H: int, W: int):
+    """The window (T, hw, ww) for a T x H x W grid: w_t = T, ww following the aspect ratio for each hw,
+    and the hw whose padded cost n'm + n'^2/m (m = T hw ww, n' = the reflect-padded token count) is
+    least."""
+    best = None
+    for hw in range(1, H + 1):
+        ww = _aspect_ww(hw, H, W)
+        if ww > W:
+            continue
+        _, Hp, Wp = padded_grid((T, H, W), (T, hw, ww))
+        if Hp - H > H - 1 or Wp - W > W - 1:
+            continue
+        n_p, m = T * Hp * Wp, T * hw * ww
+        cost = n_p * m + n_p * n_p / m
+        if best is None or cost < best[0]:
+            best = (cost, hw, ww)
+    return T, best[1], best[2]
+
+
 LOCAL_THEN_GLOBAL = "local_then_global"
 GLOBAL_THEN_LOCAL = "global_then_local"
 # Single-pass variants: each pass alone, as the paper ablates them (SQuad paper §4.4, "The need for and
@@ -167,6 +251,14 @@ def squad_attn_fwd(Q, K, V, grid, window, order=LOCAL_THEN_GLOBAL, scale=None, r
     With return_aux, also returns dict(o1=..., lse1=..., lse2=...) (pass-1 output and both passes'
     log-sum-exp).
     """
+    if not divides(grid, window):
+        # reflect-pad, run on the padded grid, crop the output (aux arrays stay on the padded grid)
+        pg = padded_grid(grid, window)
+        res = squad_attn_fwd(*(reflect_pad_tokens(_f64(X), grid, window) for X in (Q, K, V)), pg, window, order,
+                             scale, return_aux)
+        o = res[0] if return_aux else res
+        o = crop_tokens(o, grid, window)
+        return (o, res[1]) if return_aux else o
     if order in SINGLE_PASS:
         o, lse = (local_pass if order == LOCAL_ONLY else global_pass)(Q, K, V, grid, window, scale)
         return (o, dict(lse1=lse)) if return_aux else o
@@ -188,6 +280,16 @@ def squad_attn_bwd(Q, K, V, dO, grid, window, order=LOCAL_THEN_GLOBAL, scale=Non
     and dK, and dV. Q and K are used by both passes, so each receives the sum of two terms.
     """
     Q, K, V, dO = _f64(Q), _f64(K), _f64(V), _f64(dO)
+    if not divides(grid, window):
+        # the padded method: pad (reflect), both passes, crop; so dO is zero on the padded tokens and
+        # each input token's gradient sums over its padded copies
+        pg = padded_grid(grid, window)
+        B, h, _, d = dO.shape
+        do_p = np.zeros((B, h, pg[0] * pg[1] * pg[2], d))
+        do_p.reshape(B, h, pg[0], pg[1], pg[2], d)[:, :, :, :grid[1], :grid[2]] = dO.reshape(B, h, *grid, d)
+        grads = squad_attn_bwd(*(reflect_pad_tokens(X, grid, window) for X in (Q, K, V)), do_p, pg, window, order,
+                               scale)
+        return tuple(fold_reflect_grad(G, grid, window) for G in grads)
     sc = _scale(Q.shape[-1], scale)
     table = window_partition(*grid, *window)
     local_groups, global_groups = table, np.ascontiguousarray(table.T)

@@ -335,3 +335,85 @@ def test_single_passes_compose_to_squad():
     o_g = orc.squad_attn_fwd(q, k, v, grid, window, orc.GLOBAL_ONLY)
     np.testing.assert_allclose(orc.squad_attn_fwd(q, k, o_g, grid, window, orc.LOCAL_ONLY),
                                orc.squad_attn_fwd(q, k, v, grid, window, orc.GLOBAL_THEN_LOCAL), rtol=1e-12, atol=1e-13)
+
+
+# ------------------------------------------------------------------------------------------------
+# grids the window does not divide: reflect padding and the window solver
+# ------------------------------------------------------------------------------------------------
+
+def test_window_solver_recovers_the_trained_window():
+    """The pages: the rule recovers the trained 21x2x4 window at both backbones' native resolutions."""
+    assert orc.window_solve(21, 22, 40) == (21, 2, 4)
+    assert orc.window_solve(21, 30, 52) == (21, 2, 4)
+
+
+@pytest.mark.parametrize("grid", [(21, 22, 40), (21, 30, 52), (21, 44, 80), (21, 60, 104), (13, 17, 29), (5, 8, 8)])
+def test_window_solver_tracks_sqrt_n_and_is_locally_optimal(grid):
+    """m stays within a factor 2 of sqrt(n), spans all frames, and no neighbouring window with the
+    same aspect rule has a lower padded cost."""
+    T, H, W = grid
+    t, hw, ww = orc.window_solve(T, H, W)
+    n = T * H * W
+    assert t == T and 0.5 <= T * hw * ww / np.sqrt(n) <= 2.0
+
+    def cost(h_):
+        w_ = orc._aspect_ww(h_, H, W)
+        _, hp, wp = orc.padded_grid(grid, (T, h_, w_))
+        if hp - H > H - 1 or wp - W > W - 1 or w_ > W:
+            return np.inf
+        n_p, m = T * hp * wp, T * h_ * w_
+        return n_p * m + n_p * n_p / m
+    for nb in (hw - 1, hw + 1):
+        if 1 <= nb <= H:
+            assert cost(hw) <= cost(nb)
+
+
+@pytest.mark.parametrize("grid,window", [((2, 5, 7), (2, 2, 3)), ((3, 7, 4), (3, 3, 3))])
+def test_reflect_pad_is_torch_reflect(grid, window):
+    T, H, W = grid
+    _, Hp, Wp = orc.padded_grid(grid, window)
+    x = _rand((1, 2, T * H * W, 3), 5)
+    ref = torch.nn.functional.pad(torch.from_numpy(x).reshape(2 * T, H, W, 3).permute(0, 3, 1, 2),
+                                  (0, Wp - W, 0, Hp - H), mode="reflect")
+    ref = ref.permute(0, 2, 3, 1).reshape(1, 2, T * Hp * Wp, 3).numpy()
+    np.testing.assert_array_equal(orc.reflect_pad_tokens(x, grid, window), ref)
+
+
+def test_fold_is_the_adjoint_of_reflect_pad():
+    grid, window = (2, 5, 7), (2, 2, 3)
+    T, Hp, Wp = orc.padded_grid(grid, window)
+    x = _rand((1, 1, 2 * 5 * 7, 4), 6)
+    y = _rand((1, 1, T * Hp * Wp, 4), 7)
+    lhs = np.sum(orc.reflect_pad_tokens(x, grid, window) * y)
+    rhs = np.sum(x * orc.fold_reflect_grad(y, grid, window))
+    assert lhs == pytest.approx(rhs, rel=1e-12)
+
+
+@pytest.mark.parametrize("order", ORDERS + [orc.LOCAL_ONLY, orc.GLOBAL_ONLY])
+@pytest.mark.parametrize("grid,window", [((2, 5, 7), (2, 2, 3)), ((3, 7, 4), (3, 3, 3))])
+def test_padded_method_matches_torch_construction(order, grid, window):
+    """Reflect-pad with torch, the two masked dense attentions on the padded coordinates (values of the
+    second = output of the first), crop; forward and autograd backward against the oracle."""
+    T, H, W = grid
+    _, Hp, Wp = orc.padded_grid(grid, window)
+    same_window, same_slot = _masks(T, Hp, Wp, window[1], window[2])
+    masks = {orc.LOCAL_THEN_GLOBAL: (same_window, same_slot), orc.GLOBAL_THEN_LOCAL: (same_slot, same_window),
+             orc.LOCAL_ONLY: (same_window,), orc.GLOBAL_ONLY: (same_slot,)}[order]
+    q, k, v, do = (_rand((1, 2, T * H * W, 4), s) for s in (31, 32, 33, 34))
+    sc = 0.6
+    tq, tk, tv = (torch.from_numpy(x).requires_grad_(True) for x in (q, k, v))
+
+    def pad(t):
+        x = t.reshape(2 * T, H, W, 4).permute(0, 3, 1, 2)
+        x = torch.nn.functional.pad(x, (0, Wp - W, 0, Hp - H), mode="reflect")
+        return x.permute(0, 2, 3, 1).reshape(1, 2, T * Hp * Wp, 4)
+    pq, pk, vals = pad(tq), pad(tk), pad(tv)
+    for m in masks:
+        vals = _masked_attention_torch(pq, pk, vals, m, sc)
+    out = vals.reshape(1, 2, T, Hp, Wp, 4)[:, :, :, :H, :W].reshape(1, 2, T * H * W, 4)
+    np.testing.assert_allclose(orc.squad_attn_fwd(q, k, v, grid, window, order, scale=sc), out.detach().numpy(),
+                               rtol=1e-12, atol=1e-12)
+    out.backward(torch.from_numpy(do))
+    dq, dk, dv = orc.squad_attn_bwd(q, k, v, do, grid, window, order, scale=sc)
+    for got, ref in ((dq, tq.grad), (dk, tk.grad), (dv, tv.grad)):
+        np.testing.assert_allclose(got, ref.numpy(), rtol=1e-10, atol=1e-12)
