@@ -29,8 +29,8 @@ PAGES_MS = 4.27   # pages' SQuad attention latency per block for this workload (
 # DRAM traffic of one launch of the forward kernel from the ncu capture summarised in
 # profiles/short_kernel_wan22_5b_fwd.md (dram__bytes_read.sum + dram__bytes_write.sum), valid only for
 # the kernel source it was measured on (sha1 prefix below); otherwise reported as null.
-PROFILED_TRAFFIC_BYTES = (442.92224 + 194.259456) * 1e6
-PROFILED_KERNEL_SHA1 = "02bb1d3717706da7"
+PROFILED_TRAFFIC_BYTES = (438.608128 + 193.176576) * 1e6
+PROFILED_KERNEL_SHA1 = "972f88535881708b"
 PROFILED_KERNEL_SRC = os.path.join(ROOT, "sub_quadratic_two_squad_b200", "csrc", "attn_short.cu")
 
 
@@ -355,13 +355,85 @@ def run_ours(args, rank, world, local_rank):
         "single_pass": single,
         "backward": {"ms_per_block": bwd_ms,
                      "tflops_algorithmic": 2.0 * f / (bwd_ms * 1e-3) / 1e12,
-                     "flops_note": "algorithmic = 2x forward (dQ, dK, dV, dP products); the kernels execute 3.5x "
-                                   "forward (S and dP recomputed in both the row and the column kernel)",
-                     "kernels": "tcgen05 row (dQ, D) and column (dK, dV) kernels, 2 per pass"},
+                     "flops_note": "algorithmic = 2x forward (dQ, dK, dV, dP products); the kernel executes 3.5x "
+                                   "forward (S and dP recomputed for the row and for the column products)",
+                     "kernels": "tcgen05 bwd_tc_kernel, one launch per pass (rows: dQ, D; columns: dK, dV)"},
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
     print(json.dumps(line), flush=True)
+
+
+# Every block shape the measurements cover (name, B, h, d, grid, window, orders, with full attention,
+# with backward). Timed by `--sweep`, one JSON line each; the default run times only the 5B block.
+SWEEP = [
+    ("Wan-2.2-5B block", 1, 24, 128, (21, 22, 40), (21, 2, 4),
+     ("local_then_global", "global_then_local", "local_only", "global_only"), True, True),
+    ("Wan-2.1-1.3B block", 1, 12, 128, (21, 30, 52), (21, 2, 4), ("local_then_global", "global_then_local"), False, False),
+    ("high-resolution 5B block", 1, 24, 128, (21, 44, 80), (21, 4, 4), ("local_then_global",), True, False),
+    ("Wan-2.1-14B block (training step)", 1, 40, 128, (21, 22, 40), (21, 2, 4), ("local_then_global",), False, True),
+]
+
+
+def sweep(reps=30):
+    """Forward (and backward, full attention) device times for every block shape, N(0,1) inputs drawn on
+    the device, 3 rotating buffer sets, CUDA events on the launching stream."""
+    import torch
+
+    from sub_quadratic_two_squad_b200 import full_attn_fwd, squad_attn_bwd, squad_attn_fwd
+
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream()
+    hbm, tf_peak, peak_kind = peaks()
+
+    def timed(fn, n_rep):
+        fn(0)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for i in range(n_rep):
+            fn(i)
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / n_rep
+
+    for name, B, h, d, grid, window, orders, with_full, with_bwd in SWEEP:
+        w = dict(B=B, h=h, d=d, grid=grid, window=window)
+        n = n_tokens(w)
+        sets = [tuple(torch.randn(B, h, n, d, device=dev, dtype=torch.bfloat16) for _ in range(3)) for _ in range(3)]
+        outs = [torch.empty_like(x[0]) for x in sets]
+        for order in orders:
+            wss = [squad_attn_fwd(*sets[i], grid, window, order)[1] for i in range(3)]
+            ms = timed(lambda i: squad_attn_fwd(*sets[i % 3], grid, window, order, out=outs[i % 3],
+                                                workspace=wss[i % 3]), reps)
+            nw = window[0] * window[1] * window[2]
+            terms = {"local_only": n * nw, "global_only": n * n / nw}.get(order, n * nw + n * n / nw)
+            f = 4.0 * B * h * d * terms
+            t_roof = max(f / (tf_peak * 1e12), alg_bytes(w) / (hbm * 1e9)) * 1e3
+            line = {"sweep": name, "order": order, "n": n, "window": "x".join(map(str, window)), "ms_per_block": ms,
+                    "tflops": f / (ms * 1e-3) / 1e12, "roofline_ms": t_roof, "roofline_frac": t_roof / ms,
+                    "hbm_gbs_algorithmic": alg_bytes(w) / (ms * 1e-3) / 1e9, "peaks": peak_kind}
+            if with_bwd and order == "local_then_global":
+                dout = torch.randn(B, h, n, d, device=dev, dtype=torch.bfloat16)
+                q, k, v = sets[0]
+                o, ws = squad_attn_fwd(q, k, v, grid, window, order)
+                g = squad_attn_bwd(q, k, v, o, dout, ws, grid, window, order)
+                bms = timed(lambda i: squad_attn_bwd(q, k, v, o, dout, ws, grid, window, order, dq=g[0], dk=g[1],
+                                                     dv=g[2]), 10)
+                bwd_bytes = 8 * B * h * n * d * 2   # Q, K, V, O, dO in; dQ, dK, dV out (bf16), + O1 once
+                line["backward"] = {"ms_per_block": bms, "tflops_algorithmic": 2 * f / (bms * 1e-3) / 1e12,
+                                    "hbm_frac_8_tensors": bwd_bytes / (bms * 1e-3) / 1e9 / hbm}
+            print(json.dumps(line), flush=True)
+            del wss
+        if with_full:
+            q, k, v = sets[0]
+            fms = timed(lambda i: full_attn_fwd(*sets[i % 3], grid=grid, out=outs[i % 3]), 3)
+            nf = 4.0 * B * h * d * n * n
+            print(json.dumps({"sweep": name, "order": "full_attn_fwd", "n": n, "ms_per_block": fms,
+                              "tflops": nf / (fms * 1e-3) / 1e12, "tensor_frac": nf / (fms * 1e-3) / 1e12 / tf_peak}),
+                  flush=True)
+        del sets, outs
+        torch.cuda.empty_cache()
 
 
 def main():
@@ -371,7 +443,11 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true", help="time every block shape (one JSON line each) and exit")
     args = ap.parse_args()
+    if args.sweep:
+        sweep()
+        return
     args.warmup = max(args.warmup, 3)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -407,7 +407,6 @@ squad_status_t squad_attn_bwd(const squad_params_t* p, const void* q, const void
             !encode_pass_map(&b.tm_v, v, g, b.p, b.variant) || !encode_pass_map(&b.tm_do, dout, g, b.p, b.variant))
           return SQUAD_ERR_CUDA;
         b.lse = fw.lse1;
-        b.drow = bw.drow;
         b.dq_acc = bw.dq_acc;
         b.dk_acc = bw.dk_acc;
         b.dq_out = static_cast<__nv_bfloat16*>(dq);
@@ -470,7 +469,6 @@ squad_status_t squad_attn_bwd(const squad_params_t* p, const void* q, const void
           !encode_pass_map(&b1.tm_v, v, g, b1.p, b1.variant) || !encode_pass_map(&b1.tm_do, do1, g, b1.p, b1.variant))
         return SQUAD_ERR_CUDA;
       for (BwdTcArgs* b : {&b2, &b1}) {
-        b->drow = bw.drow;
         b->dq_acc = bw.dq_acc;
         b->dk_acc = bw.dk_acc;
         b->scale = scale;

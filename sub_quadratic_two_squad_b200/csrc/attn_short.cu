@@ -626,7 +626,7 @@ bool short_plan(ShortArgs& a) {
   }
   a.smem_bytes = fixed + a.ring_bytes;
   const int H = a.g.B * a.g.h;
-  a.lag = a.n_passes == 2 ? (H < 4 ? H : 4) : 0;
+  a.lag = a.n_passes == 2 ? (H < 2 ? H : 2) : 0;
   a.f_u0 = make_fastdiv(static_cast<uint32_t>(a.pass[0].units_per_head));
   if (a.n_passes == 2) {
     a.f_u1 = make_fastdiv(static_cast<uint32_t>(a.pass[1].units_per_head));

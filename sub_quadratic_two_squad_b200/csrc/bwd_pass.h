@@ -16,7 +16,6 @@ struct BwdTcArgs {
   PassGeom p;                 // one chunk per sequence (make_geom(..., 256))
   int variant;                // slot-box encoding (GLOBAL pass)
   const float* lse;           // [B, h, n] natural-log LSE of this pass's forward
-  float* drow;                // [B, h, n] D_i = sum_j P_ij dP_ij: written by the row kernel, read by the column kernel
   float* dq_acc;              // [B, h, n, d] fp32 share of dQ (written, or read and completed when final)
   float* dk_acc;              // [B, h, n, d] fp32 share of dK (likewise)
   __nv_bfloat16* dq_out;      // final dQ (final_out only)
@@ -33,7 +32,7 @@ struct BwdTcArgs {
 
 // Fills the shared-memory plan of `a` (p and g set); false if the sequences do not fit.
 bool bwd_tc_plan(BwdTcArgs& a);
-// Row kernel (dQ, D) then column kernel (dK, dV) of one pass.
+// One pass's gradients: dQ, then dK and dV, in one launch (one CTA per sequence).
 cudaError_t launch_bwd_tc(const BwdTcArgs& a, cudaStream_t stream);
 
 }  // namespace squad

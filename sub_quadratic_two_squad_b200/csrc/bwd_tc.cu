@@ -8,13 +8,14 @@
 //   dP = dO V^T,  D_i = sum_j P_ij dP_ij,  dS = P o (dP - D),
 //   dQ = scale dS K,  dK = scale dS^T Q,  dV = P^T dO.
 //
-// One CTA per sequence (160 threads): warps 0-3 own one TMEM lane (one row) per thread, warp 4
-// loads the sequence's Q, K, V, dO as whole TMA boxes and issues the tcgen05 MMAs.
-//   row kernel, per 128-query tile: S = Q K^T and dP = dO V^T into TMEM; the warps form P (bf16) and D,
-//     then dS (bf16, packed two per column over S); dQ = dS K (A from TMEM); D and dQ are written out.
-//   column kernel, per 128-key tile and 128-query chunk: S^T = K Q^T and dP^T = V dO^T into TMEM; with
-//     the per-query LSE and D of the sequence the warps form P^T and dS^T (packed over S^T and dP^T);
-//     dV += P^T dO and dK += dS^T Q accumulate in TMEM over the chunks; dV and dK are written out.
+// One kernel per pass, one CTA per sequence (160 threads): warps 0-3 own one TMEM lane (one row) per
+// thread, warp 4 loads the sequence's Q, K, V, dO once as whole TMA boxes and issues the tcgen05 MMAs.
+//   rows, per 128-query tile: S = Q K^T and dP = dO V^T into TMEM; the warps form P (bf16) and D, then
+//     dS (bf16, packed two per column over S); dQ = dS K (A from TMEM) is written out. Each row's LSE
+//     and D stay in shared memory.
+//   columns, per 128-key tile and 128-query chunk: S^T = K Q^T and dP^T = V dO^T into TMEM; with the
+//     per-query LSE and D the warps form P^T and dS^T (packed over S^T and dP^T); dV += P^T dO and
+//     dK += dS^T Q accumulate in TMEM over the chunks and are written out.
 // Rows past the sequence are computed and dropped; columns past it are masked to P = dS = 0, and the
 // shared-memory rows past each box are zeroed so every MMA operand is finite.
 #include <cuda_runtime.h>
@@ -91,7 +92,6 @@ __device__ __forceinline__ void write_row(uint32_t taddr, bool store, float mul,
   }
 }
 
-template <bool kCols>
 __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_constant__ BwdTcArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -100,14 +100,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
   uint8_t* const sk = base + alloc;
   uint8_t* const sv = base + 2 * alloc;
   uint8_t* const sdo = base + 3 * alloc;
-  float* const lse_s = reinterpret_cast<float*>(base + 4 * alloc + a.guard_bytes);
-  float* const d_s = lse_s + 256;
+  float* const lse_s = reinterpret_cast<float*>(base + 4 * alloc + a.guard_bytes);   // per query, log2 units
+  float* const d_s = lse_s + 256;                                                     // per query D
   BwdBars* const bars = reinterpret_cast<BwdBars*>(d_s + 256);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const Grid& g = a.g;
   const PassGeom& p = a.p;
   const int s = p.seq_len;
+  const int N = round16b(s);
   const int ntiles = (s + 127) / 128;
   const int bh = static_cast<int>(fdiv(blockIdx.x, p.f_per_bh));
   const int sigma = static_cast<int>(blockIdx.x) - bh * p.n_seq;
@@ -123,15 +124,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
     }
     for (uint32_t i = threadIdx.x; i < a.guard_bytes / 16u; i += kBwdThreads)
       reinterpret_cast<uint4*>(base + 4 * alloc)[i] = make_uint4(0, 0, 0, 0);
-  }
-  if (kCols) {
-    // per-query LSE (log2 units; +inf past the sequence, so P = 0 there) and D of this sequence
-    for (int j = threadIdx.x; j < 256; j += kBwdThreads) {
-      const int tok = j < s ? token_of(g, p, sigma, 0, j) : -1;
-      const size_t gi = static_cast<size_t>(bh) * g.n + (tok < 0 ? 0 : tok);
-      lse_s[j] = tok >= 0 ? a.lse[gi] * kLog2e : INFINITY;
-      d_s[j] = tok >= 0 ? a.drow[gi] : 0.f;
-    }
   }
   if (threadIdx.x == 128) {
     mbar_init(&bars->load, 1);
@@ -182,63 +174,59 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
       bool ok = mbar_wait(&bars->load, 0, ctl);
       tc_fence_after();
       const uint32_t aq = smem_u32(sq), ak = smem_u32(sk), av = smem_u32(sv), ado = smem_u32(sdo);
-      if (!kCols) {
-        const int N = round16b(s);
-        const uint32_t idesc_s = idesc_bf16(128, N, false);
-        for (int t = 0; t < ntiles && ok; ++t) {
-          if (t > 0) {   // dQ of the previous tile (over dP) has been read
-            ok = mbar_wait(&bars->o_free, (t - 1) & 1, ctl);
-            if (!ok) break;
-            tc_fence_after();
-          }
-          const uint32_t row_off = static_cast<uint32_t>(t) * 16384u;
-          for (int kk = 0; kk < 8; ++kk)   // S = Q_t K^T -> [0, N)
-            umma_bf16_ss(tmem, kdesc(aq + row_off, kk, panel), kdesc(ak, kk, panel), idesc_s, kk > 0);
-          for (int kk = 0; kk < 8; ++kk)   // dP = dO_t V^T -> [N, 2N)
-            umma_bf16_ss(tmem + N, kdesc(ado + row_off, kk, panel), kdesc(av, kk, panel), idesc_s, kk > 0);
+      uint32_t p_cnt = 0, f_cnt = 0;
+      // the row owners have read the previous tile's results out of tensor memory
+      auto wait_free = [&]() -> bool {
+        const bool r = mbar_wait(&bars->o_free, f_cnt & 1, ctl);
+        ++f_cnt;
+        if (r) tc_fence_after();
+        return r;
+      };
+      // rows: per 128-query tile, S and dP, then dQ = dS K
+      const uint32_t idesc_s = idesc_bf16(128, N, false);
+      for (int t = 0; t < ntiles && ok; ++t) {
+        if (t > 0 && !(ok = wait_free())) break;
+        const uint32_t row_off = static_cast<uint32_t>(t) * 16384u;
+        for (int kk = 0; kk < 8; ++kk)   // S = Q_t K^T -> [0, N)
+          umma_bf16_ss(tmem, kdesc(aq + row_off, kk, panel), kdesc(ak, kk, panel), idesc_s, kk > 0);
+        for (int kk = 0; kk < 8; ++kk)   // dP = dO_t V^T -> [N, 2N)
+          umma_bf16_ss(tmem + N, kdesc(ado + row_off, kk, panel), kdesc(av, kk, panel), idesc_s, kk > 0);
+        umma_commit(&bars->s_full);
+        ok = mbar_wait(&bars->p_full, p_cnt & 1, ctl);
+        ++p_cnt;
+        if (!ok) break;
+        tc_fence_after();
+        for (int kk = 0; kk < N / 16; ++kk)   // dQ = dS K -> [N, N + 128)
+          umma_bf16_ts(tmem + N, tmem + kk * 8, sw128_desc(ak + kk * 2048, panel, 1024), idesc_o, kk > 0);
+        umma_commit(&bars->o_full);
+      }
+      // columns: per 128-key tile, over 128-query chunks, S^T and dP^T, then dV += P^T dO, dK += dS^T Q
+      for (int kt = 0; kt < ntiles && ok; ++kt) {
+        if (!(ok = wait_free())) break;   // tensor memory free (the last dQ, or the previous dV and dK, read)
+        const uint32_t key_off = static_cast<uint32_t>(kt) * 16384u;
+        for (int qc = 0; qc < ntiles && ok; ++qc) {
+          const int nq = min(128, s - 128 * qc);
+          const int Nq = round16b(nq);
+          const uint32_t q_off = static_cast<uint32_t>(qc) * 16384u;
+          const uint32_t idesc_c = idesc_bf16(128, Nq, false);
+          for (int kk = 0; kk < 8; ++kk)   // S^T = K_kt Q_qc^T -> [0, Nq)
+            umma_bf16_ss(tmem, kdesc(ak + key_off, kk, panel), kdesc(aq + q_off, kk, panel), idesc_c, kk > 0);
+          for (int kk = 0; kk < 8; ++kk)   // dP^T = V_kt dO_qc^T -> [128, 128 + Nq)
+            umma_bf16_ss(tmem + 128, kdesc(av + key_off, kk, panel), kdesc(ado + q_off, kk, panel), idesc_c,
+                         kk > 0);
           umma_commit(&bars->s_full);
-          ok = mbar_wait(&bars->p_full, t & 1, ctl);
+          ok = mbar_wait(&bars->p_full, p_cnt & 1, ctl);
+          ++p_cnt;
           if (!ok) break;
           tc_fence_after();
-          for (int kk = 0; kk < N / 16; ++kk)   // dQ = dS K -> [N, N + 128)
-            umma_bf16_ts(tmem + N, tmem + kk * 8, sw128_desc(ak + kk * 2048, panel, 1024), idesc_o, kk > 0);
-          umma_commit(&bars->o_full);
+          for (int kk = 0; kk < Nq / 16; ++kk)   // dV += P^T dO_qc -> [256, 384)
+            umma_bf16_ts(tmem + 256, tmem + kk * 8, sw128_desc(ado + q_off + kk * 2048, panel, 1024), idesc_o,
+                         qc > 0 || kk > 0);
+          for (int kk = 0; kk < Nq / 16; ++kk)   // dK += dS^T Q_qc -> [384, 512)
+            umma_bf16_ts(tmem + 384, tmem + 128 + kk * 8, sw128_desc(aq + q_off + kk * 2048, panel, 1024), idesc_o,
+                         qc > 0 || kk > 0);
         }
-      } else {
-        uint32_t p_cnt = 0;
-        for (int kt = 0; kt < ntiles && ok; ++kt) {
-          if (kt > 0) {   // dV and dK of the previous key tile have been read
-            ok = mbar_wait(&bars->o_free, (kt - 1) & 1, ctl);
-            if (!ok) break;
-            tc_fence_after();
-          }
-          const uint32_t key_off = static_cast<uint32_t>(kt) * 16384u;
-          for (int qc = 0; qc < ntiles && ok; ++qc) {
-            const int nq = min(128, s - 128 * qc);
-            const int Nq = round16b(nq);
-            const uint32_t q_off = static_cast<uint32_t>(qc) * 16384u;
-            const uint32_t idesc_s = idesc_bf16(128, Nq, false);
-            for (int kk = 0; kk < 8; ++kk)   // S^T = K_kt Q_qc^T -> [0, Nq)
-              umma_bf16_ss(tmem, kdesc(ak + key_off, kk, panel), kdesc(aq + q_off, kk, panel), idesc_s, kk > 0);
-            for (int kk = 0; kk < 8; ++kk)   // dP^T = V_kt dO_qc^T -> [128, 128 + Nq)
-              umma_bf16_ss(tmem + 128, kdesc(av + key_off, kk, panel), kdesc(ado + q_off, kk, panel), idesc_s,
-                           kk > 0);
-            umma_commit(&bars->s_full);
-            ok = mbar_wait(&bars->p_full, p_cnt & 1, ctl);
-            ++p_cnt;
-            if (!ok) break;
-            tc_fence_after();
-            for (int kk = 0; kk < Nq / 16; ++kk) {   // dV += P^T dO_qc -> [256, 384)
-              umma_bf16_ts(tmem + 256, tmem + kk * 8, sw128_desc(ado + q_off + kk * 2048, panel, 1024), idesc_o,
-                           qc > 0 || kk > 0);
-            }
-            for (int kk = 0; kk < Nq / 16; ++kk) {   // dK += dS^T Q_qc -> [384, 512)
-              umma_bf16_ts(tmem + 384, tmem + 128 + kk * 8, sw128_desc(aq + q_off + kk * 2048, panel, 1024), idesc_o,
-                           qc > 0 || kk > 0);
-            }
-          }
-          if (ok) umma_commit(&bars->o_full);
-        }
+        if (ok) umma_commit(&bars->o_full);
       }
       // every MMA issued has completed before the CTA frees tensor memory
       umma_commit(&bars->drain);
@@ -249,116 +237,122 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
     const int rl = warp * 32 + lane;   // TMEM lane of this thread
     const uint32_t t_row = tmem + (static_cast<uint32_t>(warp * 32) << 16);
     const float sl2 = a.scale_log2;
-    if (!kCols) {
-      const int N = round16b(s);
-      for (int t = 0; t < ntiles; ++t) {
-        const int r = 128 * t + rl;
-        const int tok = r < s ? token_of(g, p, sigma, 0, r) : -1;
-        const size_t gi = static_cast<size_t>(bh) * g.n + (tok < 0 ? 0 : tok);
-        const float lse2 = tok >= 0 ? a.lse[gi] * kLog2e : 0.f;
-        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&bars->s_full, t & 1, ctl))) break;   // warp-uniform exit
-        tc_fence_after();
-        // P (bf16, packed over the S columns already read) and D = sum_j P_ij dP_ij
-        float dsum[4] = {0.f, 0.f, 0.f, 0.f};
+    uint32_t s_cnt = 0, o_cnt = 0;
+    bool ok = true;
+    // rows: P and D, dS, dQ; each row's LSE (log2 units) and D go to shared memory for the columns
+    for (int t = 0; t < ntiles && ok; ++t) {
+      const int r = 128 * t + rl;
+      const int tok = r < s ? token_of(g, p, sigma, 0, r) : -1;
+      const size_t gi = static_cast<size_t>(bh) * g.n + (tok < 0 ? 0 : tok);
+      const float lse2 = tok >= 0 ? a.lse[gi] * kLog2e : 0.f;
+      ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->s_full, s_cnt & 1, ctl));   // warp-uniform exit
+      ++s_cnt;
+      if (!ok) break;
+      tc_fence_after();
+      // P (bf16, packed over the S columns already read) and D = sum_j P_ij dP_ij
+      float dsum[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 1
-        for (int c = 0; c < (N + 31) / 32; ++c) {
-          uint32_t sr[32], dr[32], pk[16];
-          tmem_ld32(t_row + 32 * c, sr);
-          tmem_ld32(t_row + N + 32 * c, dr);
+      for (int c = 0; c < (N + 31) / 32; ++c) {
+        uint32_t sr[32], dr[32], pk[16];
+        tmem_ld32(t_row + 32 * c, sr);
+        tmem_ld32(t_row + N + 32 * c, dr);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int j = 32 * c + 2 * i;
-            const float p0 = j < s ? ex2_approx(fmaf(__uint_as_float(sr[2 * i]), sl2, -lse2)) : 0.f;
-            const float p1 = j + 1 < s ? ex2_approx(fmaf(__uint_as_float(sr[2 * i + 1]), sl2, -lse2)) : 0.f;
-            if (j < s) dsum[i & 3] = fmaf(p0, __uint_as_float(dr[2 * i]), dsum[i & 3]);
-            if (j + 1 < s) dsum[(i + 2) & 3] = fmaf(p1, __uint_as_float(dr[2 * i + 1]), dsum[(i + 2) & 3]);
-            pk[i] = pack2_rn(p0, p1);
-          }
-          tmem_st16(t_row + 16 * c, pk);
+        for (int i = 0; i < 16; ++i) {
+          const int j = 32 * c + 2 * i;
+          const float p0 = j < s ? ex2_approx(fmaf(__uint_as_float(sr[2 * i]), sl2, -lse2)) : 0.f;
+          const float p1 = j + 1 < s ? ex2_approx(fmaf(__uint_as_float(sr[2 * i + 1]), sl2, -lse2)) : 0.f;
+          if (j < s) dsum[i & 3] = fmaf(p0, __uint_as_float(dr[2 * i]), dsum[i & 3]);
+          if (j + 1 < s) dsum[(i + 2) & 3] = fmaf(p1, __uint_as_float(dr[2 * i + 1]), dsum[(i + 2) & 3]);
+          pk[i] = pack2_rn(p0, p1);
         }
-        const float D = (dsum[0] + dsum[1]) + (dsum[2] + dsum[3]);
-        if (tok >= 0) a.drow[gi] = D;
-        // dS = P o (dP - D), packed over P
+        tmem_st16(t_row + 16 * c, pk);
+      }
+      const float D = (dsum[0] + dsum[1]) + (dsum[2] + dsum[3]);
+      lse_s[r] = tok >= 0 ? lse2 : INFINITY;   // +inf past the sequence: P = 0 in those columns
+      d_s[r] = tok >= 0 ? D : 0.f;
+      // dS = P o (dP - D), packed over P
 #pragma unroll 1
-        for (int c = 0; c < (N + 31) / 32; ++c) {
-          uint32_t pr[16], dr[32], pk[16];
-          tmem_ld16(t_row + 16 * c, pr);
-          tmem_ld32(t_row + N + 32 * c, dr);
+      for (int c = 0; c < (N + 31) / 32; ++c) {
+        uint32_t pr[16], dr[32], pk[16];
+        tmem_ld16(t_row + 16 * c, pr);
+        tmem_ld32(t_row + N + 32 * c, dr);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int j = 32 * c + 2 * i;
+          const float p0 = __uint_as_float(pr[i] << 16), p1 = __uint_as_float(pr[i] & 0xFFFF0000u);
+          const float s0 = j < s ? p0 * (__uint_as_float(dr[2 * i]) - D) : 0.f;
+          const float s1 = j + 1 < s ? p1 * (__uint_as_float(dr[2 * i + 1]) - D) : 0.f;
+          pk[i] = pack2_rn(s0, s1);
+        }
+        tmem_st16(t_row + 16 * c, pk);
+      }
+      tc_fence_before();
+      mbar_arrive(&bars->p_full);
+      ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->o_full, o_cnt & 1, ctl));
+      ++o_cnt;
+      if (!ok) break;
+      tc_fence_after();
+      {
+        const size_t ro = gi * 128;
+        if (a.final_out)
+          write_row(t_row + N, tok >= 0, a.scale, a.accumulate ? a.dq_acc + ro : nullptr, a.dq_out + ro, nullptr);
+        else
+          write_row(t_row + N, tok >= 0, a.scale, nullptr, nullptr, a.dq_acc + ro);
+      }
+      tc_fence_before();
+      mbar_arrive(&bars->o_free);
+    }
+    named_barrier_sync(1, 128);   // every row's LSE and D is in shared memory before the columns use them
+    // columns: P^T, dS^T per 128-query chunk; dV and dK once the chunks are accumulated
+    for (int kt = 0; kt < ntiles && ok; ++kt) {
+      const int key = 128 * kt + rl;
+      const int tok = key < s ? token_of(g, p, sigma, 0, key) : -1;
+      const size_t gi = static_cast<size_t>(bh) * g.n + (tok < 0 ? 0 : tok);
+      for (int qc = 0; qc < ntiles && ok; ++qc) {
+        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->s_full, s_cnt & 1, ctl));
+        ++s_cnt;
+        if (!ok) break;
+        tc_fence_after();
+        const int nq = min(128, s - 128 * qc);
+        // P^T over S^T and dS^T over dP^T, both bf16 packed two per column
+#pragma unroll 1
+        for (int c = 0; c < (nq + 31) / 32; ++c) {
+          uint32_t sr[32], dr[32], pp[16], ps[16];
+          tmem_ld32(t_row + 32 * c, sr);
+          tmem_ld32(t_row + 128 + 32 * c, dr);
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const int j = 32 * c + 2 * i;
-            const float p0 = __uint_as_float(pr[i] << 16), p1 = __uint_as_float(pr[i] & 0xFFFF0000u);
-            const float s0 = j < s ? p0 * (__uint_as_float(dr[2 * i]) - D) : 0.f;
-            const float s1 = j + 1 < s ? p1 * (__uint_as_float(dr[2 * i + 1]) - D) : 0.f;
-            pk[i] = pack2_rn(s0, s1);
+            const int j0 = 128 * qc + 32 * c + 2 * i;   // query index of the column pair
+            const int jl = 32 * c + 2 * i;               // within this chunk
+            const bool v0 = jl < nq, v1 = jl + 1 < nq;
+            const float p0 = v0 ? ex2_approx(fmaf(__uint_as_float(sr[2 * i]), sl2, -lse_s[j0])) : 0.f;
+            const float p1 = v1 ? ex2_approx(fmaf(__uint_as_float(sr[2 * i + 1]), sl2, -lse_s[j0 + 1])) : 0.f;
+            const float s0 = v0 ? p0 * (__uint_as_float(dr[2 * i]) - d_s[j0]) : 0.f;
+            const float s1 = v1 ? p1 * (__uint_as_float(dr[2 * i + 1]) - d_s[j0 + 1]) : 0.f;
+            pp[i] = pack2_rn(p0, p1);
+            ps[i] = pack2_rn(s0, s1);
           }
-          tmem_st16(t_row + 16 * c, pk);
+          tmem_st16(t_row + 16 * c, pp);
+          tmem_st16(t_row + 128 + 16 * c, ps);
         }
         tc_fence_before();
         mbar_arrive(&bars->p_full);
-        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&bars->o_full, t & 1, ctl))) break;
-        tc_fence_after();
-        {
-          const size_t ro = gi * 128;
-          if (a.final_out)
-            write_row(t_row + N, tok >= 0, a.scale, a.accumulate ? a.dq_acc + ro : nullptr, a.dq_out + ro, nullptr);
-          else
-            write_row(t_row + N, tok >= 0, a.scale, nullptr, nullptr, a.dq_acc + ro);
-        }
-        tc_fence_before();
-        mbar_arrive(&bars->o_free);
       }
-    } else {
-      uint32_t s_cnt = 0;
-      for (int kt = 0; kt < ntiles; ++kt) {
-        const int key = 128 * kt + rl;
-        const int tok = key < s ? token_of(g, p, sigma, 0, key) : -1;
-        const size_t gi = static_cast<size_t>(bh) * g.n + (tok < 0 ? 0 : tok);
-        bool ok = true;
-        for (int qc = 0; qc < ntiles; ++qc) {
-          ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->s_full, s_cnt & 1, ctl));
-          ++s_cnt;
-          if (!ok) break;
-          tc_fence_after();
-          const int nq = min(128, s - 128 * qc);
-          // P^T over S^T and dS^T over dP^T, both bf16 packed two per column
-#pragma unroll 1
-          for (int c = 0; c < (nq + 31) / 32; ++c) {
-            uint32_t sr[32], dr[32], pp[16], ps[16];
-            tmem_ld32(t_row + 32 * c, sr);
-            tmem_ld32(t_row + 128 + 32 * c, dr);
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int j0 = 128 * qc + 32 * c + 2 * i;   // query index of the column pair
-              const int jl = 32 * c + 2 * i;               // within this chunk
-              const bool v0 = jl < nq, v1 = jl + 1 < nq;
-              const float p0 = v0 ? ex2_approx(fmaf(__uint_as_float(sr[2 * i]), sl2, -lse_s[j0])) : 0.f;
-              const float p1 = v1 ? ex2_approx(fmaf(__uint_as_float(sr[2 * i + 1]), sl2, -lse_s[j0 + 1])) : 0.f;
-              const float s0 = v0 ? p0 * (__uint_as_float(dr[2 * i]) - d_s[j0]) : 0.f;
-              const float s1 = v1 ? p1 * (__uint_as_float(dr[2 * i + 1]) - d_s[j0 + 1]) : 0.f;
-              pp[i] = pack2_rn(p0, p1);
-              ps[i] = pack2_rn(s0, s1);
-            }
-            tmem_st16(t_row + 16 * c, pp);
-            tmem_st16(t_row + 128 + 16 * c, ps);
-          }
-          tc_fence_before();
-          mbar_arrive(&bars->p_full);
-        }
-        if (!ok) break;
-        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&bars->o_full, kt & 1, ctl))) break;
-        tc_fence_after();
-        {
-          const size_t ro = gi * 128;
-          write_row(t_row + 256, tok >= 0, 1.f, nullptr, a.dv_out + ro, nullptr);
-          if (a.final_out)
-            write_row(t_row + 384, tok >= 0, a.scale, a.accumulate ? a.dk_acc + ro : nullptr, a.dk_out + ro, nullptr);
-          else
-            write_row(t_row + 384, tok >= 0, a.scale, nullptr, nullptr, a.dk_acc + ro);
-        }
-        tc_fence_before();
-        mbar_arrive(&bars->o_free);
+      if (!ok) break;
+      ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->o_full, o_cnt & 1, ctl));
+      ++o_cnt;
+      if (!ok) break;
+      tc_fence_after();
+      {
+        const size_t ro = gi * 128;
+        write_row(t_row + 256, tok >= 0, 1.f, nullptr, a.dv_out + ro, nullptr);
+        if (a.final_out)
+          write_row(t_row + 384, tok >= 0, a.scale, a.accumulate ? a.dk_acc + ro : nullptr, a.dk_out + ro, nullptr);
+        else
+          write_row(t_row + 384, tok >= 0, a.scale, nullptr, nullptr, a.dk_acc + ro);
       }
+      tc_fence_before();
+      mbar_arrive(&bars->o_free);
     }
   }
   // tcgen05.dealloc is warp-wide and aligned: reconverge warp 4 (lane 0 arrives from the issue loop)
@@ -377,19 +371,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
 cudaError_t launch_bwd_tc(const BwdTcArgs& a, cudaStream_t stream) {
   static bool configured = false;
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(bwd_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kBwdSmemLimit);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(bwd_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kBwdSmemLimit);
+    cudaError_t e = cudaFuncSetAttribute(bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kBwdSmemLimit);
     if (e != cudaSuccess) return e;
     configured = true;
   }
   const unsigned grid = static_cast<unsigned>(a.g.B * a.g.h * a.p.n_seq);
   if (grid == 0) return cudaSuccess;
-  bwd_tc_kernel<false><<<grid, kBwdThreads, a.smem_bytes, stream>>>(a);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  bwd_tc_kernel<true><<<grid, kBwdThreads, a.smem_bytes, stream>>>(a);
+  bwd_tc_kernel<<<grid, kBwdThreads, a.smem_bytes, stream>>>(a);
   return cudaGetLastError();
 }
 
