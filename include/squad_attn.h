@@ -16,6 +16,13 @@
  * Between the passes there is only re-indexing (paper §4.3); this library never materialises a
  * permuted copy: both views are strided boxes of the caller's [B, h, n, d] tensors.
  *
+ * A window that does not divide H x W forces reflect padding (paper appendix, "Conformance to the
+ * theoretical curves is quantitative"): each frame is padded at the bottom and right up to multiples
+ * of hw and ww, reflecting about the edge (the edge token is not repeated); both passes run on the
+ * padded grid (padded copies of q, k, v live in the forward workspace) and o is cropped back. The
+ * backward is that composition's gradient: zero upstream gradient on the padded tokens, and each input
+ * token's gradient summed over its padded copies. squad_window_solve picks a window.
+ *
  * Conventions shared by every entry point
  * ---------------------------------------
  * Layout:     every tensor is contiguous [B, h, n, d] (d fastest), n = T*H*W tokens ordered
@@ -77,14 +84,16 @@ typedef enum {
 typedef struct {
   int B, h, d;      /* batch, heads, head dim (d in {64, 128}; bf16 tensor-core path: d == 128)  */
   int T, H, W;      /* latent grid; n = T*H*W                                                     */
-  int tw, hw, ww;   /* window; tw must equal T (the window spans all frames), H % hw == W % ww == 0 */
+  int tw, hw, ww;   /* window; tw must equal T (the window spans all frames), 1 <= hw <= H, 1 <= ww <= W;
+                       a window that does not divide H x W is handled by reflect padding            */
   int order;        /* squad_order_t                                                              */
   int dtype;        /* squad_dtype_t                                                              */
   float scale;      /* softmax scale; 0 selects 1/sqrt(d) (paper eq. 5)                           */
 } squad_params_t;
 
 /* Bytes of forward workspace: the pass-1 output O1 ([B,h,n,d] in the tensor dtype), both passes'
- * LSE ([B,h,n] fp32 each) and a small control block. Keep the workspace unchanged between
+ * LSE ([B,h,n] fp32 each) and a small control block; for a padded grid these are sized for the
+ * padded n, plus the padded q, k, v and output. Keep the workspace unchanged between
  * squad_attn_fwd and squad_attn_bwd: the backward reads O1 and the LSEs from it. Returns 0 for
  * invalid parameters. */
 SQUAD_API size_t squad_attn_fwd_workspace_bytes(const squad_params_t* p);
@@ -100,8 +109,9 @@ SQUAD_API squad_status_t squad_attn_fwd(const squad_params_t* p, const void* q, 
 SQUAD_API squad_status_t squad_attn_fwd_status(const squad_params_t* p, const void* workspace,
                                      squad_stream_t stream);
 
-/* Bytes of backward workspace: fp32 partial dQ and dK, the fp32 gradient of the pass-1 output, the
- * per-row softmax-Jacobian terms of each pass, and a control block. Returns 0 for invalid params. */
+/* Bytes of backward workspace: fp32 partial dQ and dK, the gradient of the pass-1 output, the per-row
+ * softmax-Jacobian terms of each pass, and a control block (for a padded grid: sized for the padded n,
+ * plus the zero-padded dout and the gradients on the padded grid). Returns 0 for invalid params. */
 SQUAD_API size_t squad_attn_bwd_workspace_bytes(const squad_params_t* p);
 
 /* SQuad-Attention backward (the pages print no formula; it is the chain rule through both passes).
@@ -143,9 +153,19 @@ SQUAD_API squad_status_t squad_attn_fwd_noalloc(const squad_params_t* p, const v
                                                 const void* v, void* o, squad_stream_t stream);
 
 /* FLOPs of one call, from the paper's cost model (appendix "Conformance to the theoretical curves
- * is quantitative"): 4 B h d (n w + n^2/w) for SQuad, 4 B h d n^2 for full attention. */
+ * is quantitative"): 4 B h d (n w + n^2/w) for SQuad (one of the two terms for a single-pass order;
+ * n = the padded token count when the window does not divide the grid, the cost of the window
+ * actually used), 4 B h d n^2 for full attention. */
 SQUAD_API double squad_attn_flops(const squad_params_t* p);
 SQUAD_API double full_attn_flops(const squad_params_t* p);
+
+/* The window for a T x H x W grid, re-solved per resolution as the paper's appendix ("Conformance to
+ * the theoretical curves is quantitative") describes: tw = T; for each hw the ww whose ratio hw:ww is
+ * closest to H:W (in log ratio, the smaller ww on a tie); and, among those, the hw whose cost
+ * n'm + n'^2/m is least, m = T*hw*ww the window size and n' the reflect-padded token count (ties: the
+ * smaller hw). Recovers 21x2x4 at 21x22x40 and at 21x30x52. Writes *tw, *hw, *ww; SQUAD_ERR_INVALID_ARG
+ * for non-positive extents or null outputs. Host-only; launches nothing. */
+SQUAD_API squad_status_t squad_window_solve(int T, int H, int W, int* tw, int* hw, int* ww);
 
 /* Static string for a status code (never NULL). */
 SQUAD_API const char* squad_status_string(squad_status_t s);

@@ -12,6 +12,7 @@ from .api import (  # noqa: F401
     squad_attn_bwd,
     squad_attn_bwd_workspace_bytes,
     squad_attn_flops,
+    squad_window_solve,
     squad_attn_fwd,
     squad_attn_fwd_noalloc,
     squad_attn_fwd_status,

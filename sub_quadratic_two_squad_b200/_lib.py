@@ -33,6 +33,8 @@ SIGNATURES = {
     "full_attn_fwd": (ctypes.c_int, [_PP, _VP, _VP, _VP, _VP, _VP, _VP]),
     "squad_attn_fwd_noalloc": (ctypes.c_int, [_PP, _VP, _VP, _VP, _VP, _VP]),
     "squad_attn_flops": (ctypes.c_double, [_PP]),
+    "squad_window_solve": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_int),
+                                          ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]),
     "full_attn_flops": (ctypes.c_double, [_PP]),
     "squad_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "squad_attn_abi_version": (ctypes.c_int, []),

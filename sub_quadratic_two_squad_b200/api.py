@@ -140,6 +140,16 @@ def squad_attn_flops(B, h, d, grid, window, order="local_then_global") -> float:
     return float(_lib.load().squad_attn_flops(ctypes.byref(make_params(B, h, d, grid, window, order))))
 
 
+def squad_window_solve(grid):
+    """The window (tw, hw, ww) for a (T, H, W) grid (w_t = T, aspect-following, least padded cost)."""
+    tw, hw, ww = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+    st = _lib.load().squad_window_solve(int(grid[0]), int(grid[1]), int(grid[2]), ctypes.byref(tw), ctypes.byref(hw),
+                                        ctypes.byref(ww))
+    if st != _lib.SQUAD_OK:
+        raise SquadError(st, "squad_window_solve")
+    return tw.value, hw.value, ww.value
+
+
 def full_attn_flops(B, h, d, grid) -> float:
     return float(_lib.load().full_attn_flops(ctypes.byref(make_params(B, h, d, grid))))
 

@@ -1,5 +1,6 @@
 // C ABI of the SQuad-Attention library (include/squad_attn.h): argument validation, TMA tensor maps
 // for the window and slot views, and the launch sequence of the two passes.
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstdlib>
@@ -13,6 +14,7 @@
 #include "squad_attn.h"
 #include "geometry.cuh"
 #include "bwd_pass.h"
+#include "pad.h"
 #include "short_pass.h"
 #include "simt_pass.h"
 #include "tc_pass.h"
@@ -34,16 +36,30 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 bool aligned(const void* p, size_t a) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// The caller's grid when the window does not divide it: the kernels run on the padded grid.
+struct PadDims {
+  int H0 = 0, W0 = 0;   // original extents
+  bool padded = false;
+};
+
 // Validates the parameters and fills the grid description. `windowed` = SQuad call (window fields
-// and order are used); false = full attention (only B, h, d, T, H, W, dtype, scale).
-squad_status_t validate(const squad_params_t* p, bool windowed, Grid* g, float* scale) {
+// and order are used); false = full attention (only B, h, d, T, H, W, dtype, scale). For a window
+// that does not divide H x W, *g is the grid reflect-padded at the bottom and right up to multiples
+// of the window (SQuad paper appendix, "Conformance to the theoretical curves is quantitative"), and
+// *pd keeps the original extents.
+squad_status_t validate(const squad_params_t* p, bool windowed, Grid* g, float* scale, PadDims* pd = nullptr) {
   if (p == nullptr) return SQUAD_ERR_INVALID_ARG;
   if (p->B < 1 || p->h < 1 || p->T < 1 || p->H < 1 || p->W < 1) return SQUAD_ERR_INVALID_ARG;
   if (p->dtype != SQUAD_BF16 && p->dtype != SQUAD_FP32) return SQUAD_ERR_INVALID_ARG;
   if (p->d < 1) return SQUAD_ERR_INVALID_ARG;
   if (p->d != 64 && p->d != 128) return SQUAD_ERR_UNSUPPORTED;
   if (!(p->scale >= 0.f) || !std::isfinite(p->scale)) return SQUAD_ERR_INVALID_ARG;
-  const long long n = static_cast<long long>(p->T) * p->H * p->W;
+  int H = p->H, W = p->W;
+  if (windowed && p->hw >= 1 && p->ww >= 1) {   // padded extents (reflect padding is shorter than the extent
+    H = (p->H + p->hw - 1) / p->hw * p->hw;     // whenever hw <= H and ww <= W, checked below)
+    W = (p->W + p->ww - 1) / p->ww * p->ww;
+  }
+  const long long n = static_cast<long long>(p->T) * H * W;
   if (n > (1ll << 30)) return SQUAD_ERR_UNSUPPORTED;
   const long long bhn = static_cast<long long>(p->B) * p->h * n;
   if (bhn > (1ll << 31) - 1) return SQUAD_ERR_UNSUPPORTED;
@@ -52,21 +68,20 @@ squad_status_t validate(const squad_params_t* p, bool windowed, Grid* g, float* 
   gg.h = p->h;
   gg.d = p->d;
   gg.T = p->T;
-  gg.H = p->H;
-  gg.W = p->W;
+  gg.H = H;
+  gg.W = W;
   gg.n = static_cast<int>(n);
   if (windowed) {
     if (p->order < SQUAD_LOCAL_THEN_GLOBAL || p->order > SQUAD_GLOBAL_ONLY) return SQUAD_ERR_INVALID_ARG;
     if (p->tw < 1 || p->hw < 1 || p->ww < 1) return SQUAD_ERR_INVALID_ARG;
     if (p->tw > p->T || p->hw > p->H || p->ww > p->W) return SQUAD_ERR_INVALID_ARG;
-    // The window spans the full temporal extent and tiles space exactly; other windows (tw < T,
-    // grids that need reflect padding) are outside what this library implements.
+    // The window spans the full temporal extent (tw < T is outside the method); space is tiled by the
+    // window over the (padded) grid.
     if (p->tw != p->T) return SQUAD_ERR_UNSUPPORTED;
-    if (p->H % p->hw != 0 || p->W % p->ww != 0) return SQUAD_ERR_UNSUPPORTED;
     gg.hw = p->hw;
     gg.ww = p->ww;
-    gg.nwy = p->H / p->hw;
-    gg.nwx = p->W / p->ww;
+    gg.nwy = H / p->hw;
+    gg.nwx = W / p->ww;
   } else {
     gg.hw = 1;
     gg.ww = 1;
@@ -75,6 +90,11 @@ squad_status_t validate(const squad_params_t* p, bool windowed, Grid* g, float* 
   }
   finish_grid(gg);
   *g = gg;
+  if (pd != nullptr) {
+    pd->H0 = p->H;
+    pd->W0 = p->W;
+    pd->padded = H != p->H || W != p->W;
+  }
   *scale = p->scale > 0.f ? p->scale : 1.0f / std::sqrt(static_cast<float>(p->d));
   return SQUAD_OK;
 }
@@ -90,24 +110,35 @@ struct FwdWorkspace {
   void* o1;
   float* lse1;
   float* lse2;
+  void *qp, *kp, *vp, *op;   // padded grids only: the padded q, k, v (kept for the backward) and output
 };
 
-size_t fwd_ws_bytes(const Grid& g, size_t eb) {
+size_t fwd_ws_bytes(const Grid& g, size_t eb, bool padded) {
   const size_t bhn = static_cast<size_t>(g.B) * g.h * g.n;
-  return ctrl_bytes(g) + align256(bhn * g.d * eb) + 2 * align256(bhn * 4);
+  const size_t t = align256(bhn * g.d * eb);
+  return ctrl_bytes(g) + t + 2 * align256(bhn * 4) + (padded ? 4 * t : 0);
 }
 
-FwdWorkspace carve_fwd(void* ws, const Grid& g, size_t eb) {
+FwdWorkspace carve_fwd(void* ws, const Grid& g, size_t eb, bool padded) {
   uint8_t* b = static_cast<uint8_t*>(ws);
   const size_t bhn = static_cast<size_t>(g.B) * g.h * g.n;
+  const size_t t = align256(bhn * g.d * eb);
   FwdWorkspace w;
   w.status = reinterpret_cast<uint32_t*>(b);
   b += ctrl_bytes(g);
   w.o1 = b;
-  b += align256(bhn * g.d * eb);
+  b += t;
   w.lse1 = reinterpret_cast<float*>(b);
   b += align256(bhn * 4);
   w.lse2 = reinterpret_cast<float*>(b);
+  b += align256(bhn * 4);
+  w.qp = w.kp = w.vp = w.op = nullptr;
+  if (padded) {
+    w.qp = b;
+    w.kp = b + t;
+    w.vp = b + 2 * t;
+    w.op = b + 3 * t;
+  }
   return w;
 }
 
@@ -117,14 +148,15 @@ struct BwdWorkspace {
   float* dk_acc;
   float* do1;
   float* drow;
+  void *dop, *dqp, *dkp, *dvp;   // padded grids only: dout zero-padded, gradients on the padded grid
 };
 
-size_t bwd_ws_bytes(const Grid& g) {
+size_t bwd_ws_bytes(const Grid& g, size_t eb, bool padded) {
   const size_t bhn = static_cast<size_t>(g.B) * g.h * g.n;
-  return ctrl_bytes(g) + 3 * align256(bhn * g.d * 4) + align256(bhn * 4);
+  return ctrl_bytes(g) + 3 * align256(bhn * g.d * 4) + align256(bhn * 4) + (padded ? 4 * align256(bhn * g.d * eb) : 0);
 }
 
-BwdWorkspace carve_bwd(void* ws, const Grid& g) {
+BwdWorkspace carve_bwd(void* ws, const Grid& g, size_t eb, bool padded) {
   uint8_t* b = static_cast<uint8_t*>(ws);
   const size_t bhn = static_cast<size_t>(g.B) * g.h * g.n;
   BwdWorkspace w;
@@ -137,7 +169,29 @@ BwdWorkspace carve_bwd(void* ws, const Grid& g) {
   w.do1 = reinterpret_cast<float*>(b);
   b += align256(bhn * g.d * 4);
   w.drow = reinterpret_cast<float*>(b);
+  b += align256(bhn * 4);
+  w.dop = w.dqp = w.dkp = w.dvp = nullptr;
+  if (padded) {
+    const size_t t = align256(bhn * g.d * eb);
+    w.dop = b;
+    w.dqp = b + t;
+    w.dkp = b + 2 * t;
+    w.dvp = b + 3 * t;
+  }
   return w;
+}
+
+PadShape pad_shape(const Grid& g, const PadDims& pd, size_t eb) {
+  PadShape s;
+  s.BH = g.B * g.h;
+  s.T = g.T;
+  s.H = pd.H0;
+  s.W = pd.W0;
+  s.Hp = g.H;
+  s.Wp = g.W;
+  s.d = g.d;
+  s.vec = static_cast<int>(g.d * eb / 16);
+  return s;
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -302,6 +356,33 @@ double squad_attn_flops(const squad_params_t* p) {
   return 4.0 * p->B * p->h * p->d * terms;
 }
 
+squad_status_t squad_window_solve(int T, int H, int W, int* tw, int* hw, int* ww) {
+  if (T < 1 || H < 1 || W < 1 || tw == nullptr || hw == nullptr || ww == nullptr) return SQUAD_ERR_INVALID_ARG;
+  double best = 0.0;
+  int best_h = 0, best_w = 0;
+  for (int h = 1; h <= H; ++h) {
+    // the width whose ratio h:w is closest to H:W (log ratio), of the two around h*W/H
+    const int lo = std::max(1, static_cast<int>(std::floor(static_cast<double>(h) * W / H)));
+    const double target = std::log(static_cast<double>(H) / W);
+    const double e_lo = std::fabs(std::log(static_cast<double>(h) / lo) - target);
+    const double e_hi = std::fabs(std::log(static_cast<double>(h) / (lo + 1)) - target);
+    const int w = e_hi < e_lo ? lo + 1 : lo;
+    if (w > W) continue;
+    const double hp = static_cast<double>((H + h - 1) / h * h), wp = static_cast<double>((W + w - 1) / w * w);
+    const double np = static_cast<double>(T) * hp * wp, m = static_cast<double>(T) * h * w;
+    const double cost = np * m + np * np / m;
+    if (best_h == 0 || cost < best) {
+      best = cost;
+      best_h = h;
+      best_w = w;
+    }
+  }
+  *tw = T;
+  *hw = best_h;
+  *ww = best_w;
+  return SQUAD_OK;
+}
+
 double full_attn_flops(const squad_params_t* p) {
   Grid g;
   float sc;
@@ -313,29 +394,27 @@ double full_attn_flops(const squad_params_t* p) {
 size_t squad_attn_fwd_workspace_bytes(const squad_params_t* p) {
   Grid g;
   float sc;
-  if (validate(p, true, &g, &sc) != SQUAD_OK) return 0;
-  return fwd_ws_bytes(g, elem_bytes(p));
+  PadDims pd;
+  if (validate(p, true, &g, &sc, &pd) != SQUAD_OK) return 0;
+  return fwd_ws_bytes(g, elem_bytes(p), pd.padded);
 }
 
 size_t squad_attn_bwd_workspace_bytes(const squad_params_t* p) {
   Grid g;
   float sc;
-  if (validate(p, true, &g, &sc) != SQUAD_OK) return 0;
-  return bwd_ws_bytes(g);
+  PadDims pd;
+  if (validate(p, true, &g, &sc, &pd) != SQUAD_OK) return 0;
+  return bwd_ws_bytes(g, elem_bytes(p), pd.padded);
 }
 
-squad_status_t squad_attn_fwd(const squad_params_t* p, const void* q, const void* k, const void* v, void* o,
-                              void* workspace, squad_stream_t stream_) {
-  Grid g;
-  float scale;
-  squad_status_t st = validate(p, true, &g, &scale);
-  if (st != SQUAD_OK) return st;
-  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(workspace, 256))
-    return SQUAD_ERR_INVALID_ARG;
-  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-  const size_t eb = elem_bytes(p);
-  FwdWorkspace ws = carve_fwd(workspace, g, eb);
-  if (cudaMemsetAsync(ws.status, 0, ctrl_bytes(g), stream) != cudaSuccess) return SQUAD_ERR_CUDA;
+}  // extern "C"
+
+namespace {
+
+// The forward on the kernels' grid g (already padded where needed); the control block is zeroed.
+squad_status_t fwd_core(const squad_params_t* p, const Grid& g, float scale, const void* q, const void* k,
+                        const void* v, void* o, const FwdWorkspace& ws, cudaStream_t stream) {
+  squad_status_t st;
   const bool bf16 = p->dtype == SQUAD_BF16;
   uint32_t* ctrl = ws.status;
   if (p->order == SQUAD_LOCAL_ONLY || p->order == SQUAD_GLOBAL_ONLY) {
@@ -362,6 +441,35 @@ squad_status_t squad_attn_fwd(const squad_params_t* p, const void* q, const void
   return run_pass(p, g, second, scale, q, k, ws.o1, bf16, o, ws.lse2, ctrl, ctrl + 3, stream);
 }
 
+}  // namespace
+
+extern "C" {
+
+squad_status_t squad_attn_fwd(const squad_params_t* p, const void* q, const void* k, const void* v, void* o,
+                              void* workspace, squad_stream_t stream_) {
+  Grid g;
+  float scale;
+  PadDims pd;
+  squad_status_t st = validate(p, true, &g, &scale, &pd);
+  if (st != SQUAD_OK) return st;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(workspace, 256))
+    return SQUAD_ERR_INVALID_ARG;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  const size_t eb = elem_bytes(p);
+  FwdWorkspace ws = carve_fwd(workspace, g, eb, pd.padded);
+  if (cudaMemsetAsync(ws.status, 0, ctrl_bytes(g), stream) != cudaSuccess) return SQUAD_ERR_CUDA;
+  if (!pd.padded) return fwd_core(p, g, scale, q, k, v, o, ws, stream);
+  // Reflect-pad q, k, v into the workspace, run on the padded grid, crop the output into o.
+  const PadShape ps = pad_shape(g, pd, eb);
+  if (launch_reflect_pad(q, ws.qp, ps, false, stream) != cudaSuccess ||
+      launch_reflect_pad(k, ws.kp, ps, false, stream) != cudaSuccess ||
+      launch_reflect_pad(v, ws.vp, ps, false, stream) != cudaSuccess)
+    return SQUAD_ERR_CUDA;
+  st = fwd_core(p, g, scale, ws.qp, ws.kp, ws.vp, ws.op, ws, stream);
+  if (st != SQUAD_OK) return st;
+  return launch_crop(ws.op, o, ps, stream) == cudaSuccess ? SQUAD_OK : SQUAD_ERR_CUDA;
+}
+
 squad_status_t squad_attn_fwd_status(const squad_params_t* p, const void* workspace, squad_stream_t stream_) {
   Grid g;
   float scale;
@@ -376,23 +484,16 @@ squad_status_t squad_attn_fwd_status(const squad_params_t* p, const void* worksp
   return word == 0 ? SQUAD_OK : SQUAD_ERR_TIMEOUT;
 }
 
-squad_status_t squad_attn_bwd(const squad_params_t* p, const void* q, const void* k, const void* v, const void* o,
-                              const void* dout, const void* fwd_workspace, void* dq, void* dk, void* dv,
-                              void* bwd_workspace, squad_stream_t stream_) {
-  Grid g;
-  float scale;
-  squad_status_t st = validate(p, true, &g, &scale);
-  if (st != SQUAD_OK) return st;
-  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(dout, 16) ||
-      !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(fwd_workspace, 256) ||
-      !aligned(bwd_workspace, 256))
-    return SQUAD_ERR_INVALID_ARG;
-  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-  const size_t eb = elem_bytes(p);
+}  // extern "C"
+
+namespace {
+
+// The backward on the kernels' grid g (already padded where needed); the control block is zeroed.
+squad_status_t bwd_core(const squad_params_t* p, const Grid& g, float scale, const void* q, const void* k,
+                        const void* v, const void* o, const void* dout, const FwdWorkspace& fw,
+                        const BwdWorkspace& bw, void* dq, void* dk, void* dv, cudaStream_t stream) {
+  (void)o;   // D_i is formed from the recomputed P and dP, not from o
   const bool bf16 = p->dtype == SQUAD_BF16;
-  FwdWorkspace fw = carve_fwd(const_cast<void*>(fwd_workspace), g, eb);
-  BwdWorkspace bw = carve_bwd(bwd_workspace, g);
-  if (cudaMemsetAsync(bw.status, 0, ctrl_bytes(g), stream) != cudaSuccess) return SQUAD_ERR_CUDA;
   if (p->order == SQUAD_LOCAL_ONLY || p->order == SQUAD_GLOBAL_ONLY) {
     // One pass: values v, upstream dout, the pass's LSE in the first slot; no share to add.
     const int kind = p->order == SQUAD_LOCAL_ONLY ? kLocal : kGlobal;
@@ -527,6 +628,41 @@ squad_status_t squad_attn_bwd(const squad_params_t* p, const void* q, const void
   a.accumulate = 1;
   a.final_out = 1;
   if (launch_simt_bwd(a, stream) != cudaSuccess) return SQUAD_ERR_CUDA;
+  return SQUAD_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+squad_status_t squad_attn_bwd(const squad_params_t* p, const void* q, const void* k, const void* v, const void* o,
+                              const void* dout, const void* fwd_workspace, void* dq, void* dk, void* dv,
+                              void* bwd_workspace, squad_stream_t stream_) {
+  Grid g;
+  float scale;
+  PadDims pd;
+  squad_status_t st = validate(p, true, &g, &scale, &pd);
+  if (st != SQUAD_OK) return st;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(dout, 16) ||
+      !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(fwd_workspace, 256) ||
+      !aligned(bwd_workspace, 256))
+    return SQUAD_ERR_INVALID_ARG;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  const size_t eb = elem_bytes(p);
+  FwdWorkspace fw = carve_fwd(const_cast<void*>(fwd_workspace), g, eb, pd.padded);
+  BwdWorkspace bw = carve_bwd(bwd_workspace, g, eb, pd.padded);
+  if (cudaMemsetAsync(bw.status, 0, ctrl_bytes(g), stream) != cudaSuccess) return SQUAD_ERR_CUDA;
+  if (!pd.padded) return bwd_core(p, g, scale, q, k, v, o, dout, fw, bw, dq, dk, dv, stream);
+  // The padded method: dout is zero on the padded tokens (the adjoint of the crop); the padded q, k, v
+  // and output are the forward workspace's; each input token's gradient sums over its padded copies.
+  const PadShape ps = pad_shape(g, pd, eb);
+  if (launch_reflect_pad(dout, bw.dop, ps, true, stream) != cudaSuccess) return SQUAD_ERR_CUDA;
+  st = bwd_core(p, g, scale, fw.qp, fw.kp, fw.vp, fw.op, bw.dop, fw, bw, bw.dqp, bw.dkp, bw.dvp, stream);
+  if (st != SQUAD_OK) return st;
+  const bool bf16 = p->dtype == SQUAD_BF16;
+  if (launch_fold(bw.dqp, dq, ps, bf16, stream) != cudaSuccess || launch_fold(bw.dkp, dk, ps, bf16, stream) != cudaSuccess ||
+      launch_fold(bw.dvp, dv, ps, bf16, stream) != cudaSuccess)
+    return SQUAD_ERR_CUDA;
   return SQUAD_OK;
 }
 

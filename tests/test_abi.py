@@ -60,8 +60,6 @@ def _fwd(lib, prm, ptr=16):
 
 @pytest.mark.parametrize("kw,status", [
     (dict(window=(20, 2, 4)), _lib.SQUAD_ERR_UNSUPPORTED),      # window must span all frames
-    (dict(window=(21, 3, 4)), _lib.SQUAD_ERR_UNSUPPORTED),      # H % hw != 0 (would need reflect padding)
-    (dict(window=(21, 2, 3)), _lib.SQUAD_ERR_UNSUPPORTED),      # W % ww != 0
     (dict(window=(21, 0, 4)), _lib.SQUAD_ERR_INVALID_ARG),
     (dict(window=(22, 2, 4)), _lib.SQUAD_ERR_INVALID_ARG),      # larger than the grid
     (dict(d=96), _lib.SQUAD_ERR_UNSUPPORTED),
@@ -116,6 +114,34 @@ def test_single_pass_orders_accepted_and_counted(lib, cfg):
         fl[order] = lib.squad_attn_flops(ctypes.byref(prm))
     assert fl["local_only"] == pytest.approx(4.0 * B * h * d * n * w, rel=1e-12)
     assert fl["local_only"] + fl["global_only"] == pytest.approx(orc.squad_flops(B, h, d, n, w), rel=1e-12)
+
+
+@pytest.mark.parametrize("grid", [(21, 22, 40), (21, 30, 52), (21, 44, 80), (21, 60, 104), (13, 17, 29), (5, 8, 8),
+                                  (1, 1, 1), (3, 1, 50), (7, 31, 2)])
+def test_window_solver_matches_the_oracle(lib, grid):
+    tw, hw, ww = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+    assert lib.squad_window_solve(*grid, ctypes.byref(tw), ctypes.byref(hw), ctypes.byref(ww)) == _lib.SQUAD_OK
+    assert (tw.value, hw.value, ww.value) == orc.window_solve(*grid)
+
+
+def test_window_solver_rejects_bad_arguments(lib):
+    x = ctypes.c_int()
+    assert lib.squad_window_solve(0, 4, 4, ctypes.byref(x), ctypes.byref(x), ctypes.byref(x)) == _lib.SQUAD_ERR_INVALID_ARG
+    assert lib.squad_window_solve(4, 4, 4, None, ctypes.byref(x), ctypes.byref(x)) == _lib.SQUAD_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("window", [(21, 3, 4), (21, 2, 3), (21, 5, 7), (21, 22, 39)])
+def test_non_dividing_windows_run_on_the_padded_grid(lib, window):
+    """Accepted (reflect padding): the workspaces grow by the padded tensors and the FLOP count is the
+    cost of the padded grid."""
+    grid = (21, 22, 40)
+    prm = make_params(1, 24, 128, grid, window)
+    hp, wp = -(-22 // window[1]) * window[1], -(-40 // window[2]) * window[2]
+    n_p, w = 21 * hp * wp, window[0] * window[1] * window[2]
+    fwd = lib.squad_attn_fwd_workspace_bytes(ctypes.byref(prm))
+    assert fwd >= 5 * 24 * n_p * 128 * 2 + 2 * 24 * n_p * 4   # O1 + padded q, k, v, o + LSEs
+    assert lib.squad_attn_bwd_workspace_bytes(ctypes.byref(prm)) >= 3 * 24 * n_p * 128 * 4 + 4 * 24 * n_p * 128 * 2
+    assert lib.squad_attn_flops(ctypes.byref(prm)) == pytest.approx(orc.squad_flops(1, 24, 128, n_p, w), rel=1e-12)
 
 
 def test_workspace_sizes(lib):

@@ -209,3 +209,26 @@ def test_single_pass_wan22_5b_shape(order):
     """Windows of 168 and slot sequences of 110 tokens, one pass, forward and backward (2 heads)."""
     run_fwd(1, 24, 128, (21, 22, 40), (21, 2, 4), order, torch.bfloat16, heavy_tail=True, heads=[0, 23])
     run_bwd(1, 2, 128, (21, 22, 40), (21, 2, 4), order, torch.bfloat16)
+
+
+# ------------------------------------------------------------------------------------------------
+# grids the window does not divide (reflect padding, both passes on the padded grid, crop)
+# ------------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("order", [LG, GL, LO, GO])
+def test_padded_tiny_fp32(order):
+    """5x7x9 with a 5x2x4 window: padded to 5x8x12 (one row, three columns reflected)."""
+    run_fwd(1, 2, 64, (5, 7, 9), (5, 2, 4), order, torch.float32)
+    run_bwd(1, 2, 64, (5, 7, 9), (5, 2, 4), order, torch.float32)
+
+
+@pytest.mark.parametrize("order", [LG, GL])
+def test_padded_small_bf16(order):
+    run_fwd(1, 2, 128, (21, 5, 9), (21, 2, 4), order, torch.bfloat16)
+    run_bwd(1, 2, 128, (21, 5, 9), (21, 2, 4), order, torch.bfloat16)
+
+
+def test_padded_odd_resolution_bf16():
+    """The 5B block with one more latent row and column (21x23x41, padded to 21x24x44)."""
+    run_fwd(1, 24, 128, (21, 23, 41), (21, 2, 4), LG, torch.bfloat16, heavy_tail=True, heads=[0, 23])
+    run_bwd(1, 2, 128, (21, 23, 41), (21, 2, 4), LG, torch.bfloat16)
