@@ -77,6 +77,7 @@ __device__ __forceinline__ int pos_v(int b, int nb) { return b == nb - 1 ? 2 * n
 
 }  // namespace
 
+template <bool kSplitRows>
 __global__ void __launch_bounds__(kThreads, 1) tc_pass_kernel(const __grid_constant__ TcPassArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -311,68 +312,139 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pass_kernel(const __grid_const
         ++s_cnt;
         if (!ok) break;
         tc_fence_after();   // S(b) is ready, and so is every earlier PV (in-order tensor pipe)
-        const int valid = chunk_valid_rows(p, b);
-        uint32_t r[128];
-        float m_new = m_used;
-        if (active) {
-          tmem_ld128(t_s, r);
-          if (valid < 128)
-#pragma unroll
-            for (int i = 0; i < 128; ++i)
-              if (i >= valid) r[i] = __float_as_uint(-INFINITY);
-          // row maximum (4 independent partial maxima; the scale is positive, so it is applied to the
-          // maximum instead of to every score)
-          float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-          for (int i = 0; i < 128; ++i) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(r[i]));
-          m_new = fmaxf(m_used, fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2);
-        }
-        if (b > 0) {
-          // Rescale O only when the running maximum grew by more than 2^8 (until then the unscaled
-          // exponentials stay below 256). PV(b-1) has completed: S(b) was issued after it. This path is
-          // rare, so it reuses the score registers for O and reloads S afterwards.
-          const bool need = active && m_new > m_used + 8.f;
-          if (__any_sync(0xffffffffu, need)) {
-            const float f = need ? ex2_approx(m_used - m_new) : 1.f;
-            tmem_ld128(t_o, r);
-#pragma unroll
-            for (int i = 0; i < 128; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * f);
-            tmem_st128(t_o, r);
-            if (need) {
-              l *= f;
-              m_used = m_new;
+        if constexpr (kSplitRows) {
+          // Short sequences: the block's scores are read in 64-column halves (twice), so the softmax
+          // stays within the register budget.
+          const int valid = chunk_valid_rows(p, b);
+          float m_new = m_used;
+          if (active) {
+            // row maximum over the block, 64 columns at a time (4 independent partial maxima; the scale
+            // is positive, so it is applied to the maximum instead of to every score)
+            float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+  #pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              uint32_t r[64];
+              tmem_ld64(t_s + 64 * c, r);
+  #pragma unroll
+              for (int i = 0; i < 64; ++i)
+                if (64 * c + i < valid) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(r[i]));
             }
-            if (active) {
-              tmem_ld128(t_s, r);
-              if (valid < 128)
-#pragma unroll
-                for (int i = 0; i < 128; ++i)
-                  if (i >= valid) r[i] = __float_as_uint(-INFINITY);
+            m_new = fmaxf(m_used, fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2);
+          }
+          if (b > 0) {
+            // Rescale O only when the running maximum grew by more than 2^8 (until then the unscaled
+            // exponentials stay below 256). PV(b-1) has completed: S(b) was issued after it.
+            const bool need = active && m_new > m_used + 8.f;
+            if (__any_sync(0xffffffffu, need)) {
+              const float f = need ? ex2_approx(m_used - m_new) : 1.f;
+  #pragma unroll
+              for (int c = 0; c < 2; ++c) {
+                uint32_t o[64];
+                tmem_ld64(t_o + 64 * c, o);
+  #pragma unroll
+                for (int i = 0; i < 64; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
+                tmem_st64v(t_o + 64 * c, o);
+              }
+              if (need) {
+                l *= f;
+                m_used = m_new;
+              }
             }
+          } else {
+            m_used = m_new;
+          }
+          if (active) {
+            // P = 2^(x - m) (masked columns give 0), rounded to bf16 on the integer pipe (add half an ulp,
+            // keep the high half), packed two per 32-bit word over the first 64 TMEM columns of S: the
+            // packed half of a 64-column chunk lands on columns already read.
+            const float nm = -m_used;
+            float ls[4] = {0.f, 0.f, 0.f, 0.f};
+  #pragma unroll 1
+            for (int c = 0; c < 2; ++c) {
+              uint32_t r[64];
+              tmem_ld64(t_s + 64 * c, r);
+  #pragma unroll
+              for (int k = 0; k < 2; ++k) {
+                uint32_t pk[16];
+  #pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                  const int i0 = 32 * k + 2 * j;
+                  const float x0 = 64 * c + i0 < valid ? ex2_approx(fmaf(__uint_as_float(r[i0]), sl2, nm)) : 0.f;
+                  const float x1 = 64 * c + i0 + 1 < valid ? ex2_approx(fmaf(__uint_as_float(r[i0 + 1]), sl2, nm)) : 0.f;
+                  ls[(2 * j) & 3] += x0;
+                  ls[(2 * j + 1) & 3] += x1;
+                  pk[j] = __byte_perm(__float_as_uint(x0) + 0x8000u, __float_as_uint(x1) + 0x8000u, 0x7632);
+                }
+                tmem_st16(t_s + 32 * c + 16 * k, pk);
+              }
+            }
+            l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
           }
         } else {
-          m_used = m_new;
-        }
-        if (active) {
-          // P = 2^(x - m) (masked columns give 2^-inf = 0), rounded to bf16 on the integer pipe (add half
-          // an ulp, keep the high half), packed two per 32-bit word and stored 32 scores at a time over
-          // the first 64 TMEM columns of S (the scores are already in registers).
-          const float nm = -m_used;
-          float ls[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            uint32_t pk[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const float x0 = ex2_approx(fmaf(__uint_as_float(r[32 * k + 2 * j]), sl2, nm));
-              const float x1 = ex2_approx(fmaf(__uint_as_float(r[32 * k + 2 * j + 1]), sl2, nm));
-              ls[(2 * j) & 3] += x0;
-              ls[(2 * j + 1) & 3] += x1;
-              pk[j] = __byte_perm(__float_as_uint(x0) + 0x8000u, __float_as_uint(x1) + 0x8000u, 0x7632);
-            }
-            tmem_st16(t_s + 16 * k, pk);
+          // Long sequences (full attention): the 128 scores are read once into registers.
+          const int valid = chunk_valid_rows(p, b);
+          uint32_t r[128];
+          float m_new = m_used;
+          if (active) {
+            tmem_ld128(t_s, r);
+            if (valid < 128)
+  #pragma unroll
+              for (int i = 0; i < 128; ++i)
+                if (i >= valid) r[i] = __float_as_uint(-INFINITY);
+            // row maximum (4 independent partial maxima; the scale is positive, so it is applied to the
+            // maximum instead of to every score)
+            float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+  #pragma unroll
+            for (int i = 0; i < 128; ++i) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(r[i]));
+            m_new = fmaxf(m_used, fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2);
           }
-          l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+          if (b > 0) {
+            // Rescale O only when the running maximum grew by more than 2^8 (until then the unscaled
+            // exponentials stay below 256). PV(b-1) has completed: S(b) was issued after it. This path is
+            // rare, so it reuses the score registers for O and reloads S afterwards.
+            const bool need = active && m_new > m_used + 8.f;
+            if (__any_sync(0xffffffffu, need)) {
+              const float f = need ? ex2_approx(m_used - m_new) : 1.f;
+              tmem_ld128(t_o, r);
+  #pragma unroll
+              for (int i = 0; i < 128; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * f);
+              tmem_st128(t_o, r);
+              if (need) {
+                l *= f;
+                m_used = m_new;
+              }
+              if (active) {
+                tmem_ld128(t_s, r);
+                if (valid < 128)
+  #pragma unroll
+                  for (int i = 0; i < 128; ++i)
+                    if (i >= valid) r[i] = __float_as_uint(-INFINITY);
+              }
+            }
+          } else {
+            m_used = m_new;
+          }
+          if (active) {
+            // P = 2^(x - m) (masked columns give 2^-inf = 0), rounded to bf16 on the integer pipe (add half
+            // an ulp, keep the high half), packed two per 32-bit word and stored 32 scores at a time over
+            // the first 64 TMEM columns of S (the scores are already in registers).
+            const float nm = -m_used;
+            float ls[4] = {0.f, 0.f, 0.f, 0.f};
+  #pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              uint32_t pk[16];
+  #pragma unroll
+              for (int j = 0; j < 16; ++j) {
+                const float x0 = ex2_approx(fmaf(__uint_as_float(r[32 * k + 2 * j]), sl2, nm));
+                const float x1 = ex2_approx(fmaf(__uint_as_float(r[32 * k + 2 * j + 1]), sl2, nm));
+                ls[(2 * j) & 3] += x0;
+                ls[(2 * j + 1) & 3] += x1;
+                pk[j] = __byte_perm(__float_as_uint(x0) + 0x8000u, __float_as_uint(x1) + 0x8000u, 0x7632);
+              }
+              tmem_st16(t_s + 16 * k, pk);
+            }
+            l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+          }
         }
         tc_fence_before();
         mbar_arrive(&bars->p_full[wg]);
@@ -422,7 +494,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pass_kernel(const __grid_const
 cudaError_t launch_tc_pass(const TcPassArgs& args, int num_sms, cudaStream_t stream) {
   static bool configured = false;
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(tc_pass_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(tc_pass_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(tc_pass_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     configured = true;
   }
@@ -430,7 +504,10 @@ cudaError_t launch_tc_pass(const TcPassArgs& args, int num_sms, cudaStream_t str
   const int n_units = (total_tiles + 1) / 2;
   int grid = n_units < num_sms ? n_units : num_sms;
   if (grid < 1) return cudaSuccess;
-  tc_pass_kernel<<<grid, kThreads, kSmemBytes, stream>>>(args);
+  if (args.p.kind == kFull)
+    tc_pass_kernel<false><<<grid, kThreads, kSmemBytes, stream>>>(args);
+  else
+    tc_pass_kernel<true><<<grid, kThreads, kSmemBytes, stream>>>(args);
   return cudaGetLastError();
 }
 
