@@ -167,6 +167,12 @@ SQUAD_API double full_attn_flops(const squad_params_t* p);
  * for non-positive extents or null outputs. Host-only; launches nothing. */
 SQUAD_API squad_status_t squad_window_solve(int T, int H, int W, int* tw, int* hw, int* ww);
 
+/* Self-test of the bounded device-side waits (no counterpart in the paper): launches one small kernel
+ * that waits, with the library's bounded wait, on a barrier that nothing completes. After timeout_ns
+ * (1 ns .. 1 s) the wait gives up, writes SQUAD_ERR_TIMEOUT into *status (a device word the caller
+ * zeroed) and the kernel returns, leaving the context usable. status: 4-byte aligned device pointer. */
+SQUAD_API squad_status_t squad_wait_selftest(uint32_t* status, unsigned long long timeout_ns, squad_stream_t stream);
+
 /* Static string for a status code (never NULL). */
 SQUAD_API const char* squad_status_string(squad_status_t s);
 

@@ -36,6 +36,7 @@ SIGNATURES = {
     "squad_window_solve": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_int),
                                           ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]),
     "full_attn_flops": (ctypes.c_double, [_PP]),
+    "squad_wait_selftest": (ctypes.c_int, [_VP, ctypes.c_ulonglong, _VP]),
     "squad_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "squad_attn_abi_version": (ctypes.c_int, []),
 }

@@ -144,6 +144,13 @@ def test_non_dividing_windows_run_on_the_padded_grid(lib, window):
     assert lib.squad_attn_flops(ctypes.byref(prm)) == pytest.approx(orc.squad_flops(1, 24, 128, n_p, w), rel=1e-12)
 
 
+def test_wait_selftest_rejects_bad_arguments(lib):
+    assert lib.squad_wait_selftest(None, 1000, None) == _lib.SQUAD_ERR_INVALID_ARG
+    assert lib.squad_wait_selftest(ctypes.c_void_p(2), 1000, None) == _lib.SQUAD_ERR_INVALID_ARG      # alignment
+    assert lib.squad_wait_selftest(ctypes.c_void_p(256), 0, None) == _lib.SQUAD_ERR_INVALID_ARG
+    assert lib.squad_wait_selftest(ctypes.c_void_p(256), 2_000_000_000, None) == _lib.SQUAD_ERR_INVALID_ARG
+
+
 def test_workspace_sizes(lib):
     prm = _p()
     n = 21 * 22 * 40

@@ -184,6 +184,11 @@ def test_backward_small_bf16(order):
     run_bwd(2, 2, 128, (21, 4, 8), (21, 2, 4), order, torch.bfloat16)
 
 
+def test_backward_bf16_long_windows_cuda_core_path():
+    """336-token windows: beyond the tensor-core backward's shared memory, so the CUDA-core kernels run."""
+    run_bwd(1, 1, 128, (21, 8, 8), (21, 4, 4), LG, torch.bfloat16)
+
+
 def test_backward_wan21_14b():
     run_bwd(1, 40, 128, (21, 22, 40), (21, 2, 4), LG, torch.bfloat16, heads=[0, 13, 27, 39])
 
