@@ -1,0 +1,115 @@
+"""Sequence-parallel SQuad-Attention over a process group: one all-to-all between the passes.
+
+Both passes of SQuad-Attention are sequence-local (SQuad paper §3.2): the local pass needs the tokens of
+one window, the global pass the tokens of one slot across all windows of one frame. So the n tokens of a
+block can be split over R ranks with one exchange between the passes:
+
+* rank r holds a band of whole window rows: latent rows y in [r*H/R, (r+1)*H/R) of every frame, as a
+  [B, h, T*(H/R)*W, d] tensor in (t, y, x) order. Its windows are complete, so the local pass runs there.
+* an all-to-all regroups the band into frame groups: rank r then holds frames [r*T/R, (r+1)*T/R) of
+  every row. Its slot sequences are complete (a slot (t, dy, dx) only reaches tokens of frame t), so the
+  global pass runs there with the same window (its temporal extent is the frame group).
+* a second all-to-all returns the output to the bands.
+
+The global-then-local order runs the same steps the other way round, and the backward retraces them.
+Requirements: T % R == 0, H % hw == W % ww == 0 and (H / hw) % R == 0.
+
+Compute is the library's single-pass forward and backward (`local_only` / `global_only`); the exchange
+is torch.distributed.all_to_all_single on contiguous buffers, so on GPUs it is NCCL over NVLink. The
+per-rank compute can be replaced (`fwd`, `bwd` arguments) for testing the exchange without a GPU.
+"""
+from __future__ import annotations
+
+import torch
+import torch.distributed as dist
+
+
+class SeqParallelSquad:
+    def __init__(self, grid, window, group=None, fwd=None, bwd=None):
+        self.group = group
+        self.R = dist.get_world_size(group)
+        self.rank = dist.get_rank(group)
+        T, H, W = grid
+        tw, hw, ww = window
+        if tw != T or H % hw or W % ww or T % self.R or (H // hw) % self.R:
+            raise ValueError("needs tw == T, a window that divides H x W, T % R == 0 and (H / hw) % R == 0")
+        self.grid, self.window = tuple(grid), tuple(window)
+        self.Hb, self.Tg = H // self.R, T // self.R
+        self.band_grid = (T, self.Hb, W)                   # the local pass's grid on this rank
+        self.frame_grid = (self.Tg, H, W)                  # the global pass's grid on this rank
+        self.frame_window = (self.Tg, hw, ww)
+        if fwd is None or bwd is None:
+            from .api import squad_attn_bwd, squad_attn_fwd
+            fwd = fwd or (lambda q, k, v, g, w, o: squad_attn_fwd(q, k, v, g, w, o))
+            bwd = bwd or (lambda q, k, v, out, do, ws, g, w, o: squad_attn_bwd(q, k, v, out, do, ws, g, w, o))
+        self._fwd, self._bwd = fwd, bwd
+
+    # -------------------------------------------------------------------------------- exchange
+    def _a2a(self, send):
+        recv = torch.empty_like(send)
+        dist.all_to_all_single(recv, send, group=self.group)
+        return recv
+
+    def band_to_frames(self, x):
+        """[B, h, T*Hb*W, d] (this rank's rows, all frames) -> [B, h, Tg*H*W, d] (its frames, all rows)."""
+        B, h, _, d = x.shape
+        T, _, W = self.grid
+        R, Hb, Tg = self.R, self.Hb, self.Tg
+        send = x.reshape(B, h, R, Tg, Hb, W, d).permute(2, 0, 1, 3, 4, 5, 6).contiguous()   # chunk per frame group
+        recv = self._a2a(send)                                                              # chunk per row band
+        return recv.permute(1, 2, 3, 0, 4, 5, 6).reshape(B, h, Tg * R * Hb * W, d)
+
+    def frames_to_band(self, x):
+        """[B, h, Tg*H*W, d] -> [B, h, T*Hb*W, d], the inverse of band_to_frames."""
+        B, h, _, d = x.shape
+        T, _, W = self.grid
+        R, Hb, Tg = self.R, self.Hb, self.Tg
+        send = x.reshape(B, h, Tg, R, Hb, W, d).permute(3, 0, 1, 2, 4, 5, 6).contiguous()   # chunk per row band
+        recv = self._a2a(send)                                                              # chunk per frame group
+        return recv.permute(1, 2, 0, 3, 4, 5, 6).reshape(B, h, R * Tg * Hb * W, d)
+
+    # -------------------------------------------------------------------------------- passes
+    def _local(self, q, k, v):
+        return self._fwd(q, k, v, self.band_grid, self.window, "local_only")
+
+    def _global(self, q, k, v):
+        return self._fwd(q, k, v, self.frame_grid, self.frame_window, "global_only")
+
+    def forward(self, q, k, v, order="local_then_global"):
+        """q, k, v: this rank's band. Returns (o band, ctx for backward)."""
+        if order == "local_then_global":
+            o1, ws1 = self._local(q, k, v)
+            qf, kf, o1f = self.band_to_frames(q), self.band_to_frames(k), self.band_to_frames(o1)
+            of, ws2 = self._global(qf, kf, o1f)
+            return self.frames_to_band(of), (order, q, k, v, o1, ws1, qf, kf, o1f, of, ws2)
+        if order == "global_then_local":
+            qf, kf, vf = self.band_to_frames(q), self.band_to_frames(k), self.band_to_frames(v)
+            o1f, ws1 = self._global(qf, kf, vf)
+            o1 = self.frames_to_band(o1f)
+            o, ws2 = self._local(q, k, o1)
+            return o, (order, q, k, v, o1, o, ws2, qf, kf, vf, o1f, ws1)
+        raise ValueError(order)
+
+    def backward(self, ctx, dout):
+        """dout: this rank's band of the upstream gradient. Returns (dq, dk, dv) bands."""
+        order = ctx[0]
+        if order == "local_then_global":
+            _, q, k, v, o1, ws1, qf, kf, o1f, of, ws2 = ctx
+            dqf, dkf, do1f = self._bwd(qf, kf, o1f, of, self.band_to_frames(dout), ws2, self.frame_grid,
+                                       self.frame_window, "global_only")
+            dq_g, dk_g, do1 = self.frames_to_band(dqf), self.frames_to_band(dkf), self.frames_to_band(do1f)
+            dq_l, dk_l, dv = self._bwd(q, k, v, o1, do1, ws1, self.band_grid, self.window, "local_only")
+            return dq_l + dq_g, dk_l + dk_g, dv
+        _, q, k, v, o1, o, ws2, qf, kf, vf, o1f, ws1 = ctx
+        dq_l, dk_l, do1 = self._bwd(q, k, o1, o, dout, ws2, self.band_grid, self.window, "local_only")
+        dqf, dkf, dvf = self._bwd(qf, kf, vf, o1f, self.band_to_frames(do1), ws1, self.frame_grid,
+                                  self.frame_window, "global_only")
+        return dq_l + self.frames_to_band(dqf), dk_l + self.frames_to_band(dkf), self.frames_to_band(dvf)
+
+
+def band_of(x, grid, rank, R):
+    """The band of rows [rank*H/R, (rank+1)*H/R) of every frame of a full [B, h, T*H*W, d] tensor."""
+    B, h, _, d = x.shape
+    T, H, W = grid
+    Hb = H // R
+    return x.reshape(B, h, T, H, W, d)[:, :, :, rank * Hb:(rank + 1) * Hb].reshape(B, h, T * Hb * W, d)

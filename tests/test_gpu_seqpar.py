@@ -1,0 +1,43 @@
+"""Sequence-parallel SQuad with the CUDA kernels on one GPU (a one-rank NCCL group: the exchanges are
+the identity, every other step runs), forward and backward against the fp64 oracle (needs a B200)."""
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+
+from oracle import squad_oracle as orc
+from sub_quadratic_two_squad_b200.inputs import make_inputs
+from sub_quadratic_two_squad_b200.seqpar import SeqParallelSquad
+from test_gpu_parity import _dev, _host, check_bf16
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def one_rank_group():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    torch.cuda.set_device(0)
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                            device_id=torch.device("cuda", 0))
+    yield
+    dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("order", ["local_then_global", "global_then_local"])
+def test_sequence_parallel_one_rank(one_rank_group, order):
+    grid, window = (21, 4, 8), (21, 2, 4)
+    n = 21 * 4 * 8
+    x = make_inputs(2, 2, n, 128, dtype="bf16", with_dout=True)
+    q, k, v, do = (_dev(x[s], torch.bfloat16) for s in ("q", "k", "v", "do"))
+    sp = SeqParallelSquad(grid, window)
+    o, ctx = sp.forward(q, k, v, order)
+    dq, dk, dv = sp.backward(ctx, do)
+    oo = {"local_then_global": orc.LOCAL_THEN_GLOBAL, "global_then_local": orc.GLOBAL_THEN_LOCAL}[order]
+    check_bf16(_host(o), orc.squad_attn_fwd(x["q"], x["k"], x["v"], grid, window, oo), "O")
+    for name, mine, ref in zip(("dQ", "dK", "dV"), (dq, dk, dv),
+                               orc.squad_attn_bwd(x["q"], x["k"], x["v"], x["do"], grid, window, oo)):
+        check_bf16(_host(mine), ref, name)
