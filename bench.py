@@ -370,7 +370,8 @@ SWEEP = [
     ("Wan-2.2-5B block", 1, 24, 128, (21, 22, 40), (21, 2, 4),
      ("local_then_global", "global_then_local", "local_only", "global_only"), True, True),
     ("Wan-2.1-1.3B block", 1, 12, 128, (21, 30, 52), (21, 2, 4), ("local_then_global", "global_then_local"), False, False),
-    ("high-resolution 5B block", 1, 24, 128, (21, 44, 80), (21, 4, 4), ("local_then_global",), True, False),
+    ("high-resolution 5B block", 1, 24, 128, (21, 44, 80), (21, 4, 4), ("local_then_global", "local_only", "global_only"),
+     True, False),
     ("Wan-2.1-14B block (training step)", 1, 40, 128, (21, 22, 40), (21, 2, 4), ("local_then_global",), False, True),
 ]
 
