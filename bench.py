@@ -376,7 +376,7 @@ SWEEP = [
 ]
 
 
-def sweep(reps=30):
+def sweep(reps=30, only=None, n_sets=3):
     """Forward (and backward, full attention) device times for every block shape, N(0,1) inputs drawn on
     the device, 3 rotating buffer sets, CUDA events on the launching stream."""
     import torch
@@ -399,14 +399,17 @@ def sweep(reps=30):
         return a.elapsed_time(b) / n_rep
 
     for name, B, h, d, grid, window, orders, with_full, with_bwd in SWEEP:
+        if only is not None and only not in name:
+            continue
         w = dict(B=B, h=h, d=d, grid=grid, window=window)
         n = n_tokens(w)
-        sets = [tuple(torch.randn(B, h, n, d, device=dev, dtype=torch.bfloat16) for _ in range(3)) for _ in range(3)]
+        ns = n_sets
+        sets = [tuple(torch.randn(B, h, n, d, device=dev, dtype=torch.bfloat16) for _ in range(3)) for _ in range(ns)]
         outs = [torch.empty_like(x[0]) for x in sets]
         for order in orders:
-            wss = [squad_attn_fwd(*sets[i], grid, window, order)[1] for i in range(3)]
-            ms = timed(lambda i: squad_attn_fwd(*sets[i % 3], grid, window, order, out=outs[i % 3],
-                                                workspace=wss[i % 3]), reps)
+            wss = [squad_attn_fwd(*sets[i], grid, window, order)[1] for i in range(ns)]
+            ms = timed(lambda i: squad_attn_fwd(*sets[i % ns], grid, window, order, out=outs[i % ns],
+                                                workspace=wss[i % ns]), reps)
             nw = window[0] * window[1] * window[2]
             terms = {"local_only": n * nw, "global_only": n * n / nw}.get(order, n * nw + n * n / nw)
             f = 4.0 * B * h * d * terms
@@ -428,7 +431,7 @@ def sweep(reps=30):
             del wss
         if with_full:
             q, k, v = sets[0]
-            fms = timed(lambda i: full_attn_fwd(*sets[i % 3], grid=grid, out=outs[i % 3]), 3)
+            fms = timed(lambda i: full_attn_fwd(*sets[i % ns], grid=grid, out=outs[i % ns]), 3)
             nf = 4.0 * B * h * d * n * n
             print(json.dumps({"sweep": name, "order": "full_attn_fwd", "n": n, "ms_per_block": fms,
                               "tflops": nf / (fms * 1e-3) / 1e12, "tensor_frac": nf / (fms * 1e-3) / 1e12 / tf_peak}),
@@ -445,9 +448,12 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true", help="time every block shape (one JSON line each) and exit")
+    ap.add_argument("--only", default=None, help="with --sweep: only the block shapes whose name contains this")
+    ap.add_argument("--sets", type=int, default=3, help="with --sweep: rotating buffer sets (3 keep inputs > L2)")
+    ap.add_argument("--reps", type=int, default=30, help="with --sweep: timed calls per order")
     args = ap.parse_args()
     if args.sweep:
-        sweep()
+        sweep(reps=args.reps, only=args.only, n_sets=args.sets)
         return
     args.warmup = max(args.warmup, 3)
     world = int(os.environ.get("WORLD_SIZE", "1"))
