@@ -622,7 +622,10 @@ bool short_plan(ShortArgs& a) {
   // One unit holds up to 6 allocations (or 3 for a shared pair) at once.
   for (int i = 0; i < a.n_passes; ++i) {
     const uint32_t need = (a.pass[i].p.seq_len > 128 ? 3u : 6u) * a.pass[i].alloc_bytes;
-    if (need + max_alloc > a.ring_bytes) return false;   // + max_alloc: room lost to a wrap
+    if (need + max_alloc <= a.ring_bytes) continue;   // + max_alloc: room lost to a wrap
+    // One pass has one allocation size: a ring of whole allocations loses nothing at the wrap.
+    if (a.n_passes != 1 || need > a.ring_bytes) return false;
+    a.ring_bytes = a.ring_bytes / a.pass[i].alloc_bytes * a.pass[i].alloc_bytes;
   }
   a.smem_bytes = fixed + a.ring_bytes;
   const int H = a.g.B * a.g.h;
