@@ -29,8 +29,8 @@ PAGES_MS = 4.27   # pages' SQuad attention latency per block for this workload (
 # DRAM traffic of one launch of the forward kernel from the ncu capture summarised in
 # profiles/short_kernel_wan22_5b_fwd.md (dram__bytes_read.sum + dram__bytes_write.sum), valid only for
 # the kernel source it was measured on (sha1 prefix below); otherwise reported as null.
-PROFILED_TRAFFIC_BYTES = (438.608128 + 193.176576) * 1e6
-PROFILED_KERNEL_SHA1 = "972f88535881708b"
+PROFILED_TRAFFIC_BYTES = (440.588288 + 192.799744) * 1e6
+PROFILED_KERNEL_SHA1 = "2468718f45f72560"
 PROFILED_KERNEL_SRC = os.path.join(ROOT, "sub_quadratic_two_squad_b200", "csrc", "attn_short.cu")
 
 
