@@ -292,13 +292,13 @@ __global__ void __launch_bounds__(kThreads, 1) short_kernel(const __grid_constan
         vstart[idx % kND] = vs;
         return true;
       };
-      auto load = [&](const PassView& ps, const CUtensorMap* m, int bh, int sigma, uint32_t idx, uint32_t off,
+      // Q, K and V of one sequence are the same box of three tensors: its coordinates c are computed
+      // once per sequence.
+      auto load = [&](const PassView& ps, const CUtensorMap* m, const int (&c)[5], uint32_t idx, uint32_t off,
                       uint32_t vs) -> bool {
         if (!make_room(idx, vs, ps.alloc)) return false;
         uint64_t* fb = &bars->full[idx % kND];
         mbar_arrive_expect_tx(fb, 2u * static_cast<uint32_t>(ps.p.seq_len) * 128u);
-        int c[5];
-        chunk_coords(g, ps.p, ps.variant, bh, sigma, 0, 0, c);
         tma_load_5d(ring + off, m, fb, c[0], c[1], c[2], c[3], c[4]);
         tma_load_5d(ring + off + ps.panel, m, fb, c[0] + 64, c[1], c[2], c[3], c[4]);
         return true;
@@ -315,11 +315,15 @@ __global__ void __launch_bounds__(kThreads, 1) short_kernel(const __grid_constan
         const Unit u = plan_unit(a, U, cur, RB);
         const PassView ps = view_of(a, u.pass);
         const int nsrc = u.shared ? 1 : u.nw;
+        int cs[2][5];
+#pragma unroll
+        for (int w = 0; w < 2; ++w)
+          if (w < nsrc) chunk_coords(g, ps.p, ps.variant, u.bh, u.sigma[w], 0, 0, cs[w]);
 #pragma unroll
         for (int w = 0; w < 2; ++w) {
           if (w < nsrc && ok) {
-            ok = load(ps, ps.q, u.bh, u.sigma[w], u.q[w], u.qo[w], u.qvs[w]);
-            if (ok) ok = load(ps, ps.k, u.bh, u.sigma[w], u.k[w], u.ko[w], u.kvs[w]);
+            ok = load(ps, ps.q, cs[w], u.q[w], u.qo[w], u.qvs[w]);
+            if (ok) ok = load(ps, ps.k, cs[w], u.k[w], u.ko[w], u.kvs[w]);
           }
         }
         if (ok && u.pass == 1) {
@@ -341,7 +345,7 @@ __global__ void __launch_bounds__(kThreads, 1) short_kernel(const __grid_constan
         }
 #pragma unroll
         for (int w = 0; w < 2; ++w)
-          if (w < nsrc && ok) ok = load(ps, ps.v, u.bh, u.sigma[w], u.v[w], u.vo[w], u.vvs[w]);
+          if (w < nsrc && ok) ok = load(ps, ps.v, cs[w], u.v[w], u.vo[w], u.vvs[w]);
       }
       if (!ok) {   // make sure the other warps see the end of the work
         for (int i = 0; i < kQ; ++i) {
