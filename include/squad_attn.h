@@ -2,22 +2,23 @@
  * squad_attn.h -- C ABI of the SQuad-Attention CUDA library (sm_100a, one GPU).
  *
  * SQuad-Attention ("SQuad: Sub-Quadratic Attention Distillation for Efficient Video Generation")
- * replaces full softmax self-attention over a T x H x W latent token grid by two ordinary softmax
- * attentions run one after the other (paper §3.2; agihunt digest, "SQuad-Attention composes two
- * ordinary softmax attentions"):
+ * replaces full softmax self-attention over a T x H x W latent token grid by a sequence of two plain
+ * softmax attentions, the second fed by the first (paper §3.2; agihunt.info digest, the paragraph that
+ * defines the operator):
  *
  *   local pass  Attn_L: every token attends to the w = tw*hw*ww tokens of its window. A window spans
- *                       the full temporal extent (tw = T) and an hw x ww block of space (agihunt
- *                       digest, "The window size carries the whole argument": 21x2x4 = 168).
+ *                       every frame (tw = T) and an hw x ww block of space (agihunt.info digest,
+ *                       the paragraph on the window size: 21x2x4 = 168 at n = 18480).
  *   global pass Attn_G: the n/w tokens that occupy the same slot (t, y mod hw, x mod ww) in every
  *                       window attend to one another; the pass-1 output is its value stream (paper
  *                       appendix "Reachability": the two-hop path (c',j') -> (c',j) -> (c,j)).
  *
- * Between the passes there is only re-indexing (paper §4.3); this library never materialises a
- * permuted copy: both views are strided boxes of the caller's [B, h, n, d] tensors.
+ * The passes are joined by re-indexing alone, with no arithmetic (paper appendix "Cost of the two
+ * passes"); this library never materialises a permuted copy: both views are strided boxes of the
+ * caller's [B, h, n, d] tensors.
  *
- * A window that does not divide H x W forces reflect padding (paper appendix, "Conformance to the
- * theoretical curves is quantitative"): each frame is padded at the bottom and right up to multiples
+ * When hw does not divide H or ww does not divide W, the grid is reflect-padded (paper appendix,
+ * "Conformance to the theoretical curves is quantitative"): each frame is padded at the bottom and right up to multiples
  * of hw and ww, reflecting about the edge (the edge token is not repeated); both passes run on the
  * padded grid (padded copies of q, k, v live in the forward workspace) and o is cropped back. The
  * backward is that composition's gradient: zero upstream gradient on the padded tokens, and each input
@@ -85,7 +86,7 @@ typedef struct {
   int B, h, d;      /* batch, heads, head dim (d in {64, 128}; bf16 tensor-core path: d == 128)  */
   int T, H, W;      /* latent grid; n = T*H*W                                                     */
   int tw, hw, ww;   /* window; tw must equal T (the window spans all frames), 1 <= hw <= H, 1 <= ww <= W;
-                       a window that does not divide H x W is handled by reflect padding            */
+                       hw not dividing H or ww not dividing W is handled by reflect padding        */
   int order;        /* squad_order_t                                                              */
   int dtype;        /* squad_dtype_t                                                              */
   float scale;      /* softmax scale; 0 selects 1/sqrt(d) (paper eq. 5)                           */
@@ -159,8 +160,9 @@ SQUAD_API squad_status_t squad_attn_fwd_noalloc(const squad_params_t* p, const v
 SQUAD_API double squad_attn_flops(const squad_params_t* p);
 SQUAD_API double full_attn_flops(const squad_params_t* p);
 
-/* The window for a T x H x W grid, re-solved per resolution as the paper's appendix ("Conformance to
- * the theoretical curves is quantitative") describes: tw = T; for each hw the ww whose ratio hw:ww is
+/* The window for a T x H x W grid, chosen anew at each resolution as the paper's appendix describes
+ * ("What is measured" for the rule; "Conformance to the theoretical curves is quantitative" for the
+ * cost of the window actually used): tw = T; for each hw the ww whose ratio hw:ww is
  * closest to H:W (in log ratio, the smaller ww on a tie); and, among those, the hw whose cost
  * n'm + n'^2/m is least, m = T*hw*ww the window size and n' the reflect-padded token count (ties: the
  * smaller hw). Recovers 21x2x4 at 21x22x40 and at 21x30x52. Writes *tw, *hw, *ww; SQUAD_ERR_INVALID_ARG

@@ -6,20 +6,20 @@ reference``) may use it. It shares no code with the CUDA library; both sides are
 generator in ``sub_quadratic_two_squad_b200/inputs.py``, which holds no attention arithmetic.
 
 Sources ("SQuad: Sub-Quadratic Attention Distillation for Efficient Video Generation", as printed on
-the paperpeel page, the agihunt digest and the romaanj.github.io review):
+the paperpeel.com page, the agihunt.info digest, the romaanj.github.io review and the gist.science
+summary):
 
 * Full softmax self-attention softmax(Q K^T / sqrt(d)) V per head -- paper §3.1 (eq. 5).
-* SQuad-Attention is two ordinary softmax attentions run one after the other; between them there is
-  only re-indexing, the attended axis becomes the sequence and the other axis is folded into the
-  batch/head dimension -- agihunt digest, paragraph "SQuad-Attention composes two ordinary softmax
-  attentions"; paper §4.3 ("two passes are ordinary softmax attentions separated by pure
-  re-indexing").
-* Local pass: each token attends inside its window; the window spans the full temporal extent and
-  tiles space (e.g. 21x2x4 = 168 tokens at n = 18480) -- agihunt digest, "The window size carries the
-  whole argument"; review, "Method".
+* SQuad-Attention is a sequence of two plain softmax attentions, the second fed by the first; the
+  passes are joined by re-indexing alone: each takes the axis it attends over as its sequence and
+  merges the remaining index into the batch of heads -- agihunt.info digest, the paragraph that
+  defines the operator; paper appendix "Cost of the two passes" and "Analyzing the results".
+* Local pass: each token attends inside its window; the window covers every frame and an hw x ww
+  block of space (e.g. 21x2x4 = 168 tokens at n = 18480) -- agihunt.info digest, the paragraph on the
+  window size; review, "Method".
 * Global pass: tokens at the same position (slot) inside their windows attend across all windows, and
   the local output is its value stream -- paper appendix "Reachability" (two-hop path (c',j') ->
-  (c',j) -> (c,j)); gist.science technical summary, "Composição".
+  (c',j) -> (c,j)); gist.science summary, item "Composição".
 * Order: local->global is the paper's default, global->local the ablated reverse; for G->L the
   effective weight is beta_{j->j'}^{c} alpha_{c->c'}^{j'} -- paper appendix "On the ordering".
 * Cost: 4hd(n w + n^2 / w) for the two passes and 4hdn^2 for full attention -- paper appendix
@@ -34,8 +34,8 @@ Readings where the pages are silent (equations 7-9 were lost in extraction):
   not depend on these orders (softmax sums are permutation invariant; outputs go back to token order).
 * The backward pass is the chain rule through both passes; the pages do not print it.
 * Grids the window does not divide (paper appendix, "Conformance to the theoretical curves is
-  quantitative": such a window "forces a little reflect padding", and the window is re-solved per
-  resolution with w_t = T and w_h:w_w following the grid's aspect ratio). Readings: reflect padding
+  quantitative": such grids are reflect-padded, and at each resolution the window is chosen anew,
+  spanning all frames, with a height-to-width split set by the grid's aspect ratio). Readings: reflect padding
   (the edge token is not repeated) at the bottom of H and the right of W in every frame, up to the next
   multiple of the window; both passes run on the padded grid and the output is cropped back, so the
   gradient of an input token sums over its padded copies. The solver takes, among windows with
@@ -60,7 +60,7 @@ def window_partition(T: int, H: int, W: int, tw: int, hw: int, ww: int) -> np.nd
     lists the N_w tokens that occupy slot j in every window (the global pass attends along a column).
     """
     if tw != T:
-        raise ValueError("the window spans the full temporal extent: tw must equal T")
+        raise ValueError("the window covers every frame: tw must equal T")
     if H % hw or W % ww:
         raise ValueError("window must tile the H x W grid exactly")
     nwy, nwx = H // hw, W // ww
@@ -219,7 +219,8 @@ def _aspect_ww(hw: int, H: int, W: int) -> int:
 def window_solve(T: int, H: int, W: int):
     """The window (T, hw, ww) for a T x H x W grid: w_t = T, ww following the aspect ratio for each hw,
     and the hw whose padded cost n'm + n'^2/m (m = T hw ww, n' = the reflect-padded token count) is
-    least."""
+    least (paper appendix "What is measured" for the rule; "Conformance to the theoretical curves is
+    quantitative" for scoring the cost of the window actually used)."""
     best = None
     for hw in range(1, H + 1):
         ww = _aspect_ww(hw, H, W)
@@ -357,7 +358,7 @@ def composed_matrix(Q, K, grid, window, order=LOCAL_THEN_GLOBAL, scale=None):
 
     Obtained by pushing the n one-hot value vectors through both passes (V = identity, dv = n). Entry
     M[u, v] is the effective weight gamma from source token v to target token u (paper appendix
-    "Reachability": a product of two softmax weights).
+    "Reachability": the local weight times the global weight along the two-hop path).
     """
     B, h, n, _ = Q.shape
     eye = np.broadcast_to(np.eye(n), (B, h, n, n))

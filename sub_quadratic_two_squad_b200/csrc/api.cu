@@ -75,8 +75,8 @@ squad_status_t validate(const squad_params_t* p, bool windowed, Grid* g, float* 
     if (p->order < SQUAD_LOCAL_THEN_GLOBAL || p->order > SQUAD_GLOBAL_ONLY) return SQUAD_ERR_INVALID_ARG;
     if (p->tw < 1 || p->hw < 1 || p->ww < 1) return SQUAD_ERR_INVALID_ARG;
     if (p->tw > p->T || p->hw > p->H || p->ww > p->W) return SQUAD_ERR_INVALID_ARG;
-    // The window spans the full temporal extent (tw < T is outside the method); space is tiled by the
-    // window over the (padded) grid.
+    // The window covers every frame (tw < T is outside the method); space is tiled by the window over
+    // the (padded) grid.
     if (p->tw != p->T) return SQUAD_ERR_UNSUPPORTED;
     gg.hw = p->hw;
     gg.ww = p->ww;

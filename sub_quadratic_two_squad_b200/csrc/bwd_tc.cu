@@ -2,8 +2,8 @@
 //
 // Each pass of SQuad-Attention is ordinary softmax attention inside each sequence (a window for the
 // local pass, a slot across windows for the global pass; SQuad paper §3.2), so its gradients are those
-// of softmax attention, sequence by sequence (agihunt digest, "SQuad-Attention composes two ordinary
-// softmax attentions"; the chain rule through both passes is applied by the caller). With
+// of softmax attention, sequence by sequence (agihunt.info digest, the paragraph that defines the
+// operator; the chain rule through both passes is applied by the caller). With
 // P = softmax(scale Q K^T) recomputed from the forward's LSE, dO the gradient of the pass output:
 //   dP = dO V^T,  D_i = sum_j P_ij dP_ij,  dS = P o (dP - D),
 //   dQ = scale dS K,  dK = scale dS^T Q,  dV = P^T dO.

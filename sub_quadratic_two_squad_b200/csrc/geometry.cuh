@@ -2,8 +2,8 @@
 // into chunks of at most 128 rows (one tensor-core tile of queries, or one block of keys/values).
 //
 // SQuad re-indexes the [B, h, n, d] token grid in two ways (paper §3.2 "Construction of the local and
-// global token views"; agihunt digest: the attended axis becomes the sequence, the other axis is
-// folded into the batch/head dimension):
+// global token views"; agihunt.info digest: each pass takes the axis it attends over as its sequence
+// and merges the remaining index into the batch of heads):
 //   LOCAL  sequence sigma = window c = (wy, wx), rows ordered (t, dy, dx): "lines" are frames t,
 //          each line is the hw x ww block of one frame.
 //   GLOBAL sequence sigma = slot j = (t, dy, dx), rows ordered (wy, wx): "lines" are window rows wy,

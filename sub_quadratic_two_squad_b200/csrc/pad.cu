@@ -1,6 +1,6 @@
 // Reflect padding of the latent grid for windows that do not divide it, and its adjoints (SQuad paper,
-// appendix "Conformance to the theoretical curves is quantitative": a window that does not divide the
-// latent grid forces a little reflect padding). Each frame is padded at the bottom (H) and the right
+// appendix "Conformance to the theoretical curves is quantitative", which names reflect padding as the
+// way such grids are handled). Each frame is padded at the bottom (H) and the right
 // (W) end up to a multiple of the window; reflect = the edge token is not repeated, so padded index
 // i >= size reads index 2 (size - 1) - i. Tensors are [B*h, T, H, W, d] rows of d elements.
 #include <cuda_runtime.h>

@@ -10,8 +10,8 @@ Recipe (one Philox stream per tensor, counter-based and platform independent):
   it, so the oracle (fp64) and the kernels (bf16 operands) start from identical numbers.
 * Heavy tail (the Wan-shaped forward workloads): for every (b, head), round(0.02 * n) key tokens,
   drawn without replacement from a seeded permutation, have their K row multiplied by 4. The pages
-  describe video-DiT attention maps as sparse and heavy tailed, with the mass on a few critical tokens
-  (SQuad paper, agihunt digest, paragraph "SQuad starts from a known observation"); scaling 2 % of the
+  describe video-DiT attention maps as sparse, with most of each row's weight on a handful of keys
+  (agihunt.info digest, the paragraph on the motivating observation); scaling 2 % of the
   keys by 4 gives logits with a standard deviation of 4 on those keys and of 1 elsewhere, which
   reproduces that shape. Multiplying by 4 is exact in bf16.
 
