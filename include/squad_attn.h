@@ -126,7 +126,9 @@ SQUAD_API squad_status_t squad_attn_bwd(const squad_params_t* p, const void* q, 
 
 /* Full softmax self-attention softmax(q k^T * scale) v over all n tokens per head (paper eq. 5),
  * the operator SQuad replaces. The window fields and `order` of *p are ignored (grid still gives n).
- * lse_or_null: optional [B,h,n] fp32 output of the natural-log log-sum-exp per query. */
+ * lse_or_null: optional [B,h,n] fp32 output of the natural-log log-sum-exp per query. This call has
+ * no workspace and so no status word: its device-side waits are bounded too, but a wait that gives
+ * up (leaving o incomplete) is not reported. */
 SQUAD_API squad_status_t full_attn_fwd(const squad_params_t* p, const void* q, const void* k, const void* v,
                              void* o, float* lse_or_null, squad_stream_t stream);
 

@@ -1,6 +1,7 @@
 // C ABI of the SQuad-Attention library (include/squad_attn.h): argument validation, TMA tensor maps
 // for the window and slot views, and the launch sequence of the two passes.
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstdlib>
@@ -247,11 +248,14 @@ bool tc_eligible(const squad_params_t* prm, const Grid& g, const PassGeom& p) {
 int num_sms_current() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-  static int cache[64] = {0};
-  if (dev >= 0 && dev < 64 && cache[dev] > 0) return cache[dev];
+  static std::atomic<int> cache[64];   // per device; 0 = not looked up yet (calls may come from many threads)
+  if (dev >= 0 && dev < 64) {
+    const int c = cache[dev].load(std::memory_order_relaxed);
+    if (c > 0) return c;
+  }
   int sms = 0;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-  if (dev >= 0 && dev < 64) cache[dev] = sms;
+  if (dev >= 0 && dev < 64) cache[dev].store(sms, std::memory_order_relaxed);
   return sms;
 }
 

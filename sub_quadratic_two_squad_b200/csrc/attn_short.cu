@@ -34,6 +34,7 @@
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
+#include "host_util.h"
 #include "ptx.cuh"
 #include "geometry.cuh"
 #include "short_pass.h"
@@ -643,12 +644,9 @@ bool short_plan(ShortArgs& a) {
 }
 
 cudaError_t launch_short(const ShortArgs& args, int num_sms, cudaStream_t stream) {
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(short_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  static std::atomic<unsigned long long> set{0};
+  const cudaError_t e = max_dyn_smem_once(short_kernel, kSmemLimit, set);
+  if (e != cudaSuccess) return e;
   const int H = args.g.B * args.g.h;
   const int n_units = H * (args.pass[0].units_per_head + (args.n_passes == 2 ? args.pass[1].units_per_head : 0));
   const int grid = n_units < num_sms ? n_units : num_sms;

@@ -24,6 +24,7 @@
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
+#include "host_util.h"
 #include "ptx.cuh"
 #include "geometry.cuh"
 #include "tc_pass.h"
@@ -492,14 +493,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pass_kernel(const __grid_const
 }
 
 cudaError_t launch_tc_pass(const TcPassArgs& args, int num_sms, cudaStream_t stream) {
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(tc_pass_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(tc_pass_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  static std::atomic<unsigned long long> set_split{0}, set_whole{0};
+  cudaError_t e = max_dyn_smem_once(tc_pass_kernel<true>, kSmemBytes, set_split);
+  if (e != cudaSuccess) return e;
+  e = max_dyn_smem_once(tc_pass_kernel<false>, kSmemBytes, set_whole);
+  if (e != cudaSuccess) return e;
   const int total_tiles = args.g.B * args.g.h * args.p.n_seq * args.p.n_chunks;
   const int n_units = (total_tiles + 1) / 2;
   int grid = n_units < num_sms ? n_units : num_sms;

@@ -21,6 +21,7 @@
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
+#include "host_util.h"
 #include "ptx.cuh"
 #include "geometry.cuh"
 #include "bwd_pass.h"
@@ -369,12 +370,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
 }  // namespace
 
 cudaError_t launch_bwd_tc(const BwdTcArgs& a, cudaStream_t stream) {
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kBwdSmemLimit);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  static std::atomic<unsigned long long> set{0};
+  const cudaError_t e = max_dyn_smem_once(bwd_tc_kernel, kBwdSmemLimit, set);
+  if (e != cudaSuccess) return e;
   const unsigned grid = static_cast<unsigned>(a.g.B * a.g.h * a.p.n_seq);
   if (grid == 0) return cudaSuccess;
   bwd_tc_kernel<<<grid, kBwdThreads, a.smem_bytes, stream>>>(a);
