@@ -42,7 +42,12 @@ Readings where the pages are silent (equations 7-9 were lost in extraction):
   w_t = T and for each w_h the w_w whose ratio w_h:w_w is closest to H:W (log ratio), the one with the
   least cost n'm + n'^2/m on the padded count n'.
 
-Every array here is float64. Pins: tests/test_oracle_pins.py.
+* More than two passes (the paper names composing more passes as open, §5 "Limitations and future
+  work", and defines none): nested windows, each spatial axis factored into k levels, pass p
+  attending along level p's digits with the others fixed (pass 1 also along the frames); k = 2 is
+  SQuad, k = 1 full attention. See the k-pass section below.
+
+Every array here is float64. Pins: tests/test_oracle_pins.py and tests/test_oracle_kpass.py.
 """
 from __future__ import annotations
 
@@ -374,3 +379,136 @@ def squad_flops(B: int, h: int, d: int, n: int, w: int) -> float:
 def full_flops(B: int, h: int, d: int, n: int) -> float:
     """4 B h d n^2: QK^T and PV of full attention."""
     return 4.0 * B * h * d * n * n
+
+
+# ----------------------------------------------------------------------------------------------
+# More than two composed passes: nested windows
+# ----------------------------------------------------------------------------------------------
+# The paper names composing more than two passes as an open direction (§5 "Limitations and future
+# work"; review, "Sparks") and defines no partition for a third pass. The reading taken here is the
+# plainest generalisation of the two passes, nested windows:
+#
+# * each spatial axis is factored into k levels, H = h_1 h_2 ... h_k and W = w_1 w_2 ... w_k, and a
+#   token's row and column are mixed-radix numbers with level 1 least significant:
+#   y = a_1 + h_1 (a_2 + h_2 (a_3 + ...)), x = b_1 + w_1 (b_2 + w_2 (b_3 + ...)), 0 <= a_p < h_p,
+#   0 <= b_p < w_p;
+# * pass p attends among the tokens that agree on every digit except (a_p, b_p); pass 1 also spans
+#   all frames t (the window of the two-pass method covers every frame), the other passes keep t;
+# * every pass takes the same Q and K; its values are the previous pass's output (v for the first).
+#
+# With k = 2 this is SQuad with window (T, h_1, w_1): pass 1 is the local pass (inside a window),
+# pass 2 the global pass (one slot across the h_2 x w_2 windows). With k = 1 it is full attention.
+# "forward" runs level 1 first (the analogue of local->global), "reverse" level k first.
+
+KPASS_FORWARD = "forward"
+KPASS_REVERSE = "reverse"
+
+
+def _check_levels(grid, levels):
+    T, H, W = grid
+    levels = [(int(a), int(b)) for a, b in levels]
+    if not levels or any(a < 1 or b < 1 for a, b in levels):
+        raise ValueError("levels: k >= 1 pairs (h_p, w_p) of positive integers")
+    if int(np.prod([a for a, _ in levels])) != H or int(np.prod([b for _, b in levels])) != W:
+        raise ValueError("the levels must factor the grid: prod h_p = H and prod w_p = W")
+    return levels
+
+
+def level_groups(grid, levels, p: int) -> np.ndarray:
+    """Token indices of the sequences of pass p (0-based level), as an int array [G, s].
+
+    A row lists the tokens that share every digit except level p's (and, for p = 0, the frame), in a
+    fixed order; the rows partition the n tokens.
+    """
+    T, H, W = grid
+    levels = _check_levels(grid, levels)
+    tok = np.arange(T * H * W, dtype=np.int64)
+    t, y, x = tok // (H * W), (tok // W) % H, tok % W
+    a, b = [], []
+    for hp, wp in levels:
+        a.append(y % hp)
+        b.append(x % wp)
+        y, x = y // hp, x // wp
+    hp, wp = levels[p]
+    member = a[p] * wp + b[p]
+    size = hp * wp
+    if p == 0:
+        member = t * size + member
+        size *= T
+    key = np.zeros_like(tok)
+    for q, (hq, wq) in enumerate(levels):
+        if q != p:
+            key = key * (hq * wq) + a[q] * wq + b[q]
+    if p != 0:
+        key = key * T + t
+    order = np.lexsort((member, key))
+    return tok[order].reshape(-1, size)
+
+
+def _kpass_levels_in_order(levels, order):
+    if order not in (KPASS_FORWARD, KPASS_REVERSE):
+        raise ValueError(order)
+    idx = list(range(len(levels)))
+    return idx if order == KPASS_FORWARD else idx[::-1]
+
+
+def kpass_fwd(Q, K, V, grid, levels, order=KPASS_FORWARD, scale=None, return_aux=False):
+    """k nested-window passes composed, each taking the previous one's output as values.
+
+    grid = (T, H, W); levels = [(h_1, w_1), ..., (h_k, w_k)]. With return_aux, also returns the inputs
+    of every executed pass's values and each pass's log-sum-exp (lists in execution order).
+    """
+    Q, K, V = _f64(Q), _f64(K), _f64(V)
+    sc = _scale(Q.shape[-1], scale)
+    values, lses = [], []
+    x = V
+    for p in _kpass_levels_in_order(levels, order):
+        values.append(x)
+        x, lse = _pass(Q, K, x, level_groups(grid, levels, p), sc)
+        lses.append(lse)
+    if return_aux:
+        return x, dict(values=values, lse=lses)
+    return x
+
+
+def kpass_bwd(Q, K, V, dO, grid, levels, order=KPASS_FORWARD, scale=None):
+    """Gradients (dQ, dK, dV) of <dO, kpass_fwd(Q, K, V)>: the passes' backward in reverse execution
+    order, each passing the gradient of its values on to the pass before; dQ and dK sum every pass's
+    share."""
+    Q, K, V, dO = _f64(Q), _f64(K), _f64(V), _f64(dO)
+    sc = _scale(Q.shape[-1], scale)
+    seq = _kpass_levels_in_order(levels, order)
+    _, aux = kpass_fwd(Q, K, V, grid, levels, order, scale, return_aux=True)
+    dQ, dK = np.zeros_like(Q), np.zeros_like(K)
+    g = dO
+    B, h = Q.shape[:2]
+    for e in range(len(seq) - 1, -1, -1):
+        groups = level_groups(grid, levels, seq[e])
+        x = aux["values"][e]
+        gv = np.empty_like(x)
+        for b in range(B):
+            for hh in range(h):
+                dq, dk, dv = softmax_attention_bwd(Q[b, hh][groups], K[b, hh][groups], x[b, hh][groups],
+                                                   g[b, hh][groups], sc)
+                dQ[b, hh][groups] += dq
+                dK[b, hh][groups] += dk
+                gv[b, hh][groups] = dv
+        g = gv
+    return dQ, dK, g
+
+
+def kpass_composed_matrix(Q, K, grid, levels, order=KPASS_FORWARD, scale=None):
+    """The n x n matrix M with kpass_fwd(Q, K, V) = M V, per (b, head) (one-hot values)."""
+    B, h, n, _ = Q.shape
+    eye = np.broadcast_to(np.eye(n), (B, h, n, n))
+    return kpass_fwd(Q, K, eye, grid, levels, order, scale)
+
+
+def kpass_flops(B: int, h: int, d: int, grid, levels) -> float:
+    """4 B h d n (m_1 + ... + m_k): pass p runs n/m_p sequences of m_p tokens (m_1 = T h_1 w_1,
+    m_p = h_p w_p otherwise), each costing 4 m_p^2 d FLOPs for QK^T and PV."""
+    T, H, W = grid
+    levels = _check_levels(grid, levels)
+    n = T * H * W
+    m = [T * levels[0][0] * levels[0][1]] + [a * b for a, b in levels[1:]]
+    return 4.0 * B * h * d * n * float(sum(m))
