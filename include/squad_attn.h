@@ -18,11 +18,12 @@
  * caller's [B, h, n, d] tensors.
  *
  * When hw does not divide H or ww does not divide W, the grid is reflect-padded (paper appendix,
- * "Conformance to the theoretical curves is quantitative"): each frame is padded at the bottom and right up to multiples
- * of hw and ww, reflecting about the edge (the edge token is not repeated); both passes run on the
- * padded grid (padded copies of q, k, v live in the forward workspace) and o is cropped back. The
- * backward is that composition's gradient: zero upstream gradient on the padded tokens, and each input
- * token's gradient summed over its padded copies. squad_window_solve picks a window.
+ * "Conformance to the theoretical curves is quantitative"): each frame is padded at the bottom and
+ * right up to multiples of hw and ww, reflecting about the edge (the edge token is not repeated);
+ * both passes run on the padded grid (padded copies of q, k, v live in the forward workspace) and o
+ * is cropped back. The backward is that composition's gradient: zero upstream gradient on the padded
+ * tokens, and each input token's gradient summed over its padded copies. squad_window_solve picks a
+ * window.
  *
  * Conventions shared by every entry point
  * ---------------------------------------
@@ -176,6 +177,80 @@ SQUAD_API squad_status_t squad_window_solve(int T, int H, int W, int* tw, int* h
  * (1 ns .. 1 s) the wait gives up, writes SQUAD_ERR_TIMEOUT into *status (a device word the caller
  * zeroed) and the kernel returns, leaving the context usable. status: 4-byte aligned device pointer. */
 SQUAD_API squad_status_t squad_wait_selftest(uint32_t* status, unsigned long long timeout_ns, squad_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------------
+ * k composed passes over nested windows
+ *
+ * The paper names composing more than two passes as an open direction (§5 "Limitations and future
+ * work") and defines no partition for them. This library's reading, the plainest generalisation of
+ * the two passes: each spatial axis is factored into k levels, H = h_1 h_2 ... h_k and
+ * W = w_1 w_2 ... w_k, so that a token's row and column are mixed-radix numbers with level 1 least
+ * significant, y = a_1 + h_1 (a_2 + h_2 (a_3 + ...)) and x = b_1 + w_1 (b_2 + ...). Pass p attends
+ * among the tokens that agree on every digit except (a_p, b_p); pass 1 also spans all frames (as the
+ * two-pass window does), the others keep the frame. Every pass takes the same q and k; its values are
+ * the previous pass's output. k = 2 is SQuad with window (T, h_1, w_1); k = 1 is full attention.
+ * Cost: 4 B h d n (m_1 + ... + m_k) with m_1 = T h_1 w_1 and m_p = h_p w_p.
+ *
+ * Each pass is one single-pass problem of this library on a reinterpretation of the same contiguous
+ * [B, h, n, d] buffers (no copy): pass 1 is SQUAD_LOCAL_ONLY with window (T, h_1, w_1); pass p >= 2 is
+ * SQUAD_GLOBAL_ONLY on B' = B h T H/(h_1...h_p) sequences-of-heads of the grid
+ * (1, (h_1...h_p) W/(w_1...w_p), w_1...w_p) with window (1, (h_1...h_{p-1}) W/(w_1...w_p), w_1...w_{p-1}).
+ * squad_kpass_pass_params reports that problem. Layout, dtypes, pointers, streams and errors follow
+ * the conventions above; the levels must factor the grid exactly (no padding).
+ * ------------------------------------------------------------------------------------------------ */
+#define SQUAD_KPASS_MAX_LEVELS 4
+
+typedef enum {
+  SQUAD_KPASS_FORWARD = 0,   /* level 1 first (the analogue of local -> global) */
+  SQUAD_KPASS_REVERSE = 1    /* level k first                                   */
+} squad_kpass_order_t;
+
+typedef struct {
+  int B, h, d;                              /* as in squad_params_t                                   */
+  int T, H, W;                              /* latent grid; n = T*H*W                                 */
+  int k;                                    /* passes, 1 .. SQUAD_KPASS_MAX_LEVELS                     */
+  int level_h[SQUAD_KPASS_MAX_LEVELS];      /* h_1 .. h_k (first k used), product H                    */
+  int level_w[SQUAD_KPASS_MAX_LEVELS];      /* w_1 .. w_k, product W; every pass attends over at least
+                                               two tokens (T h_1 w_1 >= 2 and h_p w_p >= 2)             */
+  int order;                                /* squad_kpass_order_t                                     */
+  int dtype;                                /* squad_dtype_t                                           */
+  float scale;                              /* softmax scale of every pass; 0 selects 1/sqrt(d)        */
+} squad_kpass_params_t;
+
+/* The single-pass problem that level `level` (0-based: 0 is the innermost window) runs, written to
+ * *out (its order is SQUAD_LOCAL_ONLY or SQUAD_GLOBAL_ONLY). Host-only; launches nothing.
+ * SQUAD_ERR_INVALID_ARG for invalid parameters or level; SQUAD_ERR_UNSUPPORTED where a pass is not
+ * supported (as for squad_attn_fwd, or a level past the first of one token). */
+SQUAD_API squad_status_t squad_kpass_pass_params(const squad_kpass_params_t* p, int level, squad_params_t* out);
+
+/* Bytes of forward workspace: a control block, the k - 1 intermediate outputs (input dtype) and the
+ * k per-pass log-sum-exps (fp32, [B, h, n] each). 0 for invalid parameters. */
+SQUAD_API size_t squad_kpass_fwd_workspace_bytes(const squad_kpass_params_t* p);
+
+/* Forward: o = pass_k(q, k, ... pass_1(q, k, v)) in the given order. q, k, v, o: [B, h, n, d];
+ * workspace: >= squad_kpass_fwd_workspace_bytes, kept for the backward. */
+SQUAD_API squad_status_t squad_kpass_fwd(const squad_kpass_params_t* p, const void* q, const void* k,
+                                         const void* v, void* o, void* workspace, squad_stream_t stream);
+
+/* Bytes of backward workspace: a control block, fp32 dQ and dK shares, per-row softmax-Jacobian terms
+ * and up to two intermediate value gradients (input dtype). 0 for invalid parameters. */
+SQUAD_API size_t squad_kpass_bwd_workspace_bytes(const squad_kpass_params_t* p);
+
+/* Backward (the chain rule through the k passes, last executed first): gradients of <dout, o> with
+ * respect to q, k, v; dq and dk sum the k passes' shares (in fp32, rounded once). Inputs as given to /
+ * left by squad_kpass_fwd; dq, dk, dv [B, h, n, d] are overwritten. */
+SQUAD_API squad_status_t squad_kpass_bwd(const squad_kpass_params_t* p, const void* q, const void* k,
+                                         const void* v, const void* o, const void* dout,
+                                         const void* fwd_workspace, void* dq, void* dk, void* dv,
+                                         void* bwd_workspace, squad_stream_t stream);
+
+/* Device status recorded by the last squad_kpass_fwd or squad_kpass_bwd on `workspace`: SQUAD_OK or
+ * SQUAD_ERR_TIMEOUT. Synchronises `stream` first. */
+SQUAD_API squad_status_t squad_kpass_status(const squad_kpass_params_t* p, const void* workspace,
+                                            squad_stream_t stream);
+
+/* FLOPs of one k-pass forward: 4 B h d n (m_1 + ... + m_k); 0 for invalid parameters. */
+SQUAD_API double squad_kpass_flops(const squad_kpass_params_t* p);
 
 /* Static string for a status code (never NULL). */
 SQUAD_API const char* squad_status_string(squad_status_t s);

@@ -8,6 +8,7 @@ from .api import (  # noqa: F401
     SquadError,
     full_attn_flops,
     full_attn_fwd,
+    make_kpass_params,
     make_params,
     squad_attn_bwd,
     squad_attn_bwd_workspace_bytes,
@@ -17,4 +18,9 @@ from .api import (  # noqa: F401
     squad_attn_fwd_noalloc,
     squad_attn_fwd_status,
     squad_attn_fwd_workspace_bytes,
+    squad_kpass_bwd,
+    squad_kpass_flops,
+    squad_kpass_fwd,
+    squad_kpass_pass_params,
+    squad_kpass_status,
 )

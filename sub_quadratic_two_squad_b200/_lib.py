@@ -23,7 +23,20 @@ class SquadParams(ctypes.Structure):
                 ("order", ctypes.c_int), ("dtype", ctypes.c_int), ("scale", ctypes.c_float)]
 
 
+SQUAD_KPASS_MAX_LEVELS = 4
+SQUAD_KPASS_FORWARD, SQUAD_KPASS_REVERSE = 0, 1
+
+
+class SquadKpassParams(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("h", ctypes.c_int), ("d", ctypes.c_int),
+                ("T", ctypes.c_int), ("H", ctypes.c_int), ("W", ctypes.c_int),
+                ("k", ctypes.c_int),
+                ("level_h", ctypes.c_int * SQUAD_KPASS_MAX_LEVELS), ("level_w", ctypes.c_int * SQUAD_KPASS_MAX_LEVELS),
+                ("order", ctypes.c_int), ("dtype", ctypes.c_int), ("scale", ctypes.c_float)]
+
+
 _PP = ctypes.POINTER(SquadParams)
+_KP = ctypes.POINTER(SquadKpassParams)
 SIGNATURES = {
     "squad_attn_fwd_workspace_bytes": (ctypes.c_size_t, [_PP]),
     "squad_attn_fwd": (ctypes.c_int, [_PP, _VP, _VP, _VP, _VP, _VP, _VP]),
@@ -37,6 +50,13 @@ SIGNATURES = {
                                           ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]),
     "full_attn_flops": (ctypes.c_double, [_PP]),
     "squad_wait_selftest": (ctypes.c_int, [_VP, ctypes.c_ulonglong, _VP]),
+    "squad_kpass_pass_params": (ctypes.c_int, [_KP, ctypes.c_int, _PP]),
+    "squad_kpass_fwd_workspace_bytes": (ctypes.c_size_t, [_KP]),
+    "squad_kpass_fwd": (ctypes.c_int, [_KP, _VP, _VP, _VP, _VP, _VP, _VP]),
+    "squad_kpass_bwd_workspace_bytes": (ctypes.c_size_t, [_KP]),
+    "squad_kpass_bwd": (ctypes.c_int, [_KP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
+    "squad_kpass_status": (ctypes.c_int, [_KP, _VP, _VP]),
+    "squad_kpass_flops": (ctypes.c_double, [_KP]),
     "squad_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "squad_attn_abi_version": (ctypes.c_int, []),
 }

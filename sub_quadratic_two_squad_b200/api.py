@@ -110,11 +110,15 @@ def squad_attn_bwd(q, k, v, o, dout, fwd_workspace, grid, window, order="local_t
     prm = _params_for(q, grid, window, order, scale)
     lib = _lib.load()
     nbytes = lib.squad_attn_bwd_workspace_bytes(ctypes.byref(prm))
+    if nbytes == 0:
+        raise SquadError(_lib.SQUAD_ERR_INVALID_ARG, "squad_attn_bwd_workspace_bytes")
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(q) if dk is None else dk
     dv = torch.empty_like(q) if dv is None else dv
     if workspace is None:
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    elif workspace.numel() * workspace.element_size() < nbytes:
+        raise ValueError(f"workspace needs {nbytes} bytes")
     st = lib.squad_attn_bwd(ctypes.byref(prm), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(fwd_workspace),
                             _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace), _stream(stream))
     if st != _lib.SQUAD_OK:
@@ -152,6 +156,92 @@ def squad_window_solve(grid):
 
 def full_attn_flops(B, h, d, grid) -> float:
     return float(_lib.load().full_attn_flops(ctypes.byref(make_params(B, h, d, grid))))
+
+
+KPASS_ORDERS = {"forward": _lib.SQUAD_KPASS_FORWARD, "reverse": _lib.SQUAD_KPASS_REVERSE}
+
+
+def make_kpass_params(B, h, d, grid, levels, order="forward", dtype=torch.bfloat16, scale=None):
+    """squad_kpass_params_t for k = len(levels) nested-window passes; levels = [(h_1, w_1), ...]."""
+    T, H, W = grid
+    levels = [(int(a), int(b)) for a, b in levels]
+    m = _lib.SQUAD_KPASS_MAX_LEVELS
+    if not 1 <= len(levels) <= m:
+        raise ValueError(f"1 to {m} levels")
+    pad = [0] * (m - len(levels))
+    lh = (ctypes.c_int * m)(*([a for a, _ in levels] + pad))
+    lw = (ctypes.c_int * m)(*([b for _, b in levels] + pad))
+    o = KPASS_ORDERS[order] if isinstance(order, str) else int(order)
+    dt = _DTYPES[dtype] if isinstance(dtype, torch.dtype) else int(dtype)
+    return _lib.SquadKpassParams(B, h, d, T, H, W, len(levels), lh, lw, o, dt, 0.0 if scale is None else float(scale))
+
+
+def _kpass_params_for(q, grid, levels, order, scale):
+    B, h, n, d = q.shape
+    if n != grid[0] * grid[1] * grid[2]:
+        raise ValueError(f"n = {n} but T*H*W = {grid[0] * grid[1] * grid[2]}")
+    return make_kpass_params(B, h, d, grid, levels, order, q.dtype, scale)
+
+
+def squad_kpass_pass_params(params, level):
+    """The single-pass problem (SquadParams) that `level` (0-based) of a k-pass call runs."""
+    out = _lib.SquadParams()
+    st = _lib.load().squad_kpass_pass_params(ctypes.byref(params), int(level), ctypes.byref(out))
+    if st != _lib.SQUAD_OK:
+        raise SquadError(st, "squad_kpass_pass_params")
+    return out
+
+
+def squad_kpass_fwd(q, k, v, grid, levels, order="forward", scale=None, out=None, workspace=None, stream=None):
+    """k nested-window passes composed. Returns (out, workspace); keep the workspace for the backward."""
+    _check_qkv(q, k, v)
+    prm = _kpass_params_for(q, grid, levels, order, scale)
+    lib = _lib.load()
+    nbytes = lib.squad_kpass_fwd_workspace_bytes(ctypes.byref(prm))
+    if nbytes == 0:
+        raise SquadError(_lib.SQUAD_ERR_INVALID_ARG, "squad_kpass_fwd_workspace_bytes")
+    out = torch.empty_like(q) if out is None else out
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    elif workspace.numel() * workspace.element_size() < nbytes:
+        raise ValueError(f"workspace needs {nbytes} bytes")
+    st = lib.squad_kpass_fwd(ctypes.byref(prm), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(workspace), _stream(stream))
+    if st != _lib.SQUAD_OK:
+        raise SquadError(st, "squad_kpass_fwd")
+    return out, workspace
+
+
+def squad_kpass_bwd(q, k, v, o, dout, fwd_workspace, grid, levels, order="forward", scale=None, dq=None, dk=None,
+                    dv=None, workspace=None, stream=None):
+    """Gradients (dq, dk, dv) of <dout, o> for squad_kpass_fwd; `fwd_workspace` as it left it."""
+    _check_qkv(q, k, v, o, dout)
+    prm = _kpass_params_for(q, grid, levels, order, scale)
+    lib = _lib.load()
+    nbytes = lib.squad_kpass_bwd_workspace_bytes(ctypes.byref(prm))
+    if nbytes == 0:
+        raise SquadError(_lib.SQUAD_ERR_INVALID_ARG, "squad_kpass_bwd_workspace_bytes")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    elif workspace.numel() * workspace.element_size() < nbytes:
+        raise ValueError(f"workspace needs {nbytes} bytes")
+    st = lib.squad_kpass_bwd(ctypes.byref(prm), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(fwd_workspace),
+                             _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace), _stream(stream))
+    if st != _lib.SQUAD_OK:
+        raise SquadError(st, "squad_kpass_bwd")
+    return dq, dk, dv
+
+
+def squad_kpass_status(workspace, q, grid, levels, order="forward", scale=None, stream=None) -> int:
+    """Device status of the last k-pass call on `workspace` (synchronises the stream): 0 ok, 4 timeout."""
+    prm = _kpass_params_for(q, grid, levels, order, scale)
+    return int(_lib.load().squad_kpass_status(ctypes.byref(prm), _ptr(workspace), _stream(stream)))
+
+
+def squad_kpass_flops(B, h, d, grid, levels) -> float:
+    return float(_lib.load().squad_kpass_flops(ctypes.byref(make_kpass_params(B, h, d, grid, levels))))
 
 
 class HostRunner:

@@ -684,3 +684,324 @@ squad_status_t full_attn_fwd(const squad_params_t* p, const void* q, const void*
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------------------------------
+// k composed passes over nested windows. Each pass is one single-pass problem on a reinterpretation
+// of the caller's contiguous [B, h, n, d] buffers: a token's linear row (b h n + token) is the same in
+// every view, so outputs, log-sum-exps and the fp32 dQ/dK shares of all passes line up.
+// ------------------------------------------------------------------------------------------------
+
+namespace {
+
+constexpr size_t kKpassCtrlBytes = 256;   // word 0 the status, words 1..k the passes' work counters
+
+struct KpassPlan {
+  int k;
+  squad_params_t sub[SQUAD_KPASS_MAX_LEVELS];   // the single-pass problem of each level
+  Grid g[SQUAD_KPASS_MAX_LEVELS];
+  int kind[SQUAD_KPASS_MAX_LEVELS];
+  int exec[SQUAD_KPASS_MAX_LEVELS];             // level of each executed pass, in execution order
+  float scale;
+  size_t eb;                                    // element bytes of the input dtype
+  size_t bhn;                                   // B * h * n rows
+};
+
+// Level 0: the windows of h_1 x w_1 tokens over all frames (a local pass). Level p >= 1: with
+// hb, wb the products of the levels below and gy, gx the number of level-p blocks along H and W, the
+// rows of one (b, head, frame, block row) form a grid (1, hb h_p gx, wb w_p) whose window
+// (1, hb gx, wb) has exactly h_p x w_p windows; its slots are the level-p sequences (a global pass).
+void kpass_level_params(const squad_kpass_params_t* p, int level, squad_params_t* s) {
+  std::memset(s, 0, sizeof(*s));
+  s->d = p->d;
+  s->dtype = p->dtype;
+  s->scale = p->scale;
+  if (level == 0) {
+    s->B = p->B;
+    s->h = p->h;
+    s->T = p->T;
+    s->H = p->H;
+    s->W = p->W;
+    s->tw = p->T;
+    s->hw = p->level_h[0];
+    s->ww = p->level_w[0];
+    s->order = SQUAD_LOCAL_ONLY;
+    return;
+  }
+  long long hb = 1, wb = 1;
+  for (int q = 0; q < level; ++q) {
+    hb *= p->level_h[q];
+    wb *= p->level_w[q];
+  }
+  const long long hu = hb * p->level_h[level], wu = wb * p->level_w[level];
+  const long long gy = p->H / hu, gx = p->W / wu;
+  s->B = static_cast<int>(static_cast<long long>(p->B) * p->h * p->T * gy);
+  s->h = 1;
+  s->T = 1;
+  s->H = static_cast<int>(hu * gx);
+  s->W = static_cast<int>(wu);
+  s->tw = 1;
+  s->hw = static_cast<int>(hb * gx);
+  s->ww = static_cast<int>(wb);
+  s->order = SQUAD_GLOBAL_ONLY;
+}
+
+squad_status_t kpass_check(const squad_kpass_params_t* p) {
+  if (p == nullptr) return SQUAD_ERR_INVALID_ARG;
+  if (p->k < 1 || p->k > SQUAD_KPASS_MAX_LEVELS) return SQUAD_ERR_INVALID_ARG;
+  if (p->order != SQUAD_KPASS_FORWARD && p->order != SQUAD_KPASS_REVERSE) return SQUAD_ERR_INVALID_ARG;
+  if (p->B < 1 || p->h < 1 || p->T < 1 || p->H < 1 || p->W < 1) return SQUAD_ERR_INVALID_ARG;
+  long long ph = 1, pw = 1;
+  for (int l = 0; l < p->k; ++l) {
+    if (p->level_h[l] < 1 || p->level_w[l] < 1) return SQUAD_ERR_INVALID_ARG;
+    ph *= p->level_h[l];
+    pw *= p->level_w[l];
+    if (ph > p->H || pw > p->W) return SQUAD_ERR_INVALID_ARG;
+  }
+  if (ph != p->H || pw != p->W) return SQUAD_ERR_INVALID_ARG;   // the levels factor the grid exactly
+  if (static_cast<long long>(p->B) * p->h * p->T * p->H > INT32_MAX) return SQUAD_ERR_UNSUPPORTED;
+  // every pass attends over at least two tokens
+  if (static_cast<long long>(p->T) * p->level_h[0] * p->level_w[0] < 2) return SQUAD_ERR_UNSUPPORTED;
+  for (int l = 1; l < p->k; ++l)
+    if (static_cast<long long>(p->level_h[l]) * p->level_w[l] < 2) return SQUAD_ERR_UNSUPPORTED;
+  return SQUAD_OK;
+}
+
+squad_status_t kpass_plan(const squad_kpass_params_t* p, KpassPlan* pl) {
+  squad_status_t st = kpass_check(p);
+  if (st != SQUAD_OK) return st;
+  pl->k = p->k;
+  for (int l = 0; l < p->k; ++l) {
+    kpass_level_params(p, l, &pl->sub[l]);
+    PadDims pd;
+    st = validate(&pl->sub[l], true, &pl->g[l], &pl->scale, &pd);
+    if (st != SQUAD_OK) return st;
+    if (pd.padded) return SQUAD_ERR_INVALID_ARG;   // unreachable: each view's window divides its grid
+    pl->kind[l] = l == 0 ? kLocal : kGlobal;
+  }
+  for (int e = 0; e < p->k; ++e) pl->exec[e] = p->order == SQUAD_KPASS_FORWARD ? e : p->k - 1 - e;
+  pl->eb = elem_bytes(&pl->sub[0]);
+  pl->bhn = static_cast<size_t>(p->B) * p->h * p->T * p->H * p->W;
+  return SQUAD_OK;
+}
+
+struct KpassFwdWs {
+  uint32_t* ctrl;
+  void* inter[SQUAD_KPASS_MAX_LEVELS];   // outputs of executed passes 0 .. k-2 (input dtype)
+  float* lse[SQUAD_KPASS_MAX_LEVELS];    // log-sum-exp of executed pass e
+};
+
+size_t kpass_fwd_bytes(const KpassPlan& pl) {
+  const size_t t = align256(pl.bhn * pl.sub[0].d * pl.eb), l = align256(pl.bhn * 4);
+  return kKpassCtrlBytes + static_cast<size_t>(pl.k - 1) * t + static_cast<size_t>(pl.k) * l;
+}
+
+KpassFwdWs carve_kpass_fwd(void* ws, const KpassPlan& pl) {
+  const size_t t = align256(pl.bhn * pl.sub[0].d * pl.eb), l = align256(pl.bhn * 4);
+  uint8_t* b = static_cast<uint8_t*>(ws);
+  KpassFwdWs w{};
+  w.ctrl = reinterpret_cast<uint32_t*>(b);
+  b += kKpassCtrlBytes;
+  for (int e = 0; e + 1 < pl.k; ++e, b += t) w.inter[e] = b;
+  for (int e = 0; e < pl.k; ++e, b += l) w.lse[e] = reinterpret_cast<float*>(b);
+  return w;
+}
+
+struct KpassBwdWs {
+  uint32_t* ctrl;
+  float* dq_acc;    // fp32 dQ and dK shares [B, h, n, d]
+  float* dk_acc;
+  float* drow;      // [B, h, n] per-row softmax-Jacobian terms (CUDA-core kernels)
+  void* gbuf[2];    // value gradients passed between consecutive passes (input dtype)
+};
+
+size_t kpass_bwd_bytes(const KpassPlan& pl) {
+  const size_t d = static_cast<size_t>(pl.sub[0].d);
+  const size_t t = align256(pl.bhn * d * pl.eb), f = align256(pl.bhn * d * 4), l = align256(pl.bhn * 4);
+  const size_t ng = pl.k - 1 < 2 ? static_cast<size_t>(pl.k - 1) : 2;
+  return kKpassCtrlBytes + 2 * f + l + ng * t;
+}
+
+KpassBwdWs carve_kpass_bwd(void* ws, const KpassPlan& pl) {
+  const size_t d = static_cast<size_t>(pl.sub[0].d);
+  const size_t t = align256(pl.bhn * d * pl.eb), f = align256(pl.bhn * d * 4), l = align256(pl.bhn * 4);
+  uint8_t* b = static_cast<uint8_t*>(ws);
+  KpassBwdWs w{};
+  w.ctrl = reinterpret_cast<uint32_t*>(b);
+  b += kKpassCtrlBytes;
+  w.dq_acc = reinterpret_cast<float*>(b);
+  b += f;
+  w.dk_acc = reinterpret_cast<float*>(b);
+  b += f;
+  w.drow = reinterpret_cast<float*>(b);
+  b += l;
+  w.gbuf[0] = pl.k > 1 ? b : nullptr;
+  w.gbuf[1] = pl.k > 2 ? b + t : nullptr;
+  return w;
+}
+
+// One pass's backward inside a chain of passes. accumulate: add the fp32 dQ/dK shares already in the
+// accumulators; final_out: write dq, dk (input dtype) instead of the accumulators. dv_out receives the
+// gradient of this pass's values in the input dtype.
+squad_status_t bwd_one_pass(const squad_params_t* sp, const Grid& g, int kind, float scale, const void* q,
+                            const void* k, const void* values, const void* dout, const float* lse, uint32_t* status,
+                            float* dq_acc, float* dk_acc, float* drow, void* dq, void* dk, void* dv_out,
+                            bool accumulate, bool final_out, cudaStream_t stream) {
+  const bool bf16 = sp->dtype == SQUAD_BF16;
+  if (bf16) {
+    BwdTcArgs b;
+    std::memset(&b, 0, sizeof(b));
+    b.g = g;
+    b.p = make_geom(g, kind, 256);
+    if (short_eligible(sp, g, b.p) && bwd_tc_plan(b)) {
+      b.variant = kind == kGlobal ? kSlotBoxVariant : 0;
+      if (!encode_pass_map(&b.tm_q, q, g, b.p, b.variant) || !encode_pass_map(&b.tm_k, k, g, b.p, b.variant) ||
+          !encode_pass_map(&b.tm_v, values, g, b.p, b.variant) || !encode_pass_map(&b.tm_do, dout, g, b.p, b.variant))
+        return SQUAD_ERR_CUDA;
+      b.lse = lse;
+      b.dq_acc = dq_acc;
+      b.dk_acc = dk_acc;
+      b.dq_out = static_cast<__nv_bfloat16*>(dq);
+      b.dk_out = static_cast<__nv_bfloat16*>(dk);
+      b.dv_out = static_cast<__nv_bfloat16*>(dv_out);
+      b.final_out = final_out ? 1 : 0;
+      b.accumulate = accumulate ? 1 : 0;
+      b.scale = scale;
+      b.scale_log2 = scale * 1.4426950408889634f;
+      b.status = status;
+      b.timeout_ns = kWaitTimeoutNs;
+      return launch_bwd_tc(b, stream) == cudaSuccess ? SQUAD_OK : SQUAD_ERR_CUDA;
+    }
+  }
+  SimtBwdArgs a{};
+  a.q = q;
+  a.k = k;
+  a.v = values;
+  a.dout = dout;
+  a.lse = lse;
+  a.Drow = drow;
+  a.dq_acc = dq_acc;
+  a.dk_acc = dk_acc;
+  a.dq_out = dq;
+  a.dk_out = dk;
+  a.dv_out = dv_out;
+  a.g = g;
+  a.p = make_geom(g, kind);
+  a.scale = scale;
+  a.in_bf16 = bf16;
+  a.v_bf16 = bf16;
+  a.dout_bf16 = bf16;
+  a.grad_bf16 = bf16;
+  a.dv_bf16 = bf16;
+  a.accumulate = accumulate ? 1 : 0;
+  a.final_out = final_out ? 1 : 0;
+  return launch_simt_bwd(a, stream) == cudaSuccess ? SQUAD_OK : SQUAD_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+squad_status_t squad_kpass_pass_params(const squad_kpass_params_t* p, int level, squad_params_t* out) {
+  if (out == nullptr) return SQUAD_ERR_INVALID_ARG;
+  const squad_status_t st = kpass_check(p);
+  if (st != SQUAD_OK) return st;
+  if (level < 0 || level >= p->k) return SQUAD_ERR_INVALID_ARG;
+  squad_params_t s;
+  kpass_level_params(p, level, &s);
+  Grid g;
+  float sc;
+  PadDims pd;
+  const squad_status_t vs = validate(&s, true, &g, &sc, &pd);
+  if (vs != SQUAD_OK) return vs;
+  *out = s;
+  return SQUAD_OK;
+}
+
+size_t squad_kpass_fwd_workspace_bytes(const squad_kpass_params_t* p) {
+  KpassPlan pl;
+  if (kpass_plan(p, &pl) != SQUAD_OK) return 0;
+  return kpass_fwd_bytes(pl);
+}
+
+size_t squad_kpass_bwd_workspace_bytes(const squad_kpass_params_t* p) {
+  KpassPlan pl;
+  if (kpass_plan(p, &pl) != SQUAD_OK) return 0;
+  return kpass_bwd_bytes(pl);
+}
+
+double squad_kpass_flops(const squad_kpass_params_t* p) {
+  KpassPlan pl;
+  if (kpass_plan(p, &pl) != SQUAD_OK) return 0.0;
+  double total = 0.0;
+  for (int l = 0; l < pl.k; ++l) total += squad_attn_flops(&pl.sub[l]);
+  return total;
+}
+
+squad_status_t squad_kpass_fwd(const squad_kpass_params_t* p, const void* q, const void* k, const void* v, void* o,
+                               void* workspace, squad_stream_t stream_) {
+  KpassPlan pl;
+  const squad_status_t st = kpass_plan(p, &pl);
+  if (st != SQUAD_OK) return st;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(workspace, 256))
+    return SQUAD_ERR_INVALID_ARG;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  const KpassFwdWs ws = carve_kpass_fwd(workspace, pl);
+  if (cudaMemsetAsync(ws.ctrl, 0, kKpassCtrlBytes, stream) != cudaSuccess) return SQUAD_ERR_CUDA;
+  const bool bf16 = p->dtype == SQUAD_BF16;
+  const void* x = v;
+  for (int e = 0; e < pl.k; ++e) {
+    const int l = pl.exec[e];
+    void* out = e + 1 == pl.k ? o : ws.inter[e];
+    const squad_status_t ps = run_pass(&pl.sub[l], pl.g[l], pl.kind[l], pl.scale, q, k, x, bf16, out, ws.lse[e],
+                                       ws.ctrl, ws.ctrl + 1 + e, stream);
+    if (ps != SQUAD_OK) return ps;
+    x = out;
+  }
+  return SQUAD_OK;
+}
+
+squad_status_t squad_kpass_bwd(const squad_kpass_params_t* p, const void* q, const void* k, const void* v,
+                               const void* o, const void* dout, const void* fwd_workspace, void* dq, void* dk,
+                               void* dv, void* bwd_workspace, squad_stream_t stream_) {
+  (void)o;   // each pass forms its softmax-Jacobian term from the recomputed P and dP
+  KpassPlan pl;
+  const squad_status_t st = kpass_plan(p, &pl);
+  if (st != SQUAD_OK) return st;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(dout, 16) ||
+      !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(fwd_workspace, 256) ||
+      !aligned(bwd_workspace, 256))
+    return SQUAD_ERR_INVALID_ARG;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  const KpassFwdWs fw = carve_kpass_fwd(const_cast<void*>(fwd_workspace), pl);
+  const KpassBwdWs bw = carve_kpass_bwd(bwd_workspace, pl);
+  if (cudaMemsetAsync(bw.ctrl, 0, kKpassCtrlBytes, stream) != cudaSuccess) return SQUAD_ERR_CUDA;
+  // Last executed pass first; executed pass e's values are v (e = 0) or pass e-1's output, and the
+  // gradient of its values is the upstream gradient of pass e-1 (ping-pong buffers) or dv (e = 0).
+  const void* g_in = dout;
+  for (int e = pl.k - 1; e >= 0; --e) {
+    const int l = pl.exec[e];
+    const void* values = e == 0 ? v : fw.inter[e - 1];
+    void* g_out = e == 0 ? dv : bw.gbuf[e % 2];
+    const squad_status_t ps = bwd_one_pass(&pl.sub[l], pl.g[l], pl.kind[l], pl.scale, q, k, values, g_in, fw.lse[e],
+                                           bw.ctrl, bw.dq_acc, bw.dk_acc, bw.drow, dq, dk, g_out,
+                                           /*accumulate=*/e + 1 < pl.k, /*final_out=*/e == 0, stream);
+    if (ps != SQUAD_OK) return ps;
+    g_in = g_out;
+  }
+  return SQUAD_OK;
+}
+
+squad_status_t squad_kpass_status(const squad_kpass_params_t* p, const void* workspace, squad_stream_t stream_) {
+  KpassPlan pl;
+  const squad_status_t st = kpass_plan(p, &pl);
+  if (st != SQUAD_OK) return st;
+  if (!aligned(workspace, 256)) return SQUAD_ERR_INVALID_ARG;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  uint32_t word = 0;
+  if (cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+    return SQUAD_ERR_CUDA;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return SQUAD_ERR_CUDA;
+  return word == 0 ? SQUAD_OK : SQUAD_ERR_TIMEOUT;
+}
+
+}  // extern "C"

@@ -16,14 +16,15 @@ struct BwdTcArgs {
   PassGeom p;                 // one chunk per sequence (make_geom(..., 256))
   int variant;                // slot-box encoding (GLOBAL pass)
   const float* lse;           // [B, h, n] natural-log LSE of this pass's forward
-  float* dq_acc;              // [B, h, n, d] fp32 share of dQ (written, or read and completed when final)
+  float* dq_acc;              // [B, h, n, d] fp32 share of dQ: written, added to (accumulate), or read
+                              // and completed (final_out with accumulate)
   float* dk_acc;              // [B, h, n, d] fp32 share of dK (likewise)
   __nv_bfloat16* dq_out;      // final dQ (final_out only)
   __nv_bfloat16* dk_out;      // final dK (final_out only)
   __nv_bfloat16* dv_out;      // gradient of this pass's values
   float scale, scale_log2;
   int final_out;              // write dq_out / dk_out (bf16) instead of the fp32 shares
-  int accumulate;             // with final_out: add the other pass's fp32 share first
+  int accumulate;             // add the fp32 shares already in dq_acc / dk_acc (earlier passes') first
   uint32_t panel_bytes;       // rows (rounded to 8) x 128 bytes
   uint32_t guard_bytes, smem_bytes;
   uint32_t* status;           // device status word (0 = ok, 4 = a wait timed out)

@@ -298,7 +298,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
         if (a.final_out)
           write_row(t_row + N, tok >= 0, a.scale, a.accumulate ? a.dq_acc + ro : nullptr, a.dq_out + ro, nullptr);
         else
-          write_row(t_row + N, tok >= 0, a.scale, nullptr, nullptr, a.dq_acc + ro);
+          write_row(t_row + N, tok >= 0, a.scale, a.accumulate ? a.dq_acc + ro : nullptr, nullptr, a.dq_acc + ro);
       }
       tc_fence_before();
       mbar_arrive(&bars->o_free);
@@ -350,7 +350,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
         if (a.final_out)
           write_row(t_row + 384, tok >= 0, a.scale, a.accumulate ? a.dk_acc + ro : nullptr, a.dk_out + ro, nullptr);
         else
-          write_row(t_row + 384, tok >= 0, a.scale, nullptr, nullptr, a.dk_acc + ro);
+          write_row(t_row + 384, tok >= 0, a.scale, a.accumulate ? a.dk_acc + ro : nullptr, nullptr, a.dk_acc + ro);
       }
       tc_fence_before();
       mbar_arrive(&bars->o_free);

@@ -1,7 +1,6 @@
 """The kernels' index arithmetic, checked on the CPU (no GPU): a host build of csrc/geometry.cuh
 walks every TMA chunk box as the hardware traverses it and must reproduce the oracle's window and
 slot tables exactly (rows of the window table = local sequences, its columns = global sequences)."""
-import os
 import subprocess
 
 import numpy as np
@@ -9,15 +8,10 @@ import pytest
 
 from oracle import squad_oracle as orc
 
-ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-
 
 @pytest.fixture(scope="module")
-def checker(tmp_path_factory):
-    exe = str(tmp_path_factory.mktemp("geom") / "geometry_check")
-    subprocess.run(["nvcc", "-std=c++17", "-O1", "-x", "cu", "-I", os.path.join(ROOT, "sub_quadratic_two_squad_b200", "csrc"),
-                    os.path.join(ROOT, "tests", "geometry_check.cu"), "-o", exe], check=True)
-    return exe
+def checker(geometry_checker):
+    return geometry_checker
 
 
 CASES = [
