@@ -14,6 +14,7 @@
 
 #include "squad_attn.h"
 #include "geometry.cuh"
+#include "kpass_plan.h"
 #include "bwd_pass.h"
 #include "pad.h"
 #include "short_pass.h"
@@ -700,71 +701,10 @@ struct KpassPlan {
   squad_params_t sub[SQUAD_KPASS_MAX_LEVELS];   // the single-pass problem of each level
   Grid g[SQUAD_KPASS_MAX_LEVELS];
   int kind[SQUAD_KPASS_MAX_LEVELS];
-  int exec[SQUAD_KPASS_MAX_LEVELS];             // level of each executed pass, in execution order
   float scale;
   size_t eb;                                    // element bytes of the input dtype
   size_t bhn;                                   // B * h * n rows
 };
-
-// Level 0: the windows of h_1 x w_1 tokens over all frames (a local pass). Level p >= 1: with
-// hb, wb the products of the levels below and gy, gx the number of level-p blocks along H and W, the
-// rows of one (b, head, frame, block row) form a grid (1, hb h_p gx, wb w_p) whose window
-// (1, hb gx, wb) has exactly h_p x w_p windows; its slots are the level-p sequences (a global pass).
-void kpass_level_params(const squad_kpass_params_t* p, int level, squad_params_t* s) {
-  std::memset(s, 0, sizeof(*s));
-  s->d = p->d;
-  s->dtype = p->dtype;
-  s->scale = p->scale;
-  if (level == 0) {
-    s->B = p->B;
-    s->h = p->h;
-    s->T = p->T;
-    s->H = p->H;
-    s->W = p->W;
-    s->tw = p->T;
-    s->hw = p->level_h[0];
-    s->ww = p->level_w[0];
-    s->order = SQUAD_LOCAL_ONLY;
-    return;
-  }
-  long long hb = 1, wb = 1;
-  for (int q = 0; q < level; ++q) {
-    hb *= p->level_h[q];
-    wb *= p->level_w[q];
-  }
-  const long long hu = hb * p->level_h[level], wu = wb * p->level_w[level];
-  const long long gy = p->H / hu, gx = p->W / wu;
-  s->B = static_cast<int>(static_cast<long long>(p->B) * p->h * p->T * gy);
-  s->h = 1;
-  s->T = 1;
-  s->H = static_cast<int>(hu * gx);
-  s->W = static_cast<int>(wu);
-  s->tw = 1;
-  s->hw = static_cast<int>(hb * gx);
-  s->ww = static_cast<int>(wb);
-  s->order = SQUAD_GLOBAL_ONLY;
-}
-
-squad_status_t kpass_check(const squad_kpass_params_t* p) {
-  if (p == nullptr) return SQUAD_ERR_INVALID_ARG;
-  if (p->k < 1 || p->k > SQUAD_KPASS_MAX_LEVELS) return SQUAD_ERR_INVALID_ARG;
-  if (p->order != SQUAD_KPASS_FORWARD && p->order != SQUAD_KPASS_REVERSE) return SQUAD_ERR_INVALID_ARG;
-  if (p->B < 1 || p->h < 1 || p->T < 1 || p->H < 1 || p->W < 1) return SQUAD_ERR_INVALID_ARG;
-  long long ph = 1, pw = 1;
-  for (int l = 0; l < p->k; ++l) {
-    if (p->level_h[l] < 1 || p->level_w[l] < 1) return SQUAD_ERR_INVALID_ARG;
-    ph *= p->level_h[l];
-    pw *= p->level_w[l];
-    if (ph > p->H || pw > p->W) return SQUAD_ERR_INVALID_ARG;
-  }
-  if (ph != p->H || pw != p->W) return SQUAD_ERR_INVALID_ARG;   // the levels factor the grid exactly
-  if (static_cast<long long>(p->B) * p->h * p->T * p->H > INT32_MAX) return SQUAD_ERR_UNSUPPORTED;
-  // every pass attends over at least two tokens
-  if (static_cast<long long>(p->T) * p->level_h[0] * p->level_w[0] < 2) return SQUAD_ERR_UNSUPPORTED;
-  for (int l = 1; l < p->k; ++l)
-    if (static_cast<long long>(p->level_h[l]) * p->level_w[l] < 2) return SQUAD_ERR_UNSUPPORTED;
-  return SQUAD_OK;
-}
 
 squad_status_t kpass_plan(const squad_kpass_params_t* p, KpassPlan* pl) {
   squad_status_t st = kpass_check(p);
@@ -778,7 +718,6 @@ squad_status_t kpass_plan(const squad_kpass_params_t* p, KpassPlan* pl) {
     if (pd.padded) return SQUAD_ERR_INVALID_ARG;   // unreachable: each view's window divides its grid
     pl->kind[l] = l == 0 ? kLocal : kGlobal;
   }
-  for (int e = 0; e < p->k; ++e) pl->exec[e] = p->order == SQUAD_KPASS_FORWARD ? e : p->k - 1 - e;
   pl->eb = elem_bytes(&pl->sub[0]);
   pl->bhn = static_cast<size_t>(p->B) * p->h * p->T * p->H * p->W;
   return SQUAD_OK;
@@ -792,7 +731,7 @@ struct KpassFwdWs {
 
 size_t kpass_fwd_bytes(const KpassPlan& pl) {
   const size_t t = align256(pl.bhn * pl.sub[0].d * pl.eb), l = align256(pl.bhn * 4);
-  return kKpassCtrlBytes + static_cast<size_t>(pl.k - 1) * t + static_cast<size_t>(pl.k) * l;
+  return kKpassCtrlBytes + static_cast<size_t>(kpass_n_inter(pl.k)) * t + static_cast<size_t>(pl.k) * l;
 }
 
 KpassFwdWs carve_kpass_fwd(void* ws, const KpassPlan& pl) {
@@ -801,7 +740,7 @@ KpassFwdWs carve_kpass_fwd(void* ws, const KpassPlan& pl) {
   KpassFwdWs w{};
   w.ctrl = reinterpret_cast<uint32_t*>(b);
   b += kKpassCtrlBytes;
-  for (int e = 0; e + 1 < pl.k; ++e, b += t) w.inter[e] = b;
+  for (int e = 0; e < kpass_n_inter(pl.k); ++e, b += t) w.inter[e] = b;
   for (int e = 0; e < pl.k; ++e, b += l) w.lse[e] = reinterpret_cast<float*>(b);
   return w;
 }
@@ -817,8 +756,7 @@ struct KpassBwdWs {
 size_t kpass_bwd_bytes(const KpassPlan& pl) {
   const size_t d = static_cast<size_t>(pl.sub[0].d);
   const size_t t = align256(pl.bhn * d * pl.eb), f = align256(pl.bhn * d * 4), l = align256(pl.bhn * 4);
-  const size_t ng = pl.k - 1 < 2 ? static_cast<size_t>(pl.k - 1) : 2;
-  return kKpassCtrlBytes + 2 * f + l + ng * t;
+  return kKpassCtrlBytes + 2 * f + l + static_cast<size_t>(kpass_n_gbuf(pl.k)) * t;
 }
 
 KpassBwdWs carve_kpass_bwd(void* ws, const KpassPlan& pl) {
@@ -834,8 +772,8 @@ KpassBwdWs carve_kpass_bwd(void* ws, const KpassPlan& pl) {
   b += f;
   w.drow = reinterpret_cast<float*>(b);
   b += l;
-  w.gbuf[0] = pl.k > 1 ? b : nullptr;
-  w.gbuf[1] = pl.k > 2 ? b + t : nullptr;
+  w.gbuf[0] = kpass_n_gbuf(pl.k) > 0 ? b : nullptr;
+  w.gbuf[1] = kpass_n_gbuf(pl.k) > 1 ? b + t : nullptr;
   return w;
 }
 
@@ -948,14 +886,14 @@ squad_status_t squad_kpass_fwd(const squad_kpass_params_t* p, const void* q, con
   const KpassFwdWs ws = carve_kpass_fwd(workspace, pl);
   if (cudaMemsetAsync(ws.ctrl, 0, kKpassCtrlBytes, stream) != cudaSuccess) return SQUAD_ERR_CUDA;
   const bool bf16 = p->dtype == SQUAD_BF16;
-  const void* x = v;
   for (int e = 0; e < pl.k; ++e) {
-    const int l = pl.exec[e];
-    void* out = e + 1 == pl.k ? o : ws.inter[e];
-    const squad_status_t ps = run_pass(&pl.sub[l], pl.g[l], pl.kind[l], pl.scale, q, k, x, bf16, out, ws.lse[e],
-                                       ws.ctrl, ws.ctrl + 1 + e, stream);
+    const KpassFwdStep st = kpass_fwd_step(p, e);
+    const int l = st.level;
+    const void* values = st.values == kBufV ? v : ws.inter[st.values];
+    void* out = st.out == kBufO ? o : ws.inter[st.out];
+    const squad_status_t ps = run_pass(&pl.sub[l], pl.g[l], pl.kind[l], pl.scale, q, k, values, bf16, out,
+                                       ws.lse[st.lse], ws.ctrl, ws.ctrl + st.work, stream);
     if (ps != SQUAD_OK) return ps;
-    x = out;
   }
   return SQUAD_OK;
 }
@@ -975,18 +913,17 @@ squad_status_t squad_kpass_bwd(const squad_kpass_params_t* p, const void* q, con
   const KpassFwdWs fw = carve_kpass_fwd(const_cast<void*>(fwd_workspace), pl);
   const KpassBwdWs bw = carve_kpass_bwd(bwd_workspace, pl);
   if (cudaMemsetAsync(bw.ctrl, 0, kKpassCtrlBytes, stream) != cudaSuccess) return SQUAD_ERR_CUDA;
-  // Last executed pass first; executed pass e's values are v (e = 0) or pass e-1's output, and the
-  // gradient of its values is the upstream gradient of pass e-1 (ping-pong buffers) or dv (e = 0).
-  const void* g_in = dout;
+  // Last executed pass first (the schedule of kpass_bwd_step).
   for (int e = pl.k - 1; e >= 0; --e) {
-    const int l = pl.exec[e];
-    const void* values = e == 0 ? v : fw.inter[e - 1];
-    void* g_out = e == 0 ? dv : bw.gbuf[e % 2];
-    const squad_status_t ps = bwd_one_pass(&pl.sub[l], pl.g[l], pl.kind[l], pl.scale, q, k, values, g_in, fw.lse[e],
-                                           bw.ctrl, bw.dq_acc, bw.dk_acc, bw.drow, dq, dk, g_out,
-                                           /*accumulate=*/e + 1 < pl.k, /*final_out=*/e == 0, stream);
+    const KpassBwdStep st = kpass_bwd_step(p, e);
+    const int l = st.level;
+    const void* values = st.values == kBufV ? v : fw.inter[st.values];
+    const void* g_in = st.g_in == kBufDout ? dout : bw.gbuf[st.g_in];
+    void* g_out = st.g_out == kBufDv ? dv : bw.gbuf[st.g_out];
+    const squad_status_t ps = bwd_one_pass(&pl.sub[l], pl.g[l], pl.kind[l], pl.scale, q, k, values, g_in,
+                                           fw.lse[st.lse], bw.ctrl, bw.dq_acc, bw.dk_acc, bw.drow, dq, dk, g_out,
+                                           st.accumulate, st.final_out, stream);
     if (ps != SQUAD_OK) return ps;
-    g_in = g_out;
   }
   return SQUAD_OK;
 }

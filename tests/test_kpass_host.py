@@ -2,6 +2,7 @@
 reproduces the oracle's nested-window definition when each reported single-pass problem is run by the
 oracle on the reshaped buffers; argument checks, workspace sizes and FLOP counts."""
 import ctypes
+import os
 import subprocess
 
 import numpy as np
@@ -196,3 +197,17 @@ def test_kernel_boxes_of_each_view_are_the_level_groups(lib, geometry_checker, g
         n_view = s.T * s.H * s.W
         ref = {frozenset(int(t) for t in g) for g in orc.level_groups(grid, levels, lv) if g.max() < n_view}
         assert got == ref
+
+
+def test_chain_schedule(tmp_path):
+    """A host build of csrc/kpass_plan.h: the forward and backward schedules the library executes pass
+    values, log-sum-exps and value gradients along the chain (tests/kpass_check.cpp)."""
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    exe = str(tmp_path / "kpass_check")
+    subprocess.run(["g++", "-std=c++17", "-O1", "-I", os.path.join(root, "include"),
+                    "-I", os.path.join(root, "sub_quadratic_two_squad_b200", "csrc"),
+                    os.path.join(root, "tests", "kpass_check.cpp"), "-o", exe], check=True)
+    r = subprocess.run([exe], capture_output=True, text=True)
+    assert r.returncode == 0 and r.stdout.strip().endswith("ok"), r.stdout[-2000:]
+    bwd3 = [l for l in r.stdout.splitlines() if l.startswith("bwd k=3 order=0")]
+    assert [l.split()[6:8] for l in bwd3] == [["g_in=-3", "g_out=0"], ["g_in=0", "g_out=1"], ["g_in=1", "g_out=-4"]]
