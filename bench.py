@@ -375,6 +375,14 @@ SWEEP = [
     ("Wan-2.1-14B block (training step)", 1, 40, 128, (21, 22, 40), (21, 2, 4), ("local_then_global",), False, True),
 ]
 
+# k composed passes over nested windows on the Wan-2.2-5B grid: (name, B, h, d, grid, levels, orders, with_bwd).
+KPASS_SWEEP = [
+    ("Wan-2.2-5B block, k = 3 (levels 1x1, 11x2, 2x20: 21 + 22 + 40 tokens)", 1, 24, 128, (21, 22, 40),
+     [(1, 1), (11, 2), (2, 20)], ("forward", "reverse"), True),
+    ("Wan-2.2-5B block, k = 3 (levels 2x4, 11x2, 1x5: 168 + 22 + 5 tokens)", 1, 24, 128, (21, 22, 40),
+     [(2, 4), (11, 2), (1, 5)], ("forward",), False),
+]
+
 
 def sweep(reps=30, only=None, n_sets=3):
     """Forward (and backward, full attention) device times for every block shape, N(0,1) inputs drawn on
@@ -436,6 +444,39 @@ def sweep(reps=30, only=None, n_sets=3):
             print(json.dumps({"sweep": name, "order": "full_attn_fwd", "n": n, "ms_per_block": fms,
                               "tflops": nf / (fms * 1e-3) / 1e12, "tensor_frac": nf / (fms * 1e-3) / 1e12 / tf_peak}),
                   flush=True)
+        del sets, outs
+        torch.cuda.empty_cache()
+
+    from sub_quadratic_two_squad_b200 import squad_kpass_bwd, squad_kpass_flops, squad_kpass_fwd
+
+    for name, B, h, d, grid, levels, orders, with_bwd in KPASS_SWEEP:
+        if only is not None and only not in name:
+            continue
+        w = dict(B=B, h=h, d=d, grid=grid, window=(grid[0], 1, 1))
+        n = n_tokens(w)
+        ns = n_sets
+        sets = [tuple(torch.randn(B, h, n, d, device=dev, dtype=torch.bfloat16) for _ in range(3)) for _ in range(ns)]
+        outs = [torch.empty_like(x[0]) for x in sets]
+        f = squad_kpass_flops(B, h, d, grid, levels)
+        for order in orders:
+            wss = [squad_kpass_fwd(*sets[i], grid, levels, order)[1] for i in range(ns)]
+            ms = timed(lambda i: squad_kpass_fwd(*sets[i % ns], grid, levels, order, out=outs[i % ns],
+                                                 workspace=wss[i % ns]), reps)
+            t_roof = max(f / (tf_peak * 1e12), alg_bytes(w) / (hbm * 1e9)) * 1e3
+            line = {"sweep": name, "order": order, "n": n, "levels": ["x".join(map(str, l)) for l in levels],
+                    "ms_per_block": ms, "tflops": f / (ms * 1e-3) / 1e12, "roofline_ms": t_roof,
+                    "roofline_frac": t_roof / ms, "hbm_gbs_algorithmic": alg_bytes(w) / (ms * 1e-3) / 1e9,
+                    "peaks": peak_kind}
+            if with_bwd and order == "forward":
+                dout = torch.randn(B, h, n, d, device=dev, dtype=torch.bfloat16)
+                q, k, v = sets[0]
+                o, ws = squad_kpass_fwd(q, k, v, grid, levels, order)
+                g = squad_kpass_bwd(q, k, v, o, dout, ws, grid, levels, order)
+                bms = timed(lambda i: squad_kpass_bwd(q, k, v, o, dout, ws, grid, levels, order, dq=g[0], dk=g[1],
+                                                      dv=g[2]), 10)
+                line["backward"] = {"ms_per_block": bms, "tflops_algorithmic": 2 * f / (bms * 1e-3) / 1e12}
+            print(json.dumps(line), flush=True)
+            del wss
         del sets, outs
         torch.cuda.empty_cache()
 
