@@ -158,3 +158,28 @@ def test_workspace_sizes(lib):
     assert fwd >= 24 * n * 128 * 2 + 2 * 24 * n * 4
     bwd = lib.squad_attn_bwd_workspace_bytes(ctypes.byref(prm))
     assert bwd >= 3 * 24 * n * 128 * 4 + 24 * n * 4
+
+
+def test_size_limits(lib):
+    """n = T H W up to 2^30 tokens and B h n below 2^31 rows are accepted (workspace sizes computed in
+    64 bits); one past either limit is refused as unsupported before any launch."""
+    # n = 2^30 exactly: grid (1, 2^15, 2^15), one head
+    prm = make_params(1, 1, 128, (1, 1 << 15, 1 << 15), (1, 2, 4))
+    fwd = lib.squad_attn_fwd_workspace_bytes(ctypes.byref(prm))
+    assert fwd >= (1 << 30) * 128 * 2 + 2 * (1 << 30) * 4          # O1 (bf16) + two LSEs, no 32-bit wrap
+    assert lib.squad_attn_bwd_workspace_bytes(ctypes.byref(prm)) >= 3 * (1 << 30) * 128 * 4
+    # n = 2^30 + one row of tokens: refused
+    prm = make_params(1, 1, 128, (1, (1 << 15) + 1, 1 << 15), (1, 1, 4))
+    assert lib.squad_attn_fwd_workspace_bytes(ctypes.byref(prm)) == 0
+    assert _fwd(lib, prm) == _lib.SQUAD_ERR_UNSUPPORTED
+    # h = 2 heads of 2^30 tokens are 2^31 rows, one past the limit
+    prm = make_params(1, 2, 128, (1, 1 << 15, 1 << 15), (1, 2, 4))
+    assert lib.squad_attn_fwd_workspace_bytes(ctypes.byref(prm)) == 0
+    assert _fwd(lib, prm) == _lib.SQUAD_ERR_UNSUPPORTED
+    # the padded grid counts: 32767 x 32769 = 2^30 - 1 tokens is accepted as it is, but a window of
+    # height 2 pads it to 32768 x 32769 > 2^30 tokens and is refused
+    grid = (1, (1 << 15) - 1, (1 << 15) + 1)
+    assert lib.squad_attn_fwd_workspace_bytes(ctypes.byref(make_params(1, 1, 128, grid, (1, 1, 1)))) > 0
+    prm = make_params(1, 1, 128, grid, (1, 2, 1))
+    assert lib.squad_attn_fwd_workspace_bytes(ctypes.byref(prm)) == 0
+    assert _fwd(lib, prm) == _lib.SQUAD_ERR_UNSUPPORTED
