@@ -1,6 +1,6 @@
 """CUDA path vs the fp64 oracle, element by element, on the same seeded inputs (needs a B200).
 
-Tolerances (fixed by the benchmark spec of this operator and restated here):
+Tolerances (the acceptance bounds of this library against the fp64 oracle):
   fp32 mode: normwise max |gpu - ref| / max |ref| <= 1e-5.
   bf16 mode (fp32 accumulation): max |gpu - ref| <= 1e-2 * max |ref| and mean |gpu - ref| <= 1e-3 * max |ref|,
   applied to O, and to dQ, dK, dV separately.
