@@ -493,6 +493,64 @@ squad_status_t squad_attn_fwd_status(const squad_params_t* p, const void* worksp
 
 namespace {
 
+// One pass's backward inside a chain of passes. accumulate: add the fp32 dQ/dK shares already in the
+// accumulators; final_out: write dq, dk (input dtype) instead of the accumulators. dv_out receives the
+// gradient of this pass's values in the input dtype.
+squad_status_t bwd_one_pass(const squad_params_t* sp, const Grid& g, int kind, float scale, const void* q,
+                            const void* k, const void* values, const void* dout, const float* lse, uint32_t* status,
+                            float* dq_acc, float* dk_acc, float* drow, void* dq, void* dk, void* dv_out,
+                            bool accumulate, bool final_out, cudaStream_t stream) {
+  const bool bf16 = sp->dtype == SQUAD_BF16;
+  if (bf16) {
+    BwdTcArgs b;
+    std::memset(&b, 0, sizeof(b));
+    b.g = g;
+    b.p = make_geom(g, kind, 256);
+    if (short_eligible(sp, g, b.p) && bwd_tc_plan(b)) {
+      b.variant = kind == kGlobal ? kSlotBoxVariant : 0;
+      if (!encode_pass_map(&b.tm_q, q, g, b.p, b.variant) || !encode_pass_map(&b.tm_k, k, g, b.p, b.variant) ||
+          !encode_pass_map(&b.tm_v, values, g, b.p, b.variant) || !encode_pass_map(&b.tm_do, dout, g, b.p, b.variant))
+        return SQUAD_ERR_CUDA;
+      b.lse = lse;
+      b.dq_acc = dq_acc;
+      b.dk_acc = dk_acc;
+      b.dq_out = static_cast<__nv_bfloat16*>(dq);
+      b.dk_out = static_cast<__nv_bfloat16*>(dk);
+      b.dv_out = static_cast<__nv_bfloat16*>(dv_out);
+      b.final_out = final_out ? 1 : 0;
+      b.accumulate = accumulate ? 1 : 0;
+      b.scale = scale;
+      b.scale_log2 = scale * 1.4426950408889634f;
+      b.status = status;
+      b.timeout_ns = kWaitTimeoutNs;
+      return launch_bwd_tc(b, stream) == cudaSuccess ? SQUAD_OK : SQUAD_ERR_CUDA;
+    }
+  }
+  SimtBwdArgs a{};
+  a.q = q;
+  a.k = k;
+  a.v = values;
+  a.dout = dout;
+  a.lse = lse;
+  a.Drow = drow;
+  a.dq_acc = dq_acc;
+  a.dk_acc = dk_acc;
+  a.dq_out = dq;
+  a.dk_out = dk;
+  a.dv_out = dv_out;
+  a.g = g;
+  a.p = make_geom(g, kind);
+  a.scale = scale;
+  a.in_bf16 = bf16;
+  a.v_bf16 = bf16;
+  a.dout_bf16 = bf16;
+  a.grad_bf16 = bf16;
+  a.dv_bf16 = bf16;
+  a.accumulate = accumulate ? 1 : 0;
+  a.final_out = final_out ? 1 : 0;
+  return launch_simt_bwd(a, stream) == cudaSuccess ? SQUAD_OK : SQUAD_ERR_CUDA;
+}
+
 // The backward on the kernels' grid g (already padded where needed); the control block is zeroed.
 squad_status_t bwd_core(const squad_params_t* p, const Grid& g, float scale, const void* q, const void* k,
                         const void* v, const void* o, const void* dout, const FwdWorkspace& fw,
@@ -502,54 +560,8 @@ squad_status_t bwd_core(const squad_params_t* p, const Grid& g, float scale, con
   if (p->order == SQUAD_LOCAL_ONLY || p->order == SQUAD_GLOBAL_ONLY) {
     // One pass: values v, upstream dout, the pass's LSE in the first slot; no share to add.
     const int kind = p->order == SQUAD_LOCAL_ONLY ? kLocal : kGlobal;
-    if (bf16) {
-      BwdTcArgs b;
-      std::memset(&b, 0, sizeof(b));
-      b.g = g;
-      b.p = make_geom(g, kind, 256);
-      if (short_eligible(p, g, b.p) && bwd_tc_plan(b)) {
-        b.variant = kind == kGlobal ? kSlotBoxVariant : 0;
-        if (!encode_pass_map(&b.tm_q, q, g, b.p, b.variant) || !encode_pass_map(&b.tm_k, k, g, b.p, b.variant) ||
-            !encode_pass_map(&b.tm_v, v, g, b.p, b.variant) || !encode_pass_map(&b.tm_do, dout, g, b.p, b.variant))
-          return SQUAD_ERR_CUDA;
-        b.lse = fw.lse1;
-        b.dq_acc = bw.dq_acc;
-        b.dk_acc = bw.dk_acc;
-        b.dq_out = static_cast<__nv_bfloat16*>(dq);
-        b.dk_out = static_cast<__nv_bfloat16*>(dk);
-        b.dv_out = static_cast<__nv_bfloat16*>(dv);
-        b.final_out = 1;
-        b.accumulate = 0;
-        b.scale = scale;
-        b.scale_log2 = scale * 1.4426950408889634f;
-        b.status = bw.status;
-        b.timeout_ns = kWaitTimeoutNs;
-        return launch_bwd_tc(b, stream) == cudaSuccess ? SQUAD_OK : SQUAD_ERR_CUDA;
-      }
-    }
-    SimtBwdArgs a{};
-    a.q = q;
-    a.k = k;
-    a.v = v;
-    a.dout = dout;
-    a.lse = fw.lse1;
-    a.Drow = bw.drow;
-    a.dq_acc = bw.dq_acc;
-    a.dk_acc = bw.dk_acc;
-    a.dq_out = dq;
-    a.dk_out = dk;
-    a.dv_out = dv;
-    a.g = g;
-    a.p = make_geom(g, kind);
-    a.scale = scale;
-    a.in_bf16 = bf16;
-    a.v_bf16 = bf16;
-    a.dout_bf16 = bf16;
-    a.grad_bf16 = bf16;
-    a.dv_bf16 = bf16;
-    a.accumulate = 0;
-    a.final_out = 1;
-    return launch_simt_bwd(a, stream) == cudaSuccess ? SQUAD_OK : SQUAD_ERR_CUDA;
+    return bwd_one_pass(p, g, kind, scale, q, k, v, dout, fw.lse1, bw.status, bw.dq_acc, bw.dk_acc, bw.drow, dq,
+                        dk, dv, /*accumulate=*/false, /*final_out=*/true, stream);
   }
   const int first = p->order == SQUAD_LOCAL_THEN_GLOBAL ? kLocal : kGlobal;
   const int second = p->order == SQUAD_LOCAL_THEN_GLOBAL ? kGlobal : kLocal;
@@ -775,64 +787,6 @@ KpassBwdWs carve_kpass_bwd(void* ws, const KpassPlan& pl) {
   w.gbuf[0] = kpass_n_gbuf(pl.k) > 0 ? b : nullptr;
   w.gbuf[1] = kpass_n_gbuf(pl.k) > 1 ? b + t : nullptr;
   return w;
-}
-
-// One pass's backward inside a chain of passes. accumulate: add the fp32 dQ/dK shares already in the
-// accumulators; final_out: write dq, dk (input dtype) instead of the accumulators. dv_out receives the
-// gradient of this pass's values in the input dtype.
-squad_status_t bwd_one_pass(const squad_params_t* sp, const Grid& g, int kind, float scale, const void* q,
-                            const void* k, const void* values, const void* dout, const float* lse, uint32_t* status,
-                            float* dq_acc, float* dk_acc, float* drow, void* dq, void* dk, void* dv_out,
-                            bool accumulate, bool final_out, cudaStream_t stream) {
-  const bool bf16 = sp->dtype == SQUAD_BF16;
-  if (bf16) {
-    BwdTcArgs b;
-    std::memset(&b, 0, sizeof(b));
-    b.g = g;
-    b.p = make_geom(g, kind, 256);
-    if (short_eligible(sp, g, b.p) && bwd_tc_plan(b)) {
-      b.variant = kind == kGlobal ? kSlotBoxVariant : 0;
-      if (!encode_pass_map(&b.tm_q, q, g, b.p, b.variant) || !encode_pass_map(&b.tm_k, k, g, b.p, b.variant) ||
-          !encode_pass_map(&b.tm_v, values, g, b.p, b.variant) || !encode_pass_map(&b.tm_do, dout, g, b.p, b.variant))
-        return SQUAD_ERR_CUDA;
-      b.lse = lse;
-      b.dq_acc = dq_acc;
-      b.dk_acc = dk_acc;
-      b.dq_out = static_cast<__nv_bfloat16*>(dq);
-      b.dk_out = static_cast<__nv_bfloat16*>(dk);
-      b.dv_out = static_cast<__nv_bfloat16*>(dv_out);
-      b.final_out = final_out ? 1 : 0;
-      b.accumulate = accumulate ? 1 : 0;
-      b.scale = scale;
-      b.scale_log2 = scale * 1.4426950408889634f;
-      b.status = status;
-      b.timeout_ns = kWaitTimeoutNs;
-      return launch_bwd_tc(b, stream) == cudaSuccess ? SQUAD_OK : SQUAD_ERR_CUDA;
-    }
-  }
-  SimtBwdArgs a{};
-  a.q = q;
-  a.k = k;
-  a.v = values;
-  a.dout = dout;
-  a.lse = lse;
-  a.Drow = drow;
-  a.dq_acc = dq_acc;
-  a.dk_acc = dk_acc;
-  a.dq_out = dq;
-  a.dk_out = dk;
-  a.dv_out = dv_out;
-  a.g = g;
-  a.p = make_geom(g, kind);
-  a.scale = scale;
-  a.in_bf16 = bf16;
-  a.v_bf16 = bf16;
-  a.dout_bf16 = bf16;
-  a.grad_bf16 = bf16;
-  a.dv_bf16 = bf16;
-  a.accumulate = accumulate ? 1 : 0;
-  a.final_out = final_out ? 1 : 0;
-  return launch_simt_bwd(a, stream) == cudaSuccess ? SQUAD_OK : SQUAD_ERR_CUDA;
 }
 
 }  // namespace
