@@ -10,6 +10,7 @@ from .api import (  # noqa: F401
     full_attn_fwd,
     make_kpass_params,
     make_params,
+    squad_attention,
     squad_attn_bwd,
     squad_attn_bwd_workspace_bytes,
     squad_attn_flops,
@@ -18,6 +19,7 @@ from .api import (  # noqa: F401
     squad_attn_fwd_noalloc,
     squad_attn_fwd_status,
     squad_attn_fwd_workspace_bytes,
+    squad_kpass_attention,
     squad_kpass_bwd,
     squad_kpass_flops,
     squad_kpass_fwd,

@@ -244,6 +244,54 @@ def squad_kpass_flops(B, h, d, grid, levels) -> float:
     return float(_lib.load().squad_kpass_flops(ctypes.byref(make_kpass_params(B, h, d, grid, levels))))
 
 
+class _SquadAttention(torch.autograd.Function):
+    """squad_attn_fwd / squad_attn_bwd as one autograd node; the workspace is saved for the backward."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, grid, window, order, scale):
+        q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+        o, ws = squad_attn_fwd(q, k, v, grid, window, order, scale)
+        ctx.save_for_backward(q, k, v, o, ws)
+        ctx.cfg = (grid, window, order, scale)
+        return o
+
+    @staticmethod
+    def backward(ctx, do):
+        q, k, v, o, ws = ctx.saved_tensors
+        grid, window, order, scale = ctx.cfg
+        dq, dk, dv = squad_attn_bwd(q, k, v, o, do.contiguous(), ws, grid, window, order, scale)
+        return dq, dk, dv, None, None, None, None
+
+
+def squad_attention(q, k, v, grid, window, order="local_then_global", scale=None):
+    """SQuad-Attention as a differentiable torch op (the library's forward and backward kernels)."""
+    return _SquadAttention.apply(q, k, v, tuple(grid), tuple(window), order, scale)
+
+
+class _KpassAttention(torch.autograd.Function):
+    """squad_kpass_fwd / squad_kpass_bwd as one autograd node."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, grid, levels, order, scale):
+        q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+        o, ws = squad_kpass_fwd(q, k, v, grid, levels, order, scale)
+        ctx.save_for_backward(q, k, v, o, ws)
+        ctx.cfg = (grid, levels, order, scale)
+        return o
+
+    @staticmethod
+    def backward(ctx, do):
+        q, k, v, o, ws = ctx.saved_tensors
+        grid, levels, order, scale = ctx.cfg
+        dq, dk, dv = squad_kpass_bwd(q, k, v, o, do.contiguous(), ws, grid, levels, order, scale)
+        return dq, dk, dv, None, None, None, None
+
+
+def squad_kpass_attention(q, k, v, grid, levels, order="forward", scale=None):
+    """k composed nested-window passes as a differentiable torch op."""
+    return _KpassAttention.apply(q, k, v, tuple(grid), tuple(tuple(l) for l in levels), order, scale)
+
+
 class HostRunner:
     """End-to-end forward from host buffers: pinned host -> device copies, squad_attn_fwd, device -> host.
 
