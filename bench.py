@@ -373,6 +373,8 @@ SWEEP = [
     ("high-resolution 5B block", 1, 24, 128, (21, 44, 80), (21, 4, 4), ("local_then_global", "local_only", "global_only"),
      True, False),
     ("Wan-2.1-14B block (training step)", 1, 40, 128, (21, 22, 40), (21, 2, 4), ("local_then_global",), False, True),
+    ("Wan-2.2-5B grid, window 21x3x4 (reflect-padded to 21x24x40)", 1, 24, 128, (21, 22, 40), (21, 3, 4),
+     ("local_then_global",), False, True),
 ]
 
 # k composed passes over nested windows on the Wan-2.2-5B grid: (name, B, h, d, grid, levels, orders, with_bwd).
@@ -389,7 +391,7 @@ def sweep(reps=30, only=None, n_sets=3):
     the device, 3 rotating buffer sets, CUDA events on the launching stream."""
     import torch
 
-    from sub_quadratic_two_squad_b200 import full_attn_fwd, squad_attn_bwd, squad_attn_fwd
+    from sub_quadratic_two_squad_b200 import full_attn_fwd, squad_attn_bwd, squad_attn_flops, squad_attn_fwd
 
     dev = torch.device("cuda", 0)
     stream = torch.cuda.current_stream()
@@ -418,9 +420,7 @@ def sweep(reps=30, only=None, n_sets=3):
             wss = [squad_attn_fwd(*sets[i], grid, window, order)[1] for i in range(ns)]
             ms = timed(lambda i: squad_attn_fwd(*sets[i % ns], grid, window, order, out=outs[i % ns],
                                                 workspace=wss[i % ns]), reps)
-            nw = window[0] * window[1] * window[2]
-            terms = {"local_only": n * nw, "global_only": n * n / nw}.get(order, n * nw + n * n / nw)
-            f = 4.0 * B * h * d * terms
+            f = squad_attn_flops(B, h, d, grid, window, order)   # the padded grid's cost where it pads
             t_roof = max(f / (tf_peak * 1e12), alg_bytes(w) / (hbm * 1e9)) * 1e3
             line = {"sweep": name, "order": order, "n": n, "window": "x".join(map(str, window)), "ms_per_block": ms,
                     "tflops": f / (ms * 1e-3) / 1e12, "roofline_ms": t_roof, "roofline_frac": t_roof / ms,
