@@ -5,6 +5,7 @@ across all windows with the local output as values (SQuad paper §3.2, appendix 
 """
 from .api import (  # noqa: F401
     HostRunner,
+    PipelinedHostRunner,
     SquadError,
     full_attn_flops,
     full_attn_fwd,

@@ -323,3 +323,70 @@ class HostRunner:
             squad_attn_fwd(q, k, v, self.grid, self.window, self.order, out=o, workspace=self.ws, stream=self.stream)
             o_host.copy_(o, non_blocking=True)
         return o_host
+
+
+class PipelinedHostRunner:
+    """End-to-end forward from pinned host buffers with the copies overlapped.
+
+    The B*h heads are split into `chunks` groups (heads are independent in both passes). Each group's
+    host -> device copy, forward and device -> host copy run on three streams linked by events, so the
+    input copies of one group overlap the forward of the previous one and the output copy of the one
+    before, in both copy directions at once. Across calls, a group's input copy waits until the
+    previous call's forward has read that group, and its forward waits until the previous call's output
+    copy has read its output. `start` and `end` record CUDA events that bracket any number of calls.
+    """
+
+    def __init__(self, B, h, d, grid, window, order="local_then_global", dtype=torch.bfloat16, device="cuda",
+                 chunks=4):
+        n = grid[0] * grid[1] * grid[2]
+        self.shape = (B, h, n, d)
+        self.grid, self.window, self.order = grid, window, order
+        bh = B * h
+        chunks = max(1, min(int(chunks), bh))
+        self.bounds = [(bh * i) // chunks for i in range(chunks + 1)]
+        self.dev = [torch.empty((bh, n, d), dtype=dtype, device=device) for _ in range(4)]
+        widest = max(b - a for a, b in zip(self.bounds, self.bounds[1:]))
+        self.ws = torch.empty(squad_attn_fwd_workspace_bytes(make_params(1, widest, d, grid, window, order, dtype)),
+                              dtype=torch.uint8, device=device)
+        self.s_in, self.s_comp, self.s_out = (torch.cuda.Stream(device=device) for _ in range(3))
+        self.ev_in = [torch.cuda.Event() for _ in range(chunks)]
+        self.ev_comp = [torch.cuda.Event() for _ in range(chunks)]
+        self.ev_out = [torch.cuda.Event() for _ in range(chunks)]
+
+    def h2d_bytes(self):
+        return 3 * self.dev[0].numel() * self.dev[0].element_size()
+
+    def d2h_bytes(self):
+        return self.dev[3].numel() * self.dev[3].element_size()
+
+    def start(self, event):
+        """Record `event` before the next call's first copy."""
+        event.record(self.s_in)
+
+    def end(self, event):
+        """Record `event` after everything issued so far (the last output copy comes last)."""
+        event.record(self.s_out)
+
+    def __call__(self, q_host, k_host, v_host, o_host):
+        q, k, v, o = self.dev
+        bh, n, d = q.shape
+        hq, hk, hv, ho = (t.view(bh, n, d) for t in (q_host, k_host, v_host, o_host))
+        for c, (a, b) in enumerate(zip(self.bounds, self.bounds[1:])):
+            with torch.cuda.stream(self.s_in):
+                self.s_in.wait_event(self.ev_comp[c])      # the previous call's forward has read this group
+                q[a:b].copy_(hq[a:b], non_blocking=True)
+                k[a:b].copy_(hk[a:b], non_blocking=True)
+                v[a:b].copy_(hv[a:b], non_blocking=True)
+                self.ev_in[c].record(self.s_in)
+            with torch.cuda.stream(self.s_comp):
+                self.s_comp.wait_event(self.ev_in[c])
+                self.s_comp.wait_event(self.ev_out[c])     # the previous call's output copy has read this group
+                shape = (1, b - a, n, d)
+                squad_attn_fwd(q[a:b].view(shape), k[a:b].view(shape), v[a:b].view(shape), self.grid, self.window,
+                               self.order, out=o[a:b].view(shape), workspace=self.ws, stream=self.s_comp)
+                self.ev_comp[c].record(self.s_comp)
+            with torch.cuda.stream(self.s_out):
+                self.s_out.wait_event(self.ev_comp[c])
+                ho[a:b].copy_(o[a:b], non_blocking=True)
+                self.ev_out[c].record(self.s_out)
+        return o_host
