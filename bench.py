@@ -29,6 +29,7 @@ PAGES_MS = 4.27   # pages' SQuad attention latency per block for this workload (
 # DRAM traffic of one launch of the forward kernel from the ncu capture summarised in
 # profiles/short_kernel_wan22_5b_fwd.md (dram__bytes_read.sum + dram__bytes_write.sum), valid only for
 # the kernel source it was measured on (sha1 prefix below); otherwise reported as null.
+NOMINAL_HBM_GBS = 7700.0   # datasheet HBM3e bandwidth (HGX B200), context beside the measured peak
 PROFILED_TRAFFIC_BYTES = (440.588288 + 192.799744) * 1e6
 PROFILED_KERNEL_SHA1 = "2468718f45f72560"
 PROFILED_KERNEL_SRC = os.path.join(ROOT, "sub_quadratic_two_squad_b200", "csrc", "attn_short.cu")
@@ -343,7 +344,8 @@ def run_ours(args, rank, world, local_rank):
                      "traffic": profiled_traffic(), "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)",
                      "kernel": "short_kernel (both passes in one launch) + control-block memset",
                      "alg_bytes_per_launch": alg_bytes(), "mean_launch_ms": mean_launch,
-                     "tensor_frac": f / (mean_launch * 1e-3) / 1e12 / tf_peak},
+                     "tensor_frac": f / (mean_launch * 1e-3) / 1e12 / tf_peak,
+                     "nominal_peak": NOMINAL_HBM_GBS, "frac_of_nominal": achieved / NOMINAL_HBM_GBS},
         "e2e": {"value": world * f / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": runner.h2d_bytes(), "d2h_bytes_per_step": runner.d2h_bytes(),
                 "steps": e2e_steps, "api": "sub_quadratic_two_squad_b200.HostRunner (pinned host buffers)"},
