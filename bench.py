@@ -25,8 +25,8 @@ WORKLOAD_NAME = ("Wan-2.2-5B-shaped SQuad attention block: B=1 h=24 d=128, grid 
                  "window 21x2x4 (w=168, 110 windows), local->global, bf16")
 METRIC = "SQuad-attn fwd ms/block & TFLOP/s at n=18480,h=24,d=128 bf16; % of roofline"
 PAGES_MS = 4.27   # pages' SQuad attention latency per block for this workload (1x H100, bf16): context
-
 NOMINAL_HBM_GBS = 7700.0   # datasheet HBM3e bandwidth (HGX B200), context beside the measured peak
+
 # DRAM traffic of one launch of the forward kernel from the ncu capture summarised in
 # profiles/short_kernel_wan22_5b_fwd.md (dram__bytes_read.sum + dram__bytes_write.sum), valid only for
 # the kernel source it was measured on (sha1 prefix below); otherwise reported as null.
