@@ -72,3 +72,34 @@ def test_two_levels_are_the_two_pass_method(gw, seed):
     for kp, two in ((orc.KPASS_FORWARD, orc.LOCAL_THEN_GLOBAL), (orc.KPASS_REVERSE, orc.GLOBAL_THEN_LOCAL)):
         np.testing.assert_allclose(orc.kpass_fwd(q, k, v, (T, H, W), levels, kp),
                                    orc.squad_attn_fwd(q, k, v, (T, H, W), (T, hw, ww), two), rtol=0, atol=1e-12)
+
+
+@st.composite
+def grid_and_levels(draw):
+    """A small grid factored into three levels per axis (every pass over at least two tokens)."""
+    T = draw(st.integers(1, 2))
+    hs = [draw(st.integers(1, 3)) for _ in range(3)]
+    ws = [draw(st.integers(1, 3)) for _ in range(3)]
+    levels = list(zip(hs, ws))
+    if T * hs[0] * ws[0] < 2:
+        levels[0] = (hs[0], 2)
+    for i in (1, 2):
+        if levels[i][0] * levels[i][1] < 2:
+            levels[i] = (2, levels[i][1])
+    H = int(np.prod([a for a, _ in levels]))
+    W = int(np.prod([b for _, b in levels]))
+    return (T, H, W), levels
+
+
+@settings(max_examples=25, deadline=None)
+@given(grid_and_levels(), st.sampled_from([orc.KPASS_FORWARD, orc.KPASS_REVERSE]), st.integers(0, 2 ** 31 - 1))
+def test_three_levels_reach_every_token_and_keep_constants(gl, order, seed):
+    grid, levels = gl
+    n = grid[0] * grid[1] * grid[2]
+    rng = np.random.default_rng(seed)
+    q, k = rng.standard_normal((1, 1, n, 3)), rng.standard_normal((1, 1, n, 3))
+    m = orc.kpass_composed_matrix(q, k, grid, levels, order)
+    np.testing.assert_allclose(m.sum(-1), 1.0, rtol=0, atol=1e-12)
+    assert (m > 0).all()
+    v = np.broadcast_to(rng.standard_normal((1, 1, 1, 4)), (1, 1, n, 4))
+    np.testing.assert_allclose(orc.kpass_fwd(q, k, v, grid, levels, order), v, rtol=0, atol=1e-12)
