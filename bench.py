@@ -27,9 +27,9 @@ METRIC = "SQuad-attn fwd ms/block & TFLOP/s at n=18480,h=24,d=128 bf16; % of roo
 PAGES_MS = 4.27   # pages' SQuad attention latency per block for this workload (1x H100, bf16): context
 NOMINAL_HBM_GBS = 7700.0   # datasheet HBM3e bandwidth (HGX B200), context beside the measured peak
 
-# DRAM traffic of one launch of the forward kernel from the ncu capture summarised in
-# profiles/short_kernel_wan22_5b_fwd.md (dram__bytes_read.sum + dram__bytes_write.sum), valid only for
-# the kernel source it was measured on (sha1 prefix below); otherwise reported as null.
+# DRAM traffic of one launch of the forward kernel from an ncu capture of this workload
+# (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the kernel source it was measured on
+# (sha1 prefix below); otherwise reported as null.
 PROFILED_TRAFFIC_BYTES = (440.588288 + 192.799744) * 1e6
 PROFILED_KERNEL_SHA1 = "2468718f45f72560"
 PROFILED_KERNEL_SRC = os.path.join(ROOT, "sub_quadratic_two_squad_b200", "csrc", "attn_short.cu")
@@ -142,6 +142,20 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def cpu_model():
+    """The host CPU's model name (from /proc/cpuinfo), or the platform's processor string."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+
+    return platform.processor() or "unknown"
+
+
 def cpu_baseline(budget_s=12.0):
     """The fp64 oracle timed on the host cores, on whole heads of the same workload."""
     import numpy as np
@@ -163,6 +177,7 @@ def cpu_baseline(budget_s=12.0):
     per_head_flops = flops(dict(w, h=1))
     threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
     return {"value": per_head_flops * done / el / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "cpu_model": cpu_model(), "host_cpus": os.cpu_count(),
             "sample": f"{done} of 24 heads of the same block (fp64 numpy oracle, {el:.1f} s)",
             "ms_per_block_extrapolated": el / done * w["h"] * 1e3}
 
@@ -198,6 +213,7 @@ def run_reference(args, rank, world):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": WORKLOAD_NAME, "sample_heads": heads},
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                             "cpu_model": cpu_model(), "host_cpus": os.cpu_count(),
                              "sample": f"{heads} of 24 heads per step"},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)

@@ -148,9 +148,12 @@ SQUAD_API squad_status_t full_attn_fwd(const squad_params_t* p, const void* q, c
  * which every GPU that loads the library holds until the process exits. It is shared by every call:
  * calls that may overlap on the GPU (different streams, or different host threads, without ordering
  * between them) race on it and must be serialised by the caller. Each call zeroes what must start at
- * zero. The first call on a device looks up the array's device address (once per device, with that
- * device current); make that first call before any stream capture on the device. The LSEs and the
- * device status word of this entry point stay inside the scratch and are not exposed.
+ * zero. Every call looks up the array's device address on the current device (a host-side query
+ * with no stream work); make the first call on a device before any stream capture on it. q, k, v
+ * and o must be device memory of the current device (SQUAD_ERR_INVALID_ARG otherwise: the scratch
+ * used is the current device's). The LSEs and the device status word of this entry point stay inside the scratch
+ * and are not exposed: a bounded device-side wait that gives up leaves o incomplete and is not
+ * reported to the caller (the workspace entry point reports it through squad_attn_fwd_status).
  * Returns SQUAD_ERR_UNSUPPORTED, before launching anything, when squad_attn_fwd_workspace_bytes(p)
  * exceeds SQUAD_NOALLOC_MAX_WORKSPACE_BYTES. It allocates nothing (no cudaMalloc or cudaFree). */
 SQUAD_API squad_status_t squad_attn_fwd_noalloc(const squad_params_t* p, const void* q, const void* k,

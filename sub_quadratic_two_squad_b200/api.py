@@ -42,12 +42,26 @@ def _stream(stream):
 
 
 def _check_qkv(*ts):
+    """Every tensor handed to the library (q, k, v, o, dout, dq, dk, dv; None = not given) must be a
+    contiguous CUDA tensor of q's dtype, shape and device: the kernels address them with q's layout on
+    the device the call runs on."""
     q = ts[0]
     for t in ts:
-        if not t.is_cuda or not t.is_contiguous() or t.dtype != q.dtype or t.shape != q.shape:
-            raise ValueError("q, k, v (and o, dout) must be contiguous CUDA tensors of one dtype and shape [B,h,n,d]")
+        if t is None:
+            continue
+        if (not t.is_cuda or not t.is_contiguous() or t.dtype != q.dtype or t.shape != q.shape
+                or t.device != q.device):
+            raise ValueError("q, k, v and the outputs must be contiguous CUDA tensors of one dtype, shape "
+                             "[B,h,n,d] and device")
     if q.dim() != 4:
         raise ValueError("expected [B, h, n, d]")
+
+
+def _check_workspace(ws, q, nbytes):
+    if not ws.is_cuda or ws.device != q.device or not ws.is_contiguous():
+        raise ValueError("the workspace must be a contiguous CUDA tensor on q's device")
+    if ws.numel() * ws.element_size() < nbytes:
+        raise ValueError(f"workspace needs {nbytes} bytes")
 
 
 def _params_for(q, grid, window, order, scale):
@@ -68,7 +82,7 @@ def squad_attn_bwd_workspace_bytes(params) -> int:
 def squad_attn_fwd(q, k, v, grid, window, order="local_then_global", scale=None, out=None, workspace=None,
                    stream=None):
     """SQuad-Attention forward. Returns (out, workspace); keep the workspace for squad_attn_bwd."""
-    _check_qkv(q, k, v)
+    _check_qkv(q, k, v, out)
     prm = _params_for(q, grid, window, order, scale)
     lib = _lib.load()
     nbytes = lib.squad_attn_fwd_workspace_bytes(ctypes.byref(prm))
@@ -77,9 +91,11 @@ def squad_attn_fwd(q, k, v, grid, window, order="local_then_global", scale=None,
     out = torch.empty_like(q) if out is None else out
     if workspace is None:
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
-    elif workspace.numel() * workspace.element_size() < nbytes:
-        raise ValueError(f"workspace needs {nbytes} bytes")
-    st = lib.squad_attn_fwd(ctypes.byref(prm), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(workspace), _stream(stream))
+    else:
+        _check_workspace(workspace, q, nbytes)
+    with torch.cuda.device(q.device):
+        st = lib.squad_attn_fwd(ctypes.byref(prm), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(workspace),
+                                _stream(stream))
     if st != _lib.SQUAD_OK:
         raise SquadError(st, "squad_attn_fwd")
     return out, workspace
@@ -88,10 +104,12 @@ def squad_attn_fwd(q, k, v, grid, window, order="local_then_global", scale=None,
 def squad_attn_fwd_noalloc(q, k, v, grid, window, order="local_then_global", scale=None, out=None, stream=None):
     """SQuad-Attention forward with the library's fixed device scratch instead of a workspace (for
     callers that cannot allocate device memory; calls that overlap on the GPU race on the scratch)."""
-    _check_qkv(q, k, v)
+    _check_qkv(q, k, v, out)
     prm = _params_for(q, grid, window, order, scale)
     out = torch.empty_like(q) if out is None else out
-    st = _lib.load().squad_attn_fwd_noalloc(ctypes.byref(prm), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _stream(stream))
+    with torch.cuda.device(q.device):
+        st = _lib.load().squad_attn_fwd_noalloc(ctypes.byref(prm), _ptr(q), _ptr(k), _ptr(v), _ptr(out),
+                                                _stream(stream))
     if st != _lib.SQUAD_OK:
         raise SquadError(st, "squad_attn_fwd_noalloc")
     return out
@@ -100,27 +118,30 @@ def squad_attn_fwd_noalloc(q, k, v, grid, window, order="local_then_global", sca
 def squad_attn_fwd_status(workspace, q, grid, window, order="local_then_global", scale=None, stream=None) -> int:
     """Device status of the last call on `workspace` (synchronises the stream): 0 ok, 4 timeout."""
     prm = _params_for(q, grid, window, order, scale)
-    return int(_lib.load().squad_attn_fwd_status(ctypes.byref(prm), _ptr(workspace), _stream(stream)))
+    with torch.cuda.device(q.device):
+        return int(_lib.load().squad_attn_fwd_status(ctypes.byref(prm), _ptr(workspace), _stream(stream)))
 
 
 def squad_attn_bwd(q, k, v, o, dout, fwd_workspace, grid, window, order="local_then_global", scale=None,
                    dq=None, dk=None, dv=None, workspace=None, stream=None):
     """Gradients (dq, dk, dv) of <dout, o>; `fwd_workspace` as left by squad_attn_fwd."""
-    _check_qkv(q, k, v, o, dout)
+    _check_qkv(q, k, v, o, dout, dq, dk, dv)
     prm = _params_for(q, grid, window, order, scale)
     lib = _lib.load()
     nbytes = lib.squad_attn_bwd_workspace_bytes(ctypes.byref(prm))
     if nbytes == 0:
         raise SquadError(_lib.SQUAD_ERR_INVALID_ARG, "squad_attn_bwd_workspace_bytes")
+    _check_workspace(fwd_workspace, q, lib.squad_attn_fwd_workspace_bytes(ctypes.byref(prm)))
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(q) if dk is None else dk
     dv = torch.empty_like(q) if dv is None else dv
     if workspace is None:
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
-    elif workspace.numel() * workspace.element_size() < nbytes:
-        raise ValueError(f"workspace needs {nbytes} bytes")
-    st = lib.squad_attn_bwd(ctypes.byref(prm), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(fwd_workspace),
-                            _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace), _stream(stream))
+    else:
+        _check_workspace(workspace, q, nbytes)
+    with torch.cuda.device(q.device):
+        st = lib.squad_attn_bwd(ctypes.byref(prm), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout),
+                                _ptr(fwd_workspace), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace), _stream(stream))
     if st != _lib.SQUAD_OK:
         raise SquadError(st, "squad_attn_bwd")
     return dq, dk, dv
@@ -128,13 +149,17 @@ def squad_attn_bwd(q, k, v, o, dout, fwd_workspace, grid, window, order="local_t
 
 def full_attn_fwd(q, k, v, grid=None, scale=None, out=None, lse=None, stream=None):
     """softmax(q k^T * scale) v over all n tokens per head. Returns out (and fills `lse` if given)."""
-    _check_qkv(q, k, v)
+    _check_qkv(q, k, v, out)
     B, h, n, d = q.shape
+    if lse is not None and (not lse.is_cuda or lse.device != q.device or lse.dtype != torch.float32
+                            or not lse.is_contiguous() or lse.numel() < B * h * n):
+        raise ValueError("lse must be a contiguous float32 CUDA tensor of B*h*n elements on q's device")
     grid = (1, 1, n) if grid is None else grid
     prm = _params_for(q, grid, (1, 1, 1), "local_then_global", scale)
     out = torch.empty_like(q) if out is None else out
-    st = _lib.load().full_attn_fwd(ctypes.byref(prm), _ptr(q), _ptr(k), _ptr(v), _ptr(out),
-                                   _ptr(lse), _stream(stream))
+    with torch.cuda.device(q.device):
+        st = _lib.load().full_attn_fwd(ctypes.byref(prm), _ptr(q), _ptr(k), _ptr(v), _ptr(out),
+                                       _ptr(lse), _stream(stream))
     if st != _lib.SQUAD_OK:
         raise SquadError(st, "full_attn_fwd")
     return out
@@ -194,7 +219,7 @@ def squad_kpass_pass_params(params, level):
 
 def squad_kpass_fwd(q, k, v, grid, levels, order="forward", scale=None, out=None, workspace=None, stream=None):
     """k nested-window passes composed. Returns (out, workspace); keep the workspace for the backward."""
-    _check_qkv(q, k, v)
+    _check_qkv(q, k, v, out)
     prm = _kpass_params_for(q, grid, levels, order, scale)
     lib = _lib.load()
     nbytes = lib.squad_kpass_fwd_workspace_bytes(ctypes.byref(prm))
@@ -203,9 +228,11 @@ def squad_kpass_fwd(q, k, v, grid, levels, order="forward", scale=None, out=None
     out = torch.empty_like(q) if out is None else out
     if workspace is None:
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
-    elif workspace.numel() * workspace.element_size() < nbytes:
-        raise ValueError(f"workspace needs {nbytes} bytes")
-    st = lib.squad_kpass_fwd(ctypes.byref(prm), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(workspace), _stream(stream))
+    else:
+        _check_workspace(workspace, q, nbytes)
+    with torch.cuda.device(q.device):
+        st = lib.squad_kpass_fwd(ctypes.byref(prm), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(workspace),
+                                 _stream(stream))
     if st != _lib.SQUAD_OK:
         raise SquadError(st, "squad_kpass_fwd")
     return out, workspace
@@ -214,21 +241,23 @@ def squad_kpass_fwd(q, k, v, grid, levels, order="forward", scale=None, out=None
 def squad_kpass_bwd(q, k, v, o, dout, fwd_workspace, grid, levels, order="forward", scale=None, dq=None, dk=None,
                     dv=None, workspace=None, stream=None):
     """Gradients (dq, dk, dv) of <dout, o> for squad_kpass_fwd; `fwd_workspace` as it left it."""
-    _check_qkv(q, k, v, o, dout)
+    _check_qkv(q, k, v, o, dout, dq, dk, dv)
     prm = _kpass_params_for(q, grid, levels, order, scale)
     lib = _lib.load()
     nbytes = lib.squad_kpass_bwd_workspace_bytes(ctypes.byref(prm))
     if nbytes == 0:
         raise SquadError(_lib.SQUAD_ERR_INVALID_ARG, "squad_kpass_bwd_workspace_bytes")
+    _check_workspace(fwd_workspace, q, lib.squad_kpass_fwd_workspace_bytes(ctypes.byref(prm)))
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(q) if dk is None else dk
     dv = torch.empty_like(q) if dv is None else dv
     if workspace is None:
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
-    elif workspace.numel() * workspace.element_size() < nbytes:
-        raise ValueError(f"workspace needs {nbytes} bytes")
-    st = lib.squad_kpass_bwd(ctypes.byref(prm), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(fwd_workspace),
-                             _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace), _stream(stream))
+    else:
+        _check_workspace(workspace, q, nbytes)
+    with torch.cuda.device(q.device):
+        st = lib.squad_kpass_bwd(ctypes.byref(prm), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout),
+                                 _ptr(fwd_workspace), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace), _stream(stream))
     if st != _lib.SQUAD_OK:
         raise SquadError(st, "squad_kpass_bwd")
     return dq, dk, dv
@@ -237,7 +266,8 @@ def squad_kpass_bwd(q, k, v, o, dout, fwd_workspace, grid, levels, order="forwar
 def squad_kpass_status(workspace, q, grid, levels, order="forward", scale=None, stream=None) -> int:
     """Device status of the last k-pass call on `workspace` (synchronises the stream): 0 ok, 4 timeout."""
     prm = _kpass_params_for(q, grid, levels, order, scale)
-    return int(_lib.load().squad_kpass_status(ctypes.byref(prm), _ptr(workspace), _stream(stream)))
+    with torch.cuda.device(q.device):
+        return int(_lib.load().squad_kpass_status(ctypes.byref(prm), _ptr(workspace), _stream(stream)))
 
 
 def squad_kpass_flops(B, h, d, grid, levels) -> float:

@@ -1,7 +1,6 @@
 // squad_attn_fwd_noalloc: the SQuad forward with its scratch in a fixed device array, for callers that
 // cannot allocate device memory (see include/squad_attn.h).
 #include <cstddef>
-#include <mutex>
 
 #include <cuda_runtime.h>
 
@@ -14,22 +13,26 @@ namespace {
 constexpr size_t kStaticScratchBytes = static_cast<size_t>(SQUAD_NOALLOC_MAX_WORKSPACE_BYTES);
 __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
-constexpr int kMaxDevices = 64;
-
 // Device address of g_static_scratch on the current device. In host code the symbol itself is only a
-// host-side stand-in, so the address is looked up once per device, with that device current.
+// host-side stand-in, so the address is looked up with the device current. The lookup is a host-side
+// query with no stream work and is repeated on every call, so a context that was torn down and created
+// again (cudaDeviceReset) never sees a stale address.
 void* scratch_on_current_device() {
-  static std::mutex mu;
-  static void* addr[kMaxDevices] = {nullptr};
+  void* ptr = nullptr;
+  if (cudaGetSymbolAddress(&ptr, g_static_scratch) != cudaSuccess) return nullptr;
+  return ptr;
+}
+
+// True when `p` is device memory of the current device (the kernels run there, with its scratch).
+bool on_current_device(const void* p) {
   int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  std::lock_guard<std::mutex> lock(mu);
-  if (addr[dev] == nullptr) {
-    void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_static_scratch) != cudaSuccess) return nullptr;
-    addr[dev] = ptr;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  cudaPointerAttributes at{};
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    cudaGetLastError();   // an unknown pointer's error is not sticky: clear it for later callers
+    return false;
   }
-  return addr[dev];
+  return (at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged) && at.device == dev;
 }
 
 }  // namespace
@@ -39,6 +42,10 @@ extern "C" squad_status_t squad_attn_fwd_noalloc(const squad_params_t* p, const 
   const size_t need = squad_attn_fwd_workspace_bytes(p);
   if (need == 0) return SQUAD_ERR_INVALID_ARG;
   if (need > kStaticScratchBytes) return SQUAD_ERR_UNSUPPORTED;
+  // Every tensor must live on the current device: the scratch used below is that device's copy.
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return SQUAD_ERR_INVALID_ARG;
+  if (!on_current_device(q) || !on_current_device(k) || !on_current_device(v) || !on_current_device(o))
+    return SQUAD_ERR_INVALID_ARG;
   void* scratch = scratch_on_current_device();
   if (scratch == nullptr) return SQUAD_ERR_CUDA;
   // The forward zeroes the control block at the start of every call; the rest of the scratch is
