@@ -159,6 +159,32 @@ SQUAD_API squad_status_t full_attn_fwd(const squad_params_t* p, const void* q, c
 SQUAD_API squad_status_t squad_attn_fwd_noalloc(const squad_params_t* p, const void* q, const void* k,
                                                 const void* v, void* o, squad_stream_t stream);
 
+/* squad_attn_fwd from host memory, end to end: q, k, v are copied from host to the device buffers, the
+ * forward runs, and o is copied back to host memory. The B*h (batch, head) pairs are split into
+ * `groups` runs of consecutive pairs; every pair is independent in both passes (each pass folds the
+ * axis it does not attend over into the batch of heads: agihunt.info digest, the paragraph that
+ * defines the operator), so each run is a forward of its own on contiguous slices of the tensors. The
+ * run's host-to-device copies go on copy_in, its forward on compute and its device-to-host copy on
+ * copy_out, ordered by events: the input copies of one run overlap the forward of the previous run
+ * and the output copy of the one before (the three streams may be the same stream, which serialises
+ * everything). The call only enqueues work: q_host, k_host, v_host must stay unchanged until copy_in
+ * has passed this call, and o_host is complete once copy_out has. Host buffers should be pinned
+ * (cudaHostAlloc / cudaHostRegister) for the copies to be asynchronous.
+ * q_dev, k_dev, v_dev, o_dev: device buffers of the full [B,h,n,d] size (16-byte aligned);
+ * workspace: >= squad_attn_fwd_host_workspace_bytes(p, groups) (256-byte aligned), reused by the runs
+ * one after another on `compute`. Work already queued on `compute` or `copy_out` when the call is made
+ * is finished before this call's copies overwrite the device buffers. 1 <= groups <= min(64, B*h).
+ * The library creates 130 CUDA events per device on the first call there and keeps them until the
+ * process exits; calls on one device enqueue one at a time. Argument errors return
+ * SQUAD_ERR_INVALID_ARG before anything is enqueued; a failed copy or launch returns SQUAD_ERR_CUDA (or
+ * the forward's own status) with the runs before it enqueued. */
+SQUAD_API size_t squad_attn_fwd_host_workspace_bytes(const squad_params_t* p, int groups);
+SQUAD_API squad_status_t squad_attn_fwd_host(const squad_params_t* p, const void* q_host, const void* k_host,
+                                             const void* v_host, void* o_host, void* q_dev, void* k_dev,
+                                             void* v_dev, void* o_dev, void* workspace, int groups,
+                                             squad_stream_t copy_in, squad_stream_t compute,
+                                             squad_stream_t copy_out);
+
 /* FLOPs of one call, from the paper's cost model (appendix "Conformance to the theoretical curves
  * is quantitative"): 4 B h d (n w + n^2/w) for SQuad (one of the two terms for a single-pass order;
  * n = the padded token count when the window does not divide the grid, the cost of the window

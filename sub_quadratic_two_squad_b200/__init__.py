@@ -5,7 +5,6 @@ across all windows with the local output as values (SQuad paper §3.2, appendix 
 """
 from .api import (  # noqa: F401
     HostRunner,
-    PipelinedHostRunner,
     SquadError,
     full_attn_flops,
     full_attn_fwd,
@@ -17,6 +16,8 @@ from .api import (  # noqa: F401
     squad_attn_flops,
     squad_window_solve,
     squad_attn_fwd,
+    squad_attn_fwd_host,
+    squad_attn_fwd_host_workspace_bytes,
     squad_attn_fwd_noalloc,
     squad_attn_fwd_status,
     squad_attn_fwd_workspace_bytes,

@@ -45,6 +45,9 @@ SIGNATURES = {
     "squad_attn_bwd": (ctypes.c_int, [_PP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
     "full_attn_fwd": (ctypes.c_int, [_PP, _VP, _VP, _VP, _VP, _VP, _VP]),
     "squad_attn_fwd_noalloc": (ctypes.c_int, [_PP, _VP, _VP, _VP, _VP, _VP]),
+    "squad_attn_fwd_host_workspace_bytes": (ctypes.c_size_t, [_PP, ctypes.c_int]),
+    "squad_attn_fwd_host": (ctypes.c_int, [_PP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, ctypes.c_int, _VP, _VP,
+                                           _VP]),
     "squad_attn_flops": (ctypes.c_double, [_PP]),
     "squad_window_solve": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_int),
                                           ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]),

@@ -322,66 +322,52 @@ def squad_kpass_attention(q, k, v, grid, levels, order="forward", scale=None):
     return _KpassAttention.apply(q, k, v, tuple(grid), tuple(tuple(l) for l in levels), order, scale)
 
 
+def squad_attn_fwd_host_workspace_bytes(params, groups) -> int:
+    return int(_lib.load().squad_attn_fwd_host_workspace_bytes(ctypes.byref(params), int(groups)))
+
+
+def squad_attn_fwd_host(q_host, k_host, v_host, o_host, q_dev, k_dev, v_dev, o_dev, workspace, grid, window,
+                        order="local_then_global", scale=None, groups=4, copy_in=None, compute=None, copy_out=None):
+    """The C forward from host memory (squad_attn_fwd_host): q, k, v host tensors -> device buffers ->
+    forward -> o_host, in `groups` runs of heads whose copies overlap the forwards on three streams."""
+    for t in (q_host, k_host, v_host, o_host):
+        if t.is_cuda or not t.is_contiguous() or t.shape != q_dev.shape or t.dtype != q_dev.dtype:
+            raise ValueError("host tensors must be contiguous CPU tensors of the device buffers' shape and dtype")
+    _check_qkv(q_dev, k_dev, v_dev, o_dev)
+    prm = _params_for(q_dev, grid, window, order, scale)
+    lib = _lib.load()
+    nbytes = lib.squad_attn_fwd_host_workspace_bytes(ctypes.byref(prm), int(groups))
+    if nbytes == 0:
+        raise SquadError(_lib.SQUAD_ERR_INVALID_ARG, "squad_attn_fwd_host_workspace_bytes")
+    _check_workspace(workspace, q_dev, nbytes)
+    with torch.cuda.device(q_dev.device):
+        st = lib.squad_attn_fwd_host(ctypes.byref(prm), _ptr(q_host), _ptr(k_host), _ptr(v_host), _ptr(o_host),
+                                     _ptr(q_dev), _ptr(k_dev), _ptr(v_dev), _ptr(o_dev), _ptr(workspace), int(groups),
+                                     _stream(copy_in), _stream(compute), _stream(copy_out))
+    if st != _lib.SQUAD_OK:
+        raise SquadError(st, "squad_attn_fwd_host")
+    return o_host
+
+
 class HostRunner:
-    """End-to-end forward from host buffers: pinned host -> device copies, squad_attn_fwd, device -> host.
+    """End-to-end forward from pinned host buffers through the C entry point squad_attn_fwd_host.
 
-    Device buffers are allocated once; every call() copies the inputs in and the output back on the
-    runner's stream, so the copies are part of what a caller holding host data pays.
-    """
-
-    def __init__(self, B, h, d, grid, window, order="local_then_global", dtype=torch.bfloat16, device="cuda"):
-        n = grid[0] * grid[1] * grid[2]
-        self.shape = (B, h, n, d)
-        self.grid, self.window, self.order = grid, window, order
-        self.dev = [torch.empty(self.shape, dtype=dtype, device=device) for _ in range(4)]
-        prm = make_params(B, h, d, grid, window, order, dtype)
-        self.ws = torch.empty(squad_attn_fwd_workspace_bytes(prm), dtype=torch.uint8, device=device)
-        self.stream = torch.cuda.Stream(device=device)
-
-    def h2d_bytes(self):
-        return 3 * self.dev[0].numel() * self.dev[0].element_size()
-
-    def d2h_bytes(self):
-        return self.dev[3].numel() * self.dev[3].element_size()
-
-    def __call__(self, q_host, k_host, v_host, o_host):
-        q, k, v, o = self.dev
-        with torch.cuda.stream(self.stream):
-            q.copy_(q_host, non_blocking=True)
-            k.copy_(k_host, non_blocking=True)
-            v.copy_(v_host, non_blocking=True)
-            squad_attn_fwd(q, k, v, self.grid, self.window, self.order, out=o, workspace=self.ws, stream=self.stream)
-            o_host.copy_(o, non_blocking=True)
-        return o_host
-
-
-class PipelinedHostRunner:
-    """End-to-end forward from pinned host buffers with the copies overlapped.
-
-    The B*h heads are split into `chunks` groups (heads are independent in both passes). Each group's
-    host -> device copy, forward and device -> host copy run on three streams linked by events, so the
-    input copies of one group overlap the forward of the previous one and the output copy of the one
-    before, in both copy directions at once. Across calls, a group's input copy waits until the
-    previous call's forward has read that group, and its forward waits until the previous call's output
-    copy has read its output. `start` and `end` record CUDA events that bracket any number of calls.
+    Device buffers, the workspace and three streams (input copies, forwards, output copies) are made
+    once; every call() enqueues the copies in, the forwards and the copies out for `groups` runs of
+    heads, overlapping each run's copies with the neighbouring runs' forwards. `start` and `end` record
+    CUDA events that bracket any number of calls (end: after the last output copy).
     """
 
     def __init__(self, B, h, d, grid, window, order="local_then_global", dtype=torch.bfloat16, device="cuda",
-                 chunks=4):
+                 groups=4):
         n = grid[0] * grid[1] * grid[2]
         self.shape = (B, h, n, d)
         self.grid, self.window, self.order = grid, window, order
-        bh = B * h
-        chunks = max(1, min(int(chunks), bh))
-        self.bounds = [(bh * i) // chunks for i in range(chunks + 1)]
-        self.dev = [torch.empty((bh, n, d), dtype=dtype, device=device) for _ in range(4)]
-        widest = max(b - a for a, b in zip(self.bounds, self.bounds[1:]))
-        self.ws = torch.empty(squad_attn_fwd_workspace_bytes(make_params(1, widest, d, grid, window, order, dtype)),
-                              dtype=torch.uint8, device=device)
+        self.groups = max(1, min(int(groups), B * h, 64))
+        self.dev = [torch.empty(self.shape, dtype=dtype, device=device) for _ in range(4)]
+        prm = make_params(B, h, d, grid, window, order, dtype)
+        self.ws = torch.empty(squad_attn_fwd_host_workspace_bytes(prm, self.groups), dtype=torch.uint8, device=device)
         self.s_in, self.s_comp, self.s_out = (torch.cuda.Stream(device=device) for _ in range(3))
-        self.ev_in = [torch.cuda.Event() for _ in range(chunks)]
-        self.ev_comp = [torch.cuda.Event() for _ in range(chunks)]
-        self.ev_out = [torch.cuda.Event() for _ in range(chunks)]
 
     def h2d_bytes(self):
         return 3 * self.dev[0].numel() * self.dev[0].element_size()
@@ -399,24 +385,6 @@ class PipelinedHostRunner:
 
     def __call__(self, q_host, k_host, v_host, o_host):
         q, k, v, o = self.dev
-        bh, n, d = q.shape
-        hq, hk, hv, ho = (t.view(bh, n, d) for t in (q_host, k_host, v_host, o_host))
-        for c, (a, b) in enumerate(zip(self.bounds, self.bounds[1:])):
-            with torch.cuda.stream(self.s_in):
-                self.s_in.wait_event(self.ev_comp[c])      # the previous call's forward has read this group
-                q[a:b].copy_(hq[a:b], non_blocking=True)
-                k[a:b].copy_(hk[a:b], non_blocking=True)
-                v[a:b].copy_(hv[a:b], non_blocking=True)
-                self.ev_in[c].record(self.s_in)
-            with torch.cuda.stream(self.s_comp):
-                self.s_comp.wait_event(self.ev_in[c])
-                self.s_comp.wait_event(self.ev_out[c])     # the previous call's output copy has read this group
-                shape = (1, b - a, n, d)
-                squad_attn_fwd(q[a:b].view(shape), k[a:b].view(shape), v[a:b].view(shape), self.grid, self.window,
-                               self.order, out=o[a:b].view(shape), workspace=self.ws, stream=self.s_comp)
-                self.ev_comp[c].record(self.s_comp)
-            with torch.cuda.stream(self.s_out):
-                self.s_out.wait_event(self.ev_comp[c])
-                ho[a:b].copy_(o[a:b], non_blocking=True)
-                self.ev_out[c].record(self.s_out)
-        return o_host
+        return squad_attn_fwd_host(q_host, k_host, v_host, o_host, q, k, v, o, self.ws, self.grid, self.window,
+                                   self.order, groups=self.groups, copy_in=self.s_in, compute=self.s_comp,
+                                   copy_out=self.s_out)

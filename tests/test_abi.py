@@ -183,3 +183,24 @@ def test_size_limits(lib):
     prm = make_params(1, 1, 128, grid, (1, 2, 1))
     assert lib.squad_attn_fwd_workspace_bytes(ctypes.byref(prm)) == 0
     assert _fwd(lib, prm) == _lib.SQUAD_ERR_UNSUPPORTED
+
+
+def test_host_forward_rejects_bad_arguments_before_enqueueing(lib):
+    prm = _p()
+    assert lib.squad_attn_fwd_host_workspace_bytes(ctypes.byref(prm), 4) > 0
+    assert lib.squad_attn_fwd_host_workspace_bytes(ctypes.byref(prm), 0) == 0
+    assert lib.squad_attn_fwd_host_workspace_bytes(ctypes.byref(prm), 25) == 0    # more runs than heads
+    assert lib.squad_attn_fwd_host_workspace_bytes(ctypes.byref(prm), 65) == 0
+    # a run's workspace is that of its heads only
+    one = lib.squad_attn_fwd_host_workspace_bytes(ctypes.byref(prm), 24)
+    assert one == lib.squad_attn_fwd_workspace_bytes(ctypes.byref(_p(h=1)))
+    host, dev, ws = ctypes.c_void_p(4096), ctypes.c_void_p(16), ctypes.c_void_p(256)
+
+    def call(prm=prm, groups=4, h=host, d=dev, w=ws):
+        return lib.squad_attn_fwd_host(ctypes.byref(prm), h, h, h, h, d, d, d, d, w, groups, None, None, None)
+
+    assert call(groups=0) == _lib.SQUAD_ERR_INVALID_ARG
+    assert call(prm=_p(window=(20, 2, 4))) == _lib.SQUAD_ERR_INVALID_ARG
+    assert call(h=ctypes.c_void_p(0)) == _lib.SQUAD_ERR_INVALID_ARG
+    assert call(d=ctypes.c_void_p(8)) == _lib.SQUAD_ERR_INVALID_ARG             # not 16-byte aligned
+    assert call(w=ctypes.c_void_p(128)) == _lib.SQUAD_ERR_INVALID_ARG           # not 256-byte aligned
