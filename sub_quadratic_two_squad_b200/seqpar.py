@@ -17,6 +17,8 @@ Requirements: T % R == 0, H % hw == W % ww == 0 and (H / hw) % R == 0.
 Compute is the library's single-pass forward and backward (`local_only` / `global_only`); the exchange
 is torch.distributed.all_to_all_single on contiguous buffers, so on GPUs it is NCCL over NVLink. The
 per-rank compute can be replaced (`fwd`, `bwd` arguments) for testing the exchange without a GPU.
+With one rank both exchanges are the identity and the band is the whole grid, so the library's fused
+two-pass forward and its backward run directly (no exchange buffers, no single-pass split).
 """
 from __future__ import annotations
 
@@ -38,6 +40,8 @@ class SeqParallelSquad:
         self.band_grid = (T, self.Hb, W)                   # the local pass's grid on this rank
         self.frame_grid = (self.Tg, H, W)                  # the global pass's grid on this rank
         self.frame_window = (self.Tg, hw, ww)
+        # one rank with the library's own compute: the fused launch, no exchange
+        self.whole = self.R == 1 and fwd is None and bwd is None
         if fwd is None or bwd is None:
             from .api import squad_attn_bwd, squad_attn_fwd
             fwd = fwd or (lambda q, k, v, g, w, o: squad_attn_fwd(q, k, v, g, w, o))
@@ -77,6 +81,11 @@ class SeqParallelSquad:
 
     def forward(self, q, k, v, order="local_then_global"):
         """q, k, v: this rank's band. Returns (o band, ctx for backward)."""
+        if order not in ("local_then_global", "global_then_local"):
+            raise ValueError(order)
+        if self.whole:
+            o, ws = self._fwd(q, k, v, self.grid, self.window, order)
+            return o, ("whole", order, q, k, v, o, ws)
         if order == "local_then_global":
             o1, ws1 = self._local(q, k, v)
             qf, kf, o1f = self.band_to_frames(q), self.band_to_frames(k), self.band_to_frames(o1)
@@ -92,6 +101,9 @@ class SeqParallelSquad:
 
     def backward(self, ctx, dout):
         """dout: this rank's band of the upstream gradient. Returns (dq, dk, dv) bands."""
+        if ctx[0] == "whole":
+            _, order, q, k, v, o, ws = ctx
+            return self._bwd(q, k, v, o, dout, ws, self.grid, self.window, order)
         order = ctx[0]
         if order == "local_then_global":
             _, q, k, v, o1, ws1, qf, kf, o1f, of, ws2 = ctx

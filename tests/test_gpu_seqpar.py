@@ -1,5 +1,7 @@
-"""Sequence-parallel SQuad with the CUDA kernels on one GPU (a one-rank NCCL group: the exchanges are
-the identity, every other step runs), forward and backward against the fp64 oracle (needs a B200)."""
+"""Sequence-parallel SQuad with the CUDA kernels on one GPU (a one-rank NCCL group), forward and backward
+against the fp64 oracle (needs a B200): the one-rank shortcut (the fused launch), and the split path
+forced with explicit compute functions (single-pass launches around the exchanges, which are the
+identity at one rank)."""
 import os
 import socket
 
@@ -27,13 +29,21 @@ def one_rank_group():
     dist.destroy_process_group()
 
 
+@pytest.mark.parametrize("split", [False, True])
 @pytest.mark.parametrize("order", ["local_then_global", "global_then_local"])
-def test_sequence_parallel_one_rank(one_rank_group, order):
+def test_sequence_parallel_one_rank(one_rank_group, order, split):
     grid, window = (21, 4, 8), (21, 2, 4)
     n = 21 * 4 * 8
     x = make_inputs(2, 2, n, 128, dtype="bf16", with_dout=True)
     q, k, v, do = (_dev(x[s], torch.bfloat16) for s in ("q", "k", "v", "do"))
-    sp = SeqParallelSquad(grid, window)
+    if split:
+        from sub_quadratic_two_squad_b200 import squad_attn_bwd, squad_attn_fwd
+        sp = SeqParallelSquad(grid, window, fwd=lambda q, k, v, g, w, o: squad_attn_fwd(q, k, v, g, w, o),
+                              bwd=lambda q, k, v, out, do, ws, g, w, o: squad_attn_bwd(q, k, v, out, do, ws, g, w, o))
+        assert not sp.whole
+    else:
+        sp = SeqParallelSquad(grid, window)
+        assert sp.whole
     o, ctx = sp.forward(q, k, v, order)
     dq, dk, dv = sp.backward(ctx, do)
     oo = {"local_then_global": orc.LOCAL_THEN_GLOBAL, "global_then_local": orc.GLOBAL_THEN_LOCAL}[order]
