@@ -397,6 +397,7 @@ __global__ void __launch_bounds__(kThreads, 1) short_kernel(const __grid_constan
 #pragma unroll
             for (int i = 0; i < 4; ++i) ls[i] *= f;
             uint32_t pw[16];   // 16 columns at a time: the current chunk's 64 scores stay live
+            tmem_wait_st();    // the P words written so far have landed
 #pragma unroll 1
             for (int cc = 0; cc < 2 * c; ++cc) {
               tmem_ld16(t_s + 16 * cc, pw);
@@ -420,8 +421,9 @@ __global__ void __launch_bounds__(kThreads, 1) short_kernel(const __grid_constan
             ls[(2 * j + 1) & 3] += x1;
             pk[j] = __byte_perm(__float_as_uint(x0) + 0x8000u, __float_as_uint(x1) + 0x8000u, 0x7632);
           }
-          tmem_st32(t_s + 32 * c, pk);
+          tmem_st32_nowait(t_s + 32 * c, pk);   // over scores already read; waited for below
         }
+        tmem_wait_st();
         l = (ls[0] + ls[1]) + (ls[2] + ls[3]);
       }
       tc_fence_before();

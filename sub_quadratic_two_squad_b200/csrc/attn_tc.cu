@@ -376,7 +376,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pass_kernel(const __grid_const
                   ls[(2 * j + 1) & 3] += x1;
                   pk[j] = __byte_perm(__float_as_uint(x0) + 0x8000u, __float_as_uint(x1) + 0x8000u, 0x7632);
                 }
-                tmem_st16(t_s + 32 * c + 16 * k, pk);
+                tmem_st16_nowait(t_s + 32 * c + 16 * k, pk);   // waited for before p_full
               }
             }
             l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
@@ -442,11 +442,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pass_kernel(const __grid_const
                 ls[(2 * j + 1) & 3] += x1;
                 pk[j] = __byte_perm(__float_as_uint(x0) + 0x8000u, __float_as_uint(x1) + 0x8000u, 0x7632);
               }
-              tmem_st16(t_s + 16 * k, pk);
+              tmem_st16_nowait(t_s + 16 * k, pk);   // waited for before p_full
             }
             l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
           }
         }
+        tmem_wait_st();   // every P word in tensor memory before PV reads it
         tc_fence_before();
         mbar_arrive(&bars->p_full[wg]);
       }

@@ -266,8 +266,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
           if (j + 1 < s) dsum[(i + 2) & 3] = fmaf(p1, __uint_as_float(dr[2 * i + 1]), dsum[(i + 2) & 3]);
           pk[i] = pack2_rn(p0, p1);
         }
-        tmem_st16(t_row + 16 * c, pk);
+        tmem_st16_nowait(t_row + 16 * c, pk);   // waited for below, before P is read back
       }
+      tmem_wait_st();
       const float D = (dsum[0] + dsum[1]) + (dsum[2] + dsum[3]);
       lse_s[r] = tok >= 0 ? lse2 : INFINITY;   // +inf past the sequence: P = 0 in those columns
       d_s[r] = tok >= 0 ? D : 0.f;
@@ -285,8 +286,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
           const float s1 = j + 1 < s ? p1 * (__uint_as_float(dr[2 * i + 1]) - D) : 0.f;
           pk[i] = pack2_rn(s0, s1);
         }
-        tmem_st16(t_row + 16 * c, pk);
+        tmem_st16_nowait(t_row + 16 * c, pk);
       }
+      tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bars->p_full);
       ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->o_full, o_cnt & 1, ctl));
@@ -333,9 +335,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
             pp[i] = pack2_rn(p0, p1);
             ps[i] = pack2_rn(s0, s1);
           }
-          tmem_st16(t_row + 16 * c, pp);
-          tmem_st16(t_row + 128 + 16 * c, ps);
+          tmem_st16_nowait(t_row + 16 * c, pp);
+          tmem_st16_nowait(t_row + 128 + 16 * c, ps);
         }
+        tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&bars->p_full);
       }
