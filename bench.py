@@ -392,7 +392,7 @@ SWEEP = [
      ("local_then_global", "global_then_local", "local_only", "global_only"), True, True),
     ("Wan-2.1-1.3B block", 1, 12, 128, (21, 30, 52), (21, 2, 4), ("local_then_global", "global_then_local"), False, False),
     ("high-resolution 5B block", 1, 24, 128, (21, 44, 80), (21, 4, 4), ("local_then_global", "local_only", "global_only"),
-     True, False),
+     True, True),
     ("Wan-2.1-14B block (training step)", 1, 40, 128, (21, 22, 40), (21, 2, 4), ("local_then_global",), False, True),
     ("Wan-2.2-5B grid, window 21x3x4 (reflect-padded to 21x24x40)", 1, 24, 128, (21, 22, 40), (21, 3, 4),
      ("local_then_global",), False, True),
@@ -412,7 +412,8 @@ def sweep(reps=30, only=None, n_sets=3):
     the device, 3 rotating buffer sets, CUDA events on the launching stream."""
     import torch
 
-    from sub_quadratic_two_squad_b200 import full_attn_fwd, squad_attn_bwd, squad_attn_flops, squad_attn_fwd
+    from sub_quadratic_two_squad_b200 import (full_attn_fwd, squad_attn_bwd, squad_attn_bwd_kernels, squad_attn_flops,
+                                              squad_attn_fwd)
 
     dev = torch.device("cuda", 0)
     stream = torch.cuda.current_stream()
@@ -455,7 +456,8 @@ def sweep(reps=30, only=None, n_sets=3):
                                                      dv=g[2]), 10)
                 bwd_bytes = 8 * B * h * n * d * 2   # Q, K, V, O, dO in; dQ, dK, dV out (bf16), + O1 once
                 line["backward"] = {"ms_per_block": bms, "tflops_algorithmic": 2 * f / (bms * 1e-3) / 1e12,
-                                    "hbm_frac_8_tensors": bwd_bytes / (bms * 1e-3) / 1e9 / hbm}
+                                    "hbm_frac_8_tensors": bwd_bytes / (bms * 1e-3) / 1e9 / hbm,
+                                    "kernels": squad_attn_bwd_kernels(B, h, d, grid, window, order)}
             print(json.dumps(line), flush=True)
             del wss
         if with_full:

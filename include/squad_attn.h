@@ -125,6 +125,20 @@ SQUAD_API squad_status_t squad_attn_bwd(const squad_params_t* p, const void* q, 
                               void* dq, void* dk, void* dv, void* bwd_workspace,
                               squad_stream_t stream);
 
+/* The kernel each pass of squad_attn_bwd(p, ...) runs on, in execution order of the forward:
+ * kernels[0] for the first pass, kernels[1] for the second (0 when the order has one pass). The
+ * choice depends only on p (on the padded grid where the window does not divide it):
+ *   SQUAD_BWD_TC_WHOLE    tensor cores, one CTA per sequence (bf16, d = 128, sequences of at most
+ *                         about 216 tokens, whatever fits its shared-memory plan);
+ *   SQUAD_BWD_TC_CHUNKED  tensor cores, sequences cut into chunks of whole lines of at most 128 rows
+ *                         (bf16, d = 128, lines of at most 128 tokens): any sequence length;
+ *   SQUAD_BWD_CUDA_CORE   the fp32 CUDA-core kernels (fp32 inputs, other d).
+ * Enqueues nothing. SQUAD_ERR_INVALID_ARG / SQUAD_ERR_UNSUPPORTED as squad_attn_bwd would return. */
+#define SQUAD_BWD_TC_WHOLE 1
+#define SQUAD_BWD_TC_CHUNKED 2
+#define SQUAD_BWD_CUDA_CORE 3
+SQUAD_API squad_status_t squad_attn_bwd_kernels(const squad_params_t* p, int kernels[2]);
+
 /* Full softmax self-attention softmax(q k^T * scale) v over all n tokens per head (paper eq. 5),
  * the operator SQuad replaces. The window fields and `order` of *p are ignored (grid still gives n).
  * lse_or_null: optional [B,h,n] fp32 output of the natural-log log-sum-exp per query. This call has

@@ -12,6 +12,7 @@ from .api import (  # noqa: F401
     make_params,
     squad_attention,
     squad_attn_bwd,
+    squad_attn_bwd_kernels,
     squad_attn_bwd_workspace_bytes,
     squad_attn_flops,
     squad_window_solve,

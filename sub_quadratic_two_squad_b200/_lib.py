@@ -8,6 +8,7 @@ PKG_DIR = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG_DIR, "libsquad_attn.so")
 
 SQUAD_OK, SQUAD_ERR_INVALID_ARG, SQUAD_ERR_UNSUPPORTED, SQUAD_ERR_CUDA, SQUAD_ERR_TIMEOUT = range(5)
+SQUAD_BWD_TC_WHOLE, SQUAD_BWD_TC_CHUNKED, SQUAD_BWD_CUDA_CORE = 1, 2, 3
 SQUAD_BF16, SQUAD_FP32 = 0, 1
 SQUAD_LOCAL_THEN_GLOBAL, SQUAD_GLOBAL_THEN_LOCAL, SQUAD_LOCAL_ONLY, SQUAD_GLOBAL_ONLY = 0, 1, 2, 3
 SQUAD_NOALLOC_MAX_WORKSPACE_BYTES = 128 * 1024 * 1024
@@ -43,6 +44,7 @@ SIGNATURES = {
     "squad_attn_fwd_status": (ctypes.c_int, [_PP, _VP, _VP]),
     "squad_attn_bwd_workspace_bytes": (ctypes.c_size_t, [_PP]),
     "squad_attn_bwd": (ctypes.c_int, [_PP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
+    "squad_attn_bwd_kernels": (ctypes.c_int, [_PP, ctypes.POINTER(ctypes.c_int)]),
     "full_attn_fwd": (ctypes.c_int, [_PP, _VP, _VP, _VP, _VP, _VP, _VP]),
     "squad_attn_fwd_noalloc": (ctypes.c_int, [_PP, _VP, _VP, _VP, _VP, _VP]),
     "squad_attn_fwd_host_workspace_bytes": (ctypes.c_size_t, [_PP, ctypes.c_int]),

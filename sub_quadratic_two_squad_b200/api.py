@@ -147,6 +147,20 @@ def squad_attn_bwd(q, k, v, o, dout, fwd_workspace, grid, window, order="local_t
     return dq, dk, dv
 
 
+BWD_KERNEL_NAMES = {0: None, _lib.SQUAD_BWD_TC_WHOLE: "tc_whole", _lib.SQUAD_BWD_TC_CHUNKED: "tc_chunked",
+                    _lib.SQUAD_BWD_CUDA_CORE: "cuda_core"}
+
+
+def squad_attn_bwd_kernels(B, h, d, grid, window, order="local_then_global", dtype=torch.bfloat16):
+    """The backward kernel of each pass, in forward execution order: ("tc_whole" | "tc_chunked" |
+    "cuda_core", second pass or None)."""
+    ks = (ctypes.c_int * 2)()
+    st = _lib.load().squad_attn_bwd_kernels(ctypes.byref(make_params(B, h, d, grid, window, order, dtype)), ks)
+    if st != _lib.SQUAD_OK:
+        raise SquadError(st, "squad_attn_bwd_kernels")
+    return BWD_KERNEL_NAMES[ks[0]], BWD_KERNEL_NAMES[ks[1]]
+
+
 def full_attn_fwd(q, k, v, grid=None, scale=None, out=None, lse=None, stream=None):
     """softmax(q k^T * scale) v over all n tokens per head. Returns out (and fills `lse` if given)."""
     _check_qkv(q, k, v, out)

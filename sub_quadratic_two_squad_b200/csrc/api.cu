@@ -16,6 +16,7 @@
 #include "geometry.cuh"
 #include "kpass_plan.h"
 #include "bwd_pass.h"
+#include "bwd_stream.h"
 #include "pad.h"
 #include "short_pass.h"
 #include "simt_pass.h"
@@ -493,20 +494,36 @@ squad_status_t squad_attn_fwd_status(const squad_params_t* p, const void* worksp
 
 namespace {
 
-// One pass's backward inside a chain of passes. accumulate: add the fp32 dQ/dK shares already in the
-// accumulators; final_out: write dq, dk (input dtype) instead of the accumulators. dv_out receives the
-// gradient of this pass's values in the input dtype.
-squad_status_t bwd_one_pass(const squad_params_t* sp, const Grid& g, int kind, float scale, const void* q,
-                            const void* k, const void* values, const void* dout, const float* lse, uint32_t* status,
-                            float* dq_acc, float* dk_acc, float* drow, void* dq, void* dk, void* dv_out,
-                            bool accumulate, bool final_out, cudaStream_t stream) {
-  const bool bf16 = sp->dtype == SQUAD_BF16;
-  if (bf16) {
+// The backward kernel of one pass (SQUAD_BWD_*): whole sequences on the tensor cores where the
+// shared-memory plan fits, else chunks of whole lines on the tensor cores, else the CUDA cores.
+int bwd_kernel_of(const squad_params_t* sp, const Grid& g, int kind) {
+  if (sp->dtype == SQUAD_BF16) {
     BwdTcArgs b;
     std::memset(&b, 0, sizeof(b));
     b.g = g;
     b.p = make_geom(g, kind, 256);
-    if (short_eligible(sp, g, b.p) && bwd_tc_plan(b)) {
+    if (short_eligible(sp, g, b.p) && bwd_tc_plan(b)) return SQUAD_BWD_TC_WHOLE;
+    if (g.d == 128 && bwd_stream_eligible(g, make_geom(g, kind))) return SQUAD_BWD_TC_CHUNKED;
+  }
+  return SQUAD_BWD_CUDA_CORE;
+}
+
+// One pass's backward inside a chain of passes. accumulate: add the fp32 dQ/dK shares already in the
+// accumulators; final_out: write dq, dk (input dtype) instead of the accumulators. dv_out receives the
+// gradient of this pass's values in the input dtype; out is this pass's forward output (the chunked
+// kernels form D from it).
+squad_status_t bwd_one_pass(const squad_params_t* sp, const Grid& g, int kind, float scale, const void* q,
+                            const void* k, const void* values, const void* out, const void* dout, const float* lse,
+                            uint32_t* status, float* dq_acc, float* dk_acc, float* drow, void* dq, void* dk,
+                            void* dv_out, bool accumulate, bool final_out, cudaStream_t stream) {
+  const bool bf16 = sp->dtype == SQUAD_BF16;
+  const int kernel = bwd_kernel_of(sp, g, kind);
+  if (kernel == SQUAD_BWD_TC_WHOLE) {
+    BwdTcArgs b;
+    std::memset(&b, 0, sizeof(b));
+    b.g = g;
+    b.p = make_geom(g, kind, 256);
+    if (bwd_tc_plan(b)) {
       b.variant = kind == kGlobal ? kSlotBoxVariant : 0;
       if (!encode_pass_map(&b.tm_q, q, g, b.p, b.variant) || !encode_pass_map(&b.tm_k, k, g, b.p, b.variant) ||
           !encode_pass_map(&b.tm_v, values, g, b.p, b.variant) || !encode_pass_map(&b.tm_do, dout, g, b.p, b.variant))
@@ -525,6 +542,32 @@ squad_status_t bwd_one_pass(const squad_params_t* sp, const Grid& g, int kind, f
       b.timeout_ns = kWaitTimeoutNs;
       return launch_bwd_tc(b, stream) == cudaSuccess ? SQUAD_OK : SQUAD_ERR_CUDA;
     }
+  }
+  if (kernel == SQUAD_BWD_TC_CHUNKED) {
+    // Longer sequences: the chunked tensor-core kernels (D from the pass output `out`).
+    BwdStreamArgs s;
+    std::memset(&s, 0, sizeof(s));
+    s.g = g;
+    s.p = make_geom(g, kind);
+    s.variant = kind == kGlobal ? kSlotBoxVariant : 0;
+    if (!encode_pass_map(&s.tm_q, q, g, s.p, s.variant) || !encode_pass_map(&s.tm_k, k, g, s.p, s.variant) ||
+        !encode_pass_map(&s.tm_v, values, g, s.p, s.variant) ||
+        !encode_pass_map(&s.tm_do, dout, g, s.p, s.variant) || !encode_pass_map(&s.tm_o, out, g, s.p, s.variant))
+      return SQUAD_ERR_CUDA;
+    s.lse = lse;
+    s.drow = drow;
+    s.dq_acc = dq_acc;
+    s.dk_acc = dk_acc;
+    s.dq_out = static_cast<__nv_bfloat16*>(dq);
+    s.dk_out = static_cast<__nv_bfloat16*>(dk);
+    s.dv_out = static_cast<__nv_bfloat16*>(dv_out);
+    s.final_out = final_out ? 1 : 0;
+    s.accumulate = accumulate ? 1 : 0;
+    s.scale = scale;
+    s.scale_log2 = scale * 1.4426950408889634f;
+    s.status = status;
+    s.timeout_ns = kWaitTimeoutNs;
+    return launch_bwd_stream(s, stream) == cudaSuccess ? SQUAD_OK : SQUAD_ERR_CUDA;
   }
   SimtBwdArgs a{};
   a.q = q;
@@ -555,13 +598,12 @@ squad_status_t bwd_one_pass(const squad_params_t* sp, const Grid& g, int kind, f
 squad_status_t bwd_core(const squad_params_t* p, const Grid& g, float scale, const void* q, const void* k,
                         const void* v, const void* o, const void* dout, const FwdWorkspace& fw,
                         const BwdWorkspace& bw, void* dq, void* dk, void* dv, cudaStream_t stream) {
-  (void)o;   // D_i is formed from the recomputed P and dP, not from o
   const bool bf16 = p->dtype == SQUAD_BF16;
   if (p->order == SQUAD_LOCAL_ONLY || p->order == SQUAD_GLOBAL_ONLY) {
     // One pass: values v, upstream dout, the pass's LSE in the first slot; no share to add.
     const int kind = p->order == SQUAD_LOCAL_ONLY ? kLocal : kGlobal;
-    return bwd_one_pass(p, g, kind, scale, q, k, v, dout, fw.lse1, bw.status, bw.dq_acc, bw.dk_acc, bw.drow, dq,
-                        dk, dv, /*accumulate=*/false, /*final_out=*/true, stream);
+    return bwd_one_pass(p, g, kind, scale, q, k, v, o, dout, fw.lse1, bw.status, bw.dq_acc, bw.dk_acc, bw.drow,
+                        dq, dk, dv, /*accumulate=*/false, /*final_out=*/true, stream);
   }
   const int first = p->order == SQUAD_LOCAL_THEN_GLOBAL ? kLocal : kGlobal;
   const int second = p->order == SQUAD_LOCAL_THEN_GLOBAL ? kGlobal : kLocal;
@@ -606,6 +648,16 @@ squad_status_t bwd_core(const squad_params_t* p, const Grid& g, float scale, con
       if (launch_bwd_tc(b2, stream) != cudaSuccess) return SQUAD_ERR_CUDA;
       if (launch_bwd_tc(b1, stream) != cudaSuccess) return SQUAD_ERR_CUDA;
       return SQUAD_OK;
+    }
+    if (bwd_kernel_of(p, g, second) != SQUAD_BWD_CUDA_CORE || bwd_kernel_of(p, g, first) != SQUAD_BWD_CUDA_CORE) {
+      // Pass by pass, each on the kernel that takes its sequences (whole-sequence or chunked tensor
+      // cores); dO1 is bf16 as in the fused pair.
+      squad_status_t st = bwd_one_pass(p, g, second, scale, q, k, fw.o1, o, dout, fw.lse2, bw.status, bw.dq_acc,
+                                       bw.dk_acc, bw.drow, dq, dk, bw.do1, /*accumulate=*/false,
+                                       /*final_out=*/false, stream);
+      if (st != SQUAD_OK) return st;
+      return bwd_one_pass(p, g, first, scale, q, k, v, fw.o1, bw.do1, fw.lse1, bw.status, bw.dq_acc, bw.dk_acc,
+                          bw.drow, dq, dk, dv, /*accumulate=*/true, /*final_out=*/true, stream);
     }
   }
 
@@ -680,6 +732,25 @@ squad_status_t squad_attn_bwd(const squad_params_t* p, const void* q, const void
   if (launch_fold(bw.dqp, dq, ps, bf16, stream) != cudaSuccess || launch_fold(bw.dkp, dk, ps, bf16, stream) != cudaSuccess ||
       launch_fold(bw.dvp, dv, ps, bf16, stream) != cudaSuccess)
     return SQUAD_ERR_CUDA;
+  return SQUAD_OK;
+}
+
+squad_status_t squad_attn_bwd_kernels(const squad_params_t* p, int kernels[2]) {
+  Grid g;
+  float scale;
+  PadDims pd;
+  const squad_status_t st = validate(p, true, &g, &scale, &pd);
+  if (st != SQUAD_OK) return st;
+  if (kernels == nullptr) return SQUAD_ERR_INVALID_ARG;
+  kernels[0] = kernels[1] = 0;
+  if (p->order == SQUAD_LOCAL_ONLY || p->order == SQUAD_GLOBAL_ONLY) {
+    kernels[0] = bwd_kernel_of(p, g, p->order == SQUAD_LOCAL_ONLY ? kLocal : kGlobal);
+    return SQUAD_OK;
+  }
+  const int first = p->order == SQUAD_LOCAL_THEN_GLOBAL ? kLocal : kGlobal;
+  const int second = p->order == SQUAD_LOCAL_THEN_GLOBAL ? kGlobal : kLocal;
+  kernels[0] = bwd_kernel_of(p, g, first);
+  kernels[1] = bwd_kernel_of(p, g, second);
   return SQUAD_OK;
 }
 
@@ -855,7 +926,6 @@ squad_status_t squad_kpass_fwd(const squad_kpass_params_t* p, const void* q, con
 squad_status_t squad_kpass_bwd(const squad_kpass_params_t* p, const void* q, const void* k, const void* v,
                                const void* o, const void* dout, const void* fwd_workspace, void* dq, void* dk,
                                void* dv, void* bwd_workspace, squad_stream_t stream_) {
-  (void)o;   // each pass forms its softmax-Jacobian term from the recomputed P and dP
   KpassPlan pl;
   const squad_status_t st = kpass_plan(p, &pl);
   if (st != SQUAD_OK) return st;
@@ -874,7 +944,8 @@ squad_status_t squad_kpass_bwd(const squad_kpass_params_t* p, const void* q, con
     const void* values = st.values == kBufV ? v : fw.inter[st.values];
     const void* g_in = st.g_in == kBufDout ? dout : bw.gbuf[st.g_in];
     void* g_out = st.g_out == kBufDv ? dv : bw.gbuf[st.g_out];
-    const squad_status_t ps = bwd_one_pass(&pl.sub[l], pl.g[l], pl.kind[l], pl.scale, q, k, values, g_in,
+    const void* out = e + 1 == p->k ? o : fw.inter[e];   // this pass's output: the next pass's values
+    const squad_status_t ps = bwd_one_pass(&pl.sub[l], pl.g[l], pl.kind[l], pl.scale, q, k, values, out, g_in,
                                            fw.lse[st.lse], bw.ctrl, bw.dq_acc, bw.dk_acc, bw.drow, dq, dk, g_out,
                                            st.accumulate, st.final_out, stream);
     if (ps != SQUAD_OK) return ps;

@@ -204,3 +204,22 @@ def test_host_forward_rejects_bad_arguments_before_enqueueing(lib):
     assert call(h=ctypes.c_void_p(0)) == _lib.SQUAD_ERR_INVALID_ARG
     assert call(d=ctypes.c_void_p(8)) == _lib.SQUAD_ERR_INVALID_ARG             # not 16-byte aligned
     assert call(w=ctypes.c_void_p(128)) == _lib.SQUAD_ERR_INVALID_ARG           # not 256-byte aligned
+
+
+@pytest.mark.parametrize("grid,window,order,dtype,d,expect", [
+    ((21, 22, 40), (21, 2, 4), "local_then_global", 0, 128, (1, 1)),   # 168- and 110-token sequences: whole
+    ((21, 44, 80), (21, 4, 4), "local_then_global", 0, 128, (2, 2)),   # 336-token windows, 220-token slots
+    ((21, 8, 8), (21, 4, 4), "global_then_local", 0, 128, (1, 2)),     # 4-token slots, 336-token windows
+    ((5, 48, 48), (5, 2, 2), "global_only", 0, 128, (2, 0)),           # 576-token slot sequences
+    ((21, 22, 40), (21, 3, 4), "local_then_global", 0, 128, (2, 1)),   # padded to 21x24x40: 252-token windows
+    ((21, 22, 40), (21, 2, 4), "local_then_global", 0, 64, (3, 3)),    # d = 64: CUDA cores
+    ((5, 8, 8), (5, 2, 2), "local_then_global", 1, 128, (3, 3)),       # fp32: CUDA cores
+])
+def test_backward_kernel_selection(lib, grid, window, order, dtype, d, expect):
+    """Which backward kernel each pass takes is decided on the host from the parameters alone."""
+    ks = (ctypes.c_int * 2)()
+    prm = make_params(1, 2, d, grid, window, order, dtype)
+    assert lib.squad_attn_bwd_kernels(ctypes.byref(prm), ks) == _lib.SQUAD_OK
+    assert (ks[0], ks[1]) == expect
+    assert lib.squad_attn_bwd_kernels(ctypes.byref(prm), None) == _lib.SQUAD_ERR_INVALID_ARG
+    assert lib.squad_attn_bwd_kernels(ctypes.byref(make_params(1, 2, d, grid, (4, 2, 4), order, dtype)), ks) != 0

@@ -12,7 +12,8 @@ import pytest
 import torch
 
 from oracle import squad_oracle as orc
-from sub_quadratic_two_squad_b200 import full_attn_fwd, squad_attn_bwd, squad_attn_fwd, squad_attn_fwd_status
+from sub_quadratic_two_squad_b200 import (full_attn_fwd, squad_attn_bwd, squad_attn_bwd_kernels, squad_attn_fwd,
+                                          squad_attn_fwd_status)
 from sub_quadratic_two_squad_b200.inputs import make_inputs
 
 pytestmark = pytest.mark.gpu
@@ -184,9 +185,40 @@ def test_backward_small_bf16(order):
     run_bwd(2, 2, 128, (21, 4, 8), (21, 2, 4), order, torch.bfloat16)
 
 
-def test_backward_bf16_long_windows_cuda_core_path():
-    """336-token windows: beyond the tensor-core backward's shared memory, so the CUDA-core kernels run."""
-    run_bwd(1, 1, 128, (21, 8, 8), (21, 4, 4), LG, torch.bfloat16)
+def _bwd_kernels(h, grid, window, order):
+    return squad_attn_bwd_kernels(1, h, 128, grid, window, order, torch.bfloat16)
+
+
+@pytest.mark.parametrize("order", [LG, GL])
+def test_backward_bf16_long_windows_chunked_tensor_cores(order):
+    """336-token windows (3 chunks of 8, 8 and 5 lines of 16 tokens) on the chunked tensor-core kernels;
+    the 4-token slot sequences on the whole-sequence one."""
+    ks = _bwd_kernels(1, (21, 8, 8), (21, 4, 4), order)
+    assert ks == (("tc_chunked", "tc_whole") if order == LG else ("tc_whole", "tc_chunked"))
+    run_bwd(1, 1, 128, (21, 8, 8), (21, 4, 4), order, torch.bfloat16)
+
+
+@pytest.mark.parametrize("order", [GO, LG])
+def test_backward_bf16_long_slot_sequences_chunked(order):
+    """576-token slot sequences (24 lines of 24 tokens: chunks of 5 lines, the last one 4) on the chunked
+    kernels, alone and after a 20-token local pass."""
+    ks = _bwd_kernels(2, (5, 48, 48), (5, 2, 2), order)
+    assert ks == (("tc_chunked", None) if order == GO else ("tc_whole", "tc_chunked"))
+    run_bwd(1, 2, 128, (5, 48, 48), (5, 2, 2), order, torch.bfloat16)
+
+
+def test_backward_hires_5b_chunked():
+    """The high-resolution 5B block (21x44x80, window 21x4x4): 336-token windows and 220-token slot
+    sequences, both passes on the chunked tensor-core kernels (2 heads, every element)."""
+    assert _bwd_kernels(2, (21, 44, 80), (21, 4, 4), LG) == ("tc_chunked", "tc_chunked")
+    run_bwd(1, 2, 128, (21, 44, 80), (21, 4, 4), LG, torch.bfloat16)
+
+
+def test_backward_padded_window_21x3x4_chunked():
+    """The 5B grid with a 21x3x4 window, reflect-padded to 21x24x40: 252-token windows in chunks of 10,
+    10 and 1 lines of 12 tokens (a 12-row last chunk)."""
+    assert _bwd_kernels(2, (21, 22, 40), (21, 3, 4), LG) == ("tc_chunked", "tc_whole")
+    run_bwd(1, 2, 128, (21, 22, 40), (21, 3, 4), LG, torch.bfloat16)
 
 
 def test_backward_wan21_14b():

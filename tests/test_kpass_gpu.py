@@ -24,6 +24,8 @@ CASES = [
     (1, 2, 128, (3, 8, 8), [(8, 8)], BF16),                         # k = 1: full attention over 192 tokens
     (1, 3, 128, (21, 4, 8), [(2, 4), (2, 2)], BF16),                # k = 2: the two-pass problem
     (1, 1, 128, (2, 20, 40), [(2, 2), (10, 10), (1, 2)], BF16),     # a 100-token middle level, 2-token outer
+    (1, 2, 128, (21, 16, 16), [(4, 4), (2, 2), (2, 2)], BF16),      # 336-token first level: chunked backward
+    (1, 2, 128, (2, 32, 32), [(2, 2), (16, 16)], BF16),             # 256-token outer level: chunked backward
 ]
 
 
