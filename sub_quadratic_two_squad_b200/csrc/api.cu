@@ -529,6 +529,7 @@ squad_status_t bwd_one_pass(const squad_params_t* sp, const Grid& g, int kind, f
           !encode_pass_map(&b.tm_v, values, g, b.p, b.variant) || !encode_pass_map(&b.tm_do, dout, g, b.p, b.variant))
         return SQUAD_ERR_CUDA;
       b.lse = lse;
+      b.o = static_cast<const __nv_bfloat16*>(out);
       b.dq_acc = dq_acc;
       b.dk_acc = dk_acc;
       b.dq_out = static_cast<__nv_bfloat16*>(dq);
@@ -637,9 +638,11 @@ squad_status_t bwd_core(const squad_params_t* p, const Grid& g, float scale, con
         b->timeout_ns = kWaitTimeoutNs;
       }
       b2.lse = fw.lse2;
+      b2.o = static_cast<const __nv_bfloat16*>(o);
       b2.dv_out = do1;
       b2.final_out = 0;
       b1.lse = fw.lse1;
+      b1.o = static_cast<const __nv_bfloat16*>(fw.o1);
       b1.dq_out = static_cast<__nv_bfloat16*>(dq);
       b1.dk_out = static_cast<__nv_bfloat16*>(dk);
       b1.dv_out = static_cast<__nv_bfloat16*>(dv);

@@ -16,6 +16,7 @@ struct BwdTcArgs {
   PassGeom p;                 // one chunk per sequence (make_geom(..., 256))
   int variant;                // slot-box encoding (GLOBAL pass)
   const float* lse;           // [B, h, n] natural-log LSE of this pass's forward
+  const __nv_bfloat16* o;     // [B, h, n, d] this pass's output (D_i = dO_i . O_i)
   float* dq_acc;              // [B, h, n, d] fp32 share of dQ: written, added to (accumulate), or read
                               // and completed (final_out with accumulate)
   float* dk_acc;              // [B, h, n, d] fp32 share of dK (likewise)

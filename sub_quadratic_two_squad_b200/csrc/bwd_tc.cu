@@ -4,18 +4,22 @@
 // local pass, a slot across windows for the global pass; SQuad paper §3.2), so its gradients are those
 // of softmax attention, sequence by sequence (agihunt.info digest, the paragraph that defines the
 // operator; the chain rule through both passes is applied by the caller). With
-// P = softmax(scale Q K^T) recomputed from the forward's LSE, dO the gradient of the pass output:
-//   dP = dO V^T,  D_i = sum_j P_ij dP_ij,  dS = P o (dP - D),
+// P = softmax(scale Q K^T) recomputed from the forward's LSE, O the pass output and dO its gradient:
+//   dP = dO V^T,  D_i = sum_j P_ij dP_ij = dO_i . O_i,  dS = P o (dP - D),
 //   dQ = scale dS K,  dK = scale dS^T Q,  dV = P^T dO.
 //
 // One kernel per pass, one CTA per sequence (160 threads): warps 0-3 own one TMEM lane (one row) per
-// thread, warp 4 loads the sequence's Q, K, V, dO once as whole TMA boxes and issues the tcgen05 MMAs.
-//   rows, per 128-query tile: S = Q K^T and dP = dO V^T into TMEM; the warps form P (bf16) and D, then
-//     dS (bf16, packed two per column over S); dQ = dS K (A from TMEM) is written out. Each row's LSE
-//     and D stay in shared memory.
+// thread, warp 4 loads the sequence's Q, K (first) and V, dO once as whole TMA boxes and issues the
+// tcgen05 MMAs.
+//   rows, per 128-query tile: each warp forms D from its rows of dO (shared memory) and O (global)
+//     while S = Q K^T and dP = dO V^T go into TMEM; then dS = P o (dP - D) in one pass over the
+//     scores (bf16, packed two per column over S); dQ = dS K (A from TMEM) is written out. Each row's
+//     LSE and D stay in shared memory. Where tensor memory has room, dQ has columns of its own, so the
+//     next tile's S and dP (or the first S^T and dP^T) are computed while it is written out.
 //   columns, per 128-key tile and 128-query chunk: S^T = K Q^T and dP^T = V dO^T into TMEM; with the
 //     per-query LSE and D the warps form P^T and dS^T (packed over S^T and dP^T); dV += P^T dO and
-//     dK += dS^T Q accumulate in TMEM over the chunks and are written out.
+//     dK += dS^T Q accumulate in TMEM over the chunks and are written out (the next key tile's S^T
+//     and dP^T are computed meanwhile).
 // Rows past the sequence are computed and dropped; columns past it are masked to P = dS = 0, and the
 // shared-memory rows past each box are zeroed so every MMA operand is finite.
 #include <cuda_runtime.h>
@@ -38,7 +42,7 @@ constexpr uint32_t kBwdSmemMin = 120u * 1024u;
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct BwdBars {
-  uint64_t load, s_full, p_full, o_full, o_free, drain;
+  uint64_t load_qk, load_vd, s_full, p_full, o_full, o_free, drain;
   uint32_t tmem_base;
   uint32_t abort;
 };
@@ -47,6 +51,29 @@ static_assert(sizeof(BwdBars) <= kBwdBarBytes, "barrier block");
 constexpr uint32_t kBwdVecBytes = 2u * 256u * 4u;   // per-query LSE (log2 units) and D, column kernel
 
 __device__ __forceinline__ int round16b(int x) { return (x + 15) & ~15; }
+
+// dQ gets tensor-memory columns of its own, [384, 512), where S and dP ([0, 2N)) leave them free;
+// they are also clear of the column phase's S^T and dP^T ([0, 256)).
+__device__ __forceinline__ bool dq_own_columns(int N) { return 2 * N <= 384; }
+
+// D = dO_r . O_r in fp32: row r of the dO tile (bf16, 128-byte swizzle, two 64-column panels `panel`
+// bytes apart) against the row's output held as 16 x 8 bf16 (columns 8i .. 8i + 7 in o[i]).
+__device__ __forceinline__ float row_dot_out(const uint8_t* sdo, uint32_t panel, int r, const uint4 (&o)[16]) {
+  float acc[2] = {0.f, 0.f};
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const uint32_t pnl = static_cast<uint32_t>(i >> 3), c = static_cast<uint32_t>(i & 7);
+    const uint4 x = *reinterpret_cast<const uint4*>(sdo + pnl * panel + static_cast<uint32_t>(r) * 128u +
+                                                    ((c ^ static_cast<uint32_t>(r & 7)) << 4));
+    const uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {o[i].x, o[i].y, o[i].z, o[i].w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      acc[k & 1] = fmaf(__uint_as_float(xs[k] << 16), __uint_as_float(ys[k] << 16), acc[k & 1]);
+      acc[k & 1] = fmaf(__uint_as_float(xs[k] & 0xFFFF0000u), __uint_as_float(ys[k] & 0xFFFF0000u), acc[k & 1]);
+    }
+  }
+  return acc[0] + acc[1];
+}
 
 __device__ __forceinline__ uint32_t pack2_rn(float lo, float hi) { return pack_bf16x2(lo, hi); }
 
@@ -127,7 +154,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
       reinterpret_cast<uint4*>(base + 4 * alloc)[i] = make_uint4(0, 0, 0, 0);
   }
   if (threadIdx.x == 128) {
-    mbar_init(&bars->load, 1);
+    mbar_init(&bars->load_qk, 1);
+    mbar_init(&bars->load_vd, 1);
     mbar_init(&bars->s_full, 1);
     mbar_init(&bars->p_full, 128);
     mbar_init(&bars->o_full, 1);
@@ -162,34 +190,45 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
       prefetch_tmap(&a.tm_k);
       prefetch_tmap(&a.tm_v);
       prefetch_tmap(&a.tm_do);
-      mbar_arrive_expect_tx(&bars->load, 8u * static_cast<uint32_t>(s) * 128u);
+      const uint32_t tx_half = 4u * static_cast<uint32_t>(s) * 128u;   // two tensors, both panels
+      mbar_arrive_expect_tx(&bars->load_qk, tx_half);
+      mbar_arrive_expect_tx(&bars->load_vd, tx_half);
       int c[5];
       chunk_coords(g, p, a.variant, bh, sigma, 0, 0, c);
       const CUtensorMap* maps[4] = {&a.tm_q, &a.tm_k, &a.tm_v, &a.tm_do};
       uint8_t* dsts[4] = {sq, sk, sv, sdo};
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        tma_load_5d(dsts[i], maps[i], &bars->load, c[0], c[1], c[2], c[3], c[4]);
-        tma_load_5d(dsts[i] + panel, maps[i], &bars->load, c[0] + 64, c[1], c[2], c[3], c[4]);
+        uint64_t* bar = i < 2 ? &bars->load_qk : &bars->load_vd;
+        tma_load_5d(dsts[i], maps[i], bar, c[0], c[1], c[2], c[3], c[4]);
+        tma_load_5d(dsts[i] + panel, maps[i], bar, c[0] + 64, c[1], c[2], c[3], c[4]);
       }
-      bool ok = mbar_wait(&bars->load, 0, ctl);
+      bool ok = mbar_wait(&bars->load_qk, 0, ctl);
       tc_fence_after();
       const uint32_t aq = smem_u32(sq), ak = smem_u32(sk), av = smem_u32(sv), ado = smem_u32(sdo);
       uint32_t p_cnt = 0, f_cnt = 0;
-      // the row owners have read the previous tile's results out of tensor memory
+      // the row owners have read the previous results (dQ, or dV and dK) out of tensor memory
       auto wait_free = [&]() -> bool {
         const bool r = mbar_wait(&bars->o_free, f_cnt & 1, ctl);
         ++f_cnt;
         if (r) tc_fence_after();
         return r;
       };
-      // rows: per 128-query tile, S and dP, then dQ = dS K
+      // rows: per 128-query tile, S and dP, then dQ = dS K into [qcol, qcol + 128)
       const uint32_t idesc_s = idesc_bf16(128, N, false);
+      const bool own_dq = dq_own_columns(N);
+      const uint32_t qcol = own_dq ? 384u : static_cast<uint32_t>(N);
       for (int t = 0; t < ntiles && ok; ++t) {
-        if (t > 0 && !(ok = wait_free())) break;
+        // dQ over dP's columns: the previous tile's dQ must have been read before S and dP are written
+        if (t > 0 && !own_dq && !(ok = wait_free())) break;
         const uint32_t row_off = static_cast<uint32_t>(t) * 16384u;
         for (int kk = 0; kk < 8; ++kk)   // S = Q_t K^T -> [0, N)
           umma_bf16_ss(tmem, kdesc(aq + row_off, kk, panel), kdesc(ak, kk, panel), idesc_s, kk > 0);
+        if (t == 0) {
+          ok = mbar_wait(&bars->load_vd, 0, ctl);
+          if (!ok) break;
+          tc_fence_after();
+        }
         for (int kk = 0; kk < 8; ++kk)   // dP = dO_t V^T -> [N, 2N)
           umma_bf16_ss(tmem + N, kdesc(ado + row_off, kk, panel), kdesc(av, kk, panel), idesc_s, kk > 0);
         umma_commit(&bars->s_full);
@@ -197,13 +236,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
         ++p_cnt;
         if (!ok) break;
         tc_fence_after();
-        for (int kk = 0; kk < N / 16; ++kk)   // dQ = dS K -> [N, N + 128)
-          umma_bf16_ts(tmem + N, tmem + kk * 8, sw128_desc(ak + kk * 2048, panel, 1024), idesc_o, kk > 0);
+        // dQ in columns of its own: only the previous tile's dQ must have been read
+        if (t > 0 && own_dq && !(ok = wait_free())) break;
+        for (int kk = 0; kk < N / 16; ++kk)   // dQ = dS K
+          umma_bf16_ts(tmem + qcol, tmem + kk * 8, sw128_desc(ak + kk * 2048, panel, 1024), idesc_o, kk > 0);
         umma_commit(&bars->o_full);
       }
-      // columns: per 128-key tile, over 128-query chunks, S^T and dP^T, then dV += P^T dO, dK += dS^T Q
+      // columns: per 128-key tile, over 128-query chunks, S^T and dP^T, then dV += P^T dO, dK += dS^T Q.
+      // S^T and dP^T ([0, 256)) wait for the last dQ only where it overlaps them; dV and dK ([256, 512))
+      // wait for the last dQ, or the previous key tile's dV and dK, to have been read.
+      bool pending = ok;   // an o_full whose o_free has not been waited for
       for (int kt = 0; kt < ntiles && ok; ++kt) {
-        if (!(ok = wait_free())) break;   // tensor memory free (the last dQ, or the previous dV and dK, read)
+        if (kt == 0 && !own_dq) {
+          if (!(ok = wait_free())) break;
+          pending = false;
+        }
         const uint32_t key_off = static_cast<uint32_t>(kt) * 16384u;
         for (int qc = 0; qc < ntiles && ok; ++qc) {
           const int nq = min(128, s - 128 * qc);
@@ -220,6 +267,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
           ++p_cnt;
           if (!ok) break;
           tc_fence_after();
+          if (qc == 0 && pending) {
+            if (!(ok = wait_free())) break;
+            pending = false;
+          }
           for (int kk = 0; kk < Nq / 16; ++kk)   // dV += P^T dO_qc -> [256, 384)
             umma_bf16_ts(tmem + 256, tmem + kk * 8, sw128_desc(ado + q_off + kk * 2048, panel, 1024), idesc_o,
                          qc > 0 || kk > 0);
@@ -227,7 +278,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
             umma_bf16_ts(tmem + 384, tmem + 128 + kk * 8, sw128_desc(aq + q_off + kk * 2048, panel, 1024), idesc_o,
                          qc > 0 || kk > 0);
         }
-        if (ok) umma_commit(&bars->o_full);
+        if (ok) {
+          umma_commit(&bars->o_full);
+          pending = true;
+        }
       }
       // every MMA issued has completed before the CTA frees tensor memory
       umma_commit(&bars->drain);
@@ -240,18 +294,32 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
     const float sl2 = a.scale_log2;
     uint32_t s_cnt = 0, o_cnt = 0;
     bool ok = true;
-    // rows: P and D, dS, dQ; each row's LSE (log2 units) and D go to shared memory for the columns
+    // rows: D, dS, dQ; each row's LSE (log2 units) and D go to shared memory for the columns
+    const uint32_t qcol = dq_own_columns(N) ? 384u : static_cast<uint32_t>(N);
     for (int t = 0; t < ntiles && ok; ++t) {
       const int r = 128 * t + rl;
       const int tok = r < s ? token_of(g, p, sigma, 0, r) : -1;
       const size_t gi = static_cast<size_t>(bh) * g.n + (tok < 0 ? 0 : tok);
       const float lse2 = tok >= 0 ? a.lse[gi] * kLog2e : 0.f;
+      // D_i = dO_i . O_i: the row's output from global memory, its dO row from shared memory
+      uint4 orow[16];
+      {
+        const uint4* src = reinterpret_cast<const uint4*>(a.o + gi * 128);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) orow[i] = tok >= 0 ? src[i] : make_uint4(0, 0, 0, 0);
+      }
+      if (t == 0) {
+        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->load_vd, 0, ctl));
+        if (!ok) break;
+      }
+      const float D = tok >= 0 ? row_dot_out(sdo, panel, r, orow) : 0.f;
+      lse_s[r] = tok >= 0 ? lse2 : INFINITY;   // +inf past the sequence: P = 0 in those columns
+      d_s[r] = D;
       ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->s_full, s_cnt & 1, ctl));   // warp-uniform exit
       ++s_cnt;
       if (!ok) break;
       tc_fence_after();
-      // P (bf16, packed over the S columns already read) and D = sum_j P_ij dP_ij
-      float dsum[4] = {0.f, 0.f, 0.f, 0.f};
+      // dS = P o (dP - D), P recomputed from S and the LSE; bf16, packed over the S columns already read
 #pragma unroll 1
       for (int c = 0; c < (N + 31) / 32; ++c) {
         uint32_t sr[32], dr[32], pk[16];
@@ -262,31 +330,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
           const int j = 32 * c + 2 * i;
           const float p0 = j < s ? ex2_approx(fmaf(__uint_as_float(sr[2 * i]), sl2, -lse2)) : 0.f;
           const float p1 = j + 1 < s ? ex2_approx(fmaf(__uint_as_float(sr[2 * i + 1]), sl2, -lse2)) : 0.f;
-          if (j < s) dsum[i & 3] = fmaf(p0, __uint_as_float(dr[2 * i]), dsum[i & 3]);
-          if (j + 1 < s) dsum[(i + 2) & 3] = fmaf(p1, __uint_as_float(dr[2 * i + 1]), dsum[(i + 2) & 3]);
-          pk[i] = pack2_rn(p0, p1);
-        }
-        tmem_st16_nowait(t_row + 16 * c, pk);   // waited for below, before P is read back
-      }
-      tmem_wait_st();
-      const float D = (dsum[0] + dsum[1]) + (dsum[2] + dsum[3]);
-      lse_s[r] = tok >= 0 ? lse2 : INFINITY;   // +inf past the sequence: P = 0 in those columns
-      d_s[r] = tok >= 0 ? D : 0.f;
-      // dS = P o (dP - D), packed over P
-#pragma unroll 1
-      for (int c = 0; c < (N + 31) / 32; ++c) {
-        uint32_t pr[16], dr[32], pk[16];
-        tmem_ld16(t_row + 16 * c, pr);
-        tmem_ld32(t_row + N + 32 * c, dr);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int j = 32 * c + 2 * i;
-          const float p0 = __uint_as_float(pr[i] << 16), p1 = __uint_as_float(pr[i] & 0xFFFF0000u);
           const float s0 = j < s ? p0 * (__uint_as_float(dr[2 * i]) - D) : 0.f;
           const float s1 = j + 1 < s ? p1 * (__uint_as_float(dr[2 * i + 1]) - D) : 0.f;
           pk[i] = pack2_rn(s0, s1);
         }
-        tmem_st16_nowait(t_row + 16 * c, pk);
+        tmem_st16_nowait(t_row + 16 * c, pk);   // waited for below, before the MMA reads dS
       }
       tmem_wait_st();
       tc_fence_before();
@@ -298,9 +346,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
       {
         const size_t ro = gi * 128;
         if (a.final_out)
-          write_row(t_row + N, tok >= 0, a.scale, a.accumulate ? a.dq_acc + ro : nullptr, a.dq_out + ro, nullptr);
+          write_row(t_row + qcol, tok >= 0, a.scale, a.accumulate ? a.dq_acc + ro : nullptr, a.dq_out + ro, nullptr);
         else
-          write_row(t_row + N, tok >= 0, a.scale, a.accumulate ? a.dq_acc + ro : nullptr, nullptr, a.dq_acc + ro);
+          write_row(t_row + qcol, tok >= 0, a.scale, a.accumulate ? a.dq_acc + ro : nullptr, nullptr, a.dq_acc + ro);
       }
       tc_fence_before();
       mbar_arrive(&bars->o_free);
