@@ -13,12 +13,13 @@
 //   warp 10     TMA store issuer for the outputs.
 // A work unit is a pair of 128-row query tiles, one per softmax warpgroup; when both belong to the
 // same sequence they share every K/V block. Per warpgroup, tensor memory holds the scores S (128 fp32
-// columns) and the output accumulator O (128 columns). A softmax thread owns one query row: it loads
-// the row's 128 scores with one tcgen05.ld, writes P as bf16 over the first half of S, and the PV
+// columns) and the output accumulator O (128 columns). A softmax thread owns one query row: it reads
+// the row's 128 scores in two 64-column loads, writes P as bf16 over the first half of S, and the PV
 // product reads it from there (tcgen05.mma with A in tensor memory); the MMA issue order per
 // warpgroup is ... S(b), [softmax], PV(b), S(b+1) ..., so the in-order tensor pipe finishes reading
-// P(b) before S(b+1) overwrites it. Softmax is online across K/V blocks; the rescale of O is skipped
-// unless the row maximum grew by more than 2^8. The epilogue stages O through the tile's own Q buffer
+// P(b) before S(b+1) overwrites it. Softmax is online across K/V blocks in one pass over each block's
+// scores: the reference maximum, and with it O, changes only when a score exceeds it by more than
+// 2^64 (in practice within the first block). The epilogue stages O through the tile's own Q buffer
 // (free once its last S is done); the store warp writes it back with a TMA store of the same chunk
 // box, which scatters the rows to their tokens and drops the padding rows.
 #include <cuda_runtime.h>
@@ -78,7 +79,6 @@ __device__ __forceinline__ int pos_v(int b, int nb) { return b == nb - 1 ? 2 * n
 
 }  // namespace
 
-template <bool kSplitRows>
 __global__ void __launch_bounds__(kThreads, 1) tc_pass_kernel(const __grid_constant__ TcPassArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -313,139 +313,81 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pass_kernel(const __grid_const
         ++s_cnt;
         if (!ok) break;
         tc_fence_after();   // S(b) is ready, and so is every earlier PV (in-order tensor pipe)
-        if constexpr (kSplitRows) {
-          // Short sequences: the block's scores are read in 64-column halves (twice), so the softmax
-          // stays within the register budget.
-          const int valid = chunk_valid_rows(p, b);
-          float m_new = m_used;
-          if (active) {
-            // row maximum over the block, 64 columns at a time (4 independent partial maxima; the scale
-            // is positive, so it is applied to the maximum instead of to every score)
-            float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-  #pragma unroll
-            for (int c = 0; c < 2; ++c) {
-              uint32_t r[64];
-              tmem_ld64(t_s + 64 * c, r);
-  #pragma unroll
+        const int valid = chunk_valid_rows(p, b);
+        if (active) {
+          // One pass over the block's scores, 64 columns at a time, against a reference maximum m_used
+          // (log2 units) that is raised only when a chunk's maximum exceeds it by more than 2^kHeadroom:
+          // until then P = 2^(x - m_used) <= 2^kHeadroom is exact in fp32 and bf16 (the normalisation by
+          // the row sum cancels m_used), and |O| <= n 2^kHeadroom max|V| stays far inside fp32 for any
+          // n < 2^31. Raising m_used scales the P words already written in this block, the partial sums
+          // and O by 2^(m_old - m_new), each row by its own factor (1 for rows that keep theirs); the
+          // warp takes that path together (tensor-memory accesses are warp-wide). The first chunk of the
+          // first block sets m_used (it holds at least one valid column, so its maximum is finite).
+          constexpr float kHeadroom = 64.f;
+          float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+          for (int c = 0; c < 2; ++c) {
+            uint32_t r[64];
+            tmem_ld64(t_s + 64 * c, r);
+            if (64 * c + 64 > valid) {
+#pragma unroll
               for (int i = 0; i < 64; ++i)
-                if (64 * c + i < valid) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(r[i]));
+                if (64 * c + i >= valid) r[i] = __float_as_uint(-INFINITY);
             }
-            m_new = fmaxf(m_used, fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2);
-          }
-          if (b > 0) {
-            // Rescale O only when the running maximum grew by more than 2^8 (until then the unscaled
-            // exponentials stay below 256). PV(b-1) has completed: S(b) was issued after it.
-            const bool need = active && m_new > m_used + 8.f;
-            if (__any_sync(0xffffffffu, need)) {
-              const float f = need ? ex2_approx(m_used - m_new) : 1.f;
-  #pragma unroll
-              for (int c = 0; c < 2; ++c) {
-                uint32_t o[64];
-                tmem_ld64(t_o + 64 * c, o);
-  #pragma unroll
-                for (int i = 0; i < 64; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
-                tmem_st64v(t_o + 64 * c, o);
-              }
-              if (need) {
-                l *= f;
-                m_used = m_new;
-              }
-            }
-          } else {
-            m_used = m_new;
-          }
-          if (active) {
-            // P = 2^(x - m) (masked columns give 0), rounded to bf16 on the integer pipe (add half an ulp,
-            // keep the high half), packed two per 32-bit word over the first 64 TMEM columns of S: the
-            // packed half of a 64-column chunk lands on columns already read.
-            const float nm = -m_used;
-            float ls[4] = {0.f, 0.f, 0.f, 0.f};
-  #pragma unroll 1
-            for (int c = 0; c < 2; ++c) {
-              uint32_t r[64];
-              tmem_ld64(t_s + 64 * c, r);
-  #pragma unroll
-              for (int k = 0; k < 2; ++k) {
-                uint32_t pk[16];
-  #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                  const int i0 = 32 * k + 2 * j;
-                  const float x0 = 64 * c + i0 < valid ? ex2_approx(fmaf(__uint_as_float(r[i0]), sl2, nm)) : 0.f;
-                  const float x1 = 64 * c + i0 + 1 < valid ? ex2_approx(fmaf(__uint_as_float(r[i0 + 1]), sl2, nm)) : 0.f;
-                  ls[(2 * j) & 3] += x0;
-                  ls[(2 * j + 1) & 3] += x1;
-                  pk[j] = __byte_perm(__float_as_uint(x0) + 0x8000u, __float_as_uint(x1) + 0x8000u, 0x7632);
-                }
-                tmem_st16_nowait(t_s + 32 * c + 16 * k, pk);   // waited for before p_full
-              }
-            }
-            l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-          }
-        } else {
-          // Long sequences (full attention): the 128 scores are read once into registers.
-          const int valid = chunk_valid_rows(p, b);
-          uint32_t r[128];
-          float m_new = m_used;
-          if (active) {
-            tmem_ld128(t_s, r);
-            if (valid < 128)
-  #pragma unroll
-              for (int i = 0; i < 128; ++i)
-                if (i >= valid) r[i] = __float_as_uint(-INFINITY);
-            // row maximum (4 independent partial maxima; the scale is positive, so it is applied to the
-            // maximum instead of to every score)
+            // the scale is positive, so it is applied to the maximum instead of to every score
             float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-  #pragma unroll
-            for (int i = 0; i < 128; ++i) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(r[i]));
-            m_new = fmaxf(m_used, fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2);
-          }
-          if (b > 0) {
-            // Rescale O only when the running maximum grew by more than 2^8 (until then the unscaled
-            // exponentials stay below 256). PV(b-1) has completed: S(b) was issued after it. This path is
-            // rare, so it reuses the score registers for O and reloads S afterwards.
-            const bool need = active && m_new > m_used + 8.f;
-            if (__any_sync(0xffffffffu, need)) {
-              const float f = need ? ex2_approx(m_used - m_new) : 1.f;
-              tmem_ld128(t_o, r);
-  #pragma unroll
-              for (int i = 0; i < 128; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * f);
-              tmem_st128(t_o, r);
-              if (need) {
-                l *= f;
-                m_used = m_new;
+#pragma unroll
+            for (int i = 0; i < 64; ++i) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(r[i]));
+            const float cm = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;
+            if (__any_sync(0xFFFFFFFFu, cm > m_used + kHeadroom)) {
+              const float m_new = cm > m_used + kHeadroom ? cm : m_used;
+              const float f = m_new > m_used ? ex2_approx(m_used - m_new) : 1.f;   // 0 while m_used is -inf
+              tmem_wait_st();   // this block's P words written so far have landed
+              if (c > 0) {
+                uint32_t pw[16];
+#pragma unroll 1
+                for (int cc = 0; cc < 2; ++cc) {
+                  tmem_ld16(t_s + 16 * cc, pw);
+#pragma unroll
+                  for (int j = 0; j < 16; ++j) {
+                    const float x0 = __uint_as_float(pw[j] << 16) * f;
+                    const float x1 = __uint_as_float(pw[j] & 0xFFFF0000u) * f;
+                    pw[j] = __byte_perm(__float_as_uint(x0) + 0x8000u, __float_as_uint(x1) + 0x8000u, 0x7632);
+                  }
+                  tmem_st16(t_s + 16 * cc, pw);
+                }
               }
-              if (active) {
-                tmem_ld128(t_s, r);
-                if (valid < 128)
-  #pragma unroll
-                  for (int i = 0; i < 128; ++i)
-                    if (i >= valid) r[i] = __float_as_uint(-INFINITY);
+              if (b > 0) {
+                // O of the earlier blocks: PV(b-1) has completed (S(b) was issued after it)
+#pragma unroll 1
+                for (int h = 0; h < 2; ++h) {
+                  uint32_t o[64];
+                  tmem_ld64(t_o + 64 * h, o);
+#pragma unroll
+                  for (int i = 0; i < 64; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
+                  tmem_st64v(t_o + 64 * h, o);
+                }
               }
+#pragma unroll
+              for (int i = 0; i < 4; ++i) ls[i] *= f;
+              l *= f;
+              m_used = m_new;
             }
-          } else {
-            m_used = m_new;
-          }
-          if (active) {
-            // P = 2^(x - m) (masked columns give 2^-inf = 0), rounded to bf16 on the integer pipe (add half
-            // an ulp, keep the high half), packed two per 32-bit word and stored 32 scores at a time over
-            // the first 64 TMEM columns of S (the scores are already in registers).
+            // P = 2^(x - m_used) (masked columns give 0), rounded to bf16 on the integer pipe (add half an
+            // ulp, keep the high half), packed two per 32-bit word over columns already read
             const float nm = -m_used;
-            float ls[4] = {0.f, 0.f, 0.f, 0.f};
-  #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              uint32_t pk[16];
-  #pragma unroll
-              for (int j = 0; j < 16; ++j) {
-                const float x0 = ex2_approx(fmaf(__uint_as_float(r[32 * k + 2 * j]), sl2, nm));
-                const float x1 = ex2_approx(fmaf(__uint_as_float(r[32 * k + 2 * j + 1]), sl2, nm));
-                ls[(2 * j) & 3] += x0;
-                ls[(2 * j + 1) & 3] += x1;
-                pk[j] = __byte_perm(__float_as_uint(x0) + 0x8000u, __float_as_uint(x1) + 0x8000u, 0x7632);
-              }
-              tmem_st16_nowait(t_s + 16 * k, pk);   // waited for before p_full
+            uint32_t pk[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const float x0 = ex2_approx(fmaf(__uint_as_float(r[2 * j]), sl2, nm));
+              const float x1 = ex2_approx(fmaf(__uint_as_float(r[2 * j + 1]), sl2, nm));
+              ls[(2 * j) & 3] += x0;
+              ls[(2 * j + 1) & 3] += x1;
+              pk[j] = __byte_perm(__float_as_uint(x0) + 0x8000u, __float_as_uint(x1) + 0x8000u, 0x7632);
             }
-            l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+            tmem_st32_nowait(t_s + 32 * c, pk);   // waited for before p_full
           }
+          l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
         }
         tmem_wait_st();   // every P word in tensor memory before PV reads it
         tc_fence_before();
@@ -494,19 +436,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pass_kernel(const __grid_const
 }
 
 cudaError_t launch_tc_pass(const TcPassArgs& args, int num_sms, cudaStream_t stream) {
-  static std::atomic<unsigned long long> set_split{0}, set_whole{0};
-  cudaError_t e = max_dyn_smem_once(tc_pass_kernel<true>, kSmemBytes, set_split);
-  if (e != cudaSuccess) return e;
-  e = max_dyn_smem_once(tc_pass_kernel<false>, kSmemBytes, set_whole);
+  static std::atomic<unsigned long long> set{0};
+  const cudaError_t e = max_dyn_smem_once(tc_pass_kernel, kSmemBytes, set);
   if (e != cudaSuccess) return e;
   const int total_tiles = args.g.B * args.g.h * args.p.n_seq * args.p.n_chunks;
   const int n_units = (total_tiles + 1) / 2;
   int grid = n_units < num_sms ? n_units : num_sms;
   if (grid < 1) return cudaSuccess;
-  if (args.p.kind == kFull)
-    tc_pass_kernel<false><<<grid, kThreads, kSmemBytes, stream>>>(args);
-  else
-    tc_pass_kernel<true><<<grid, kThreads, kSmemBytes, stream>>>(args);
+  tc_pass_kernel<<<grid, kThreads, kSmemBytes, stream>>>(args);
   return cudaGetLastError();
 }
 
