@@ -26,6 +26,7 @@ struct BwdTcArgs {
   float scale, scale_log2;
   int final_out;              // write dq_out / dk_out (bf16) instead of the fp32 shares
   int accumulate;             // add the fp32 shares already in dq_acc / dk_acc (earlier passes') first
+  int single;                 // sequences of at most 128 tokens: the one-tile kernel (no recomputation)
   uint32_t panel_bytes;       // rows (rounded to 8) x 128 bytes
   uint32_t guard_bytes, smem_bytes;
   uint32_t* status;           // device status word (0 = ok, 4 = a wait timed out)

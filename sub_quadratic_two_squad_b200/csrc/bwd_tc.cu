@@ -418,15 +418,226 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
   }
 }
 
+// ------------------------------------------------------------------------------------------------
+// Sequences of at most 128 tokens: one query tile and one key tile. S and dP are computed once; the
+// row-owner warps write P and dS (bf16) to shared memory, and dQ = dS K, dV = P^T dO and dK = dS^T Q
+// are three products read from there (P^T and dS^T as MN-major A operands of the same tiles).
+// ------------------------------------------------------------------------------------------------
+constexpr uint32_t kPdsPanel = 16384;   // 128 query rows x 64 keys (bf16), 128-byte swizzle
+
+__global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc1_kernel(const __grid_constant__ BwdTcArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t panel = a.panel_bytes, alloc = 2u * panel;
+  uint8_t* const sq = base;
+  uint8_t* const sk = base + alloc;
+  uint8_t* const sv = base + 2 * alloc;
+  uint8_t* const sdo = base + 3 * alloc;
+  uint8_t* const sp = base + 4 * alloc + a.guard_bytes;   // P [query][key], two 64-key panels
+  uint8_t* const sds = sp + 2 * kPdsPanel;                 // dS, the same layout
+  BwdBars* const bars = reinterpret_cast<BwdBars*>(sds + 2 * kPdsPanel);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const Grid& g = a.g;
+  const PassGeom& p = a.p;
+  const int s = p.seq_len;
+  const int N = round16b(s);
+  const int bh = static_cast<int>(fdiv(blockIdx.x, p.f_per_bh));
+  const int sigma = static_cast<int>(blockIdx.x) - bh * p.n_seq;
+
+  // Rows past the sequence in each allocation, and the guard past the last one, are read by the MMAs:
+  // zero them (the TMA boxes write exactly s rows per panel).
+  {
+    const uint32_t tail = panel - static_cast<uint32_t>(s) * 128u;   // bytes per panel
+    const uint32_t tail16 = tail / 16u;
+    for (uint32_t i = threadIdx.x; i < 8u * tail16; i += kBwdThreads) {
+      const uint32_t pnl = i / tail16, j = i - pnl * tail16;
+      reinterpret_cast<uint4*>(base + pnl * panel + static_cast<uint32_t>(s) * 128u)[j] = make_uint4(0, 0, 0, 0);
+    }
+    for (uint32_t i = threadIdx.x; i < a.guard_bytes / 16u; i += kBwdThreads)
+      reinterpret_cast<uint4*>(base + 4 * alloc)[i] = make_uint4(0, 0, 0, 0);
+  }
+  if (threadIdx.x == 128) {
+    mbar_init(&bars->load_qk, 1);
+    mbar_init(&bars->load_vd, 1);
+    mbar_init(&bars->s_full, 1);
+    mbar_init(&bars->p_full, 128);
+    mbar_init(&bars->o_full, 1);
+    mbar_init(&bars->drain, 1);
+    bars->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 4) {
+    __syncwarp();
+    tmem_alloc(&bars->tmem_base, 512);
+    tmem_relinquish();
+  }
+  fence_proxy_async_smem();   // zeroed rows -> visible to the MMAs (async proxy)
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  WaitCtl ctl{&bars->abort, a.status, a.timeout_ns};
+  const bool tmem_ok = tmem == 0u;   // all 512 columns requested: anything else is an error
+  if (!tmem_ok && threadIdx.x == 0 && a.status != nullptr) atomicCAS(a.status, 0u, kStatusTimeout);
+
+  // Tensor memory: S [0, N) then dK [0, 128); dP [128, 128 + N); dQ [256, 384); dV [384, 512).
+  if (!tmem_ok) {
+    // nothing issued: fall through to the release below
+  } else if (warp == 4) {
+    if (lane == 0) {
+      // ---------------------------------------------------------------- loads + MMA issue
+      prefetch_tmap(&a.tm_q);
+      prefetch_tmap(&a.tm_k);
+      prefetch_tmap(&a.tm_v);
+      prefetch_tmap(&a.tm_do);
+      const uint32_t tx_half = 4u * static_cast<uint32_t>(s) * 128u;   // two tensors, both panels
+      mbar_arrive_expect_tx(&bars->load_qk, tx_half);
+      mbar_arrive_expect_tx(&bars->load_vd, tx_half);
+      int c[5];
+      chunk_coords(g, p, a.variant, bh, sigma, 0, 0, c);
+      const CUtensorMap* maps[4] = {&a.tm_q, &a.tm_k, &a.tm_v, &a.tm_do};
+      uint8_t* dsts[4] = {sq, sk, sv, sdo};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        uint64_t* bar = i < 2 ? &bars->load_qk : &bars->load_vd;
+        tma_load_5d(dsts[i], maps[i], bar, c[0], c[1], c[2], c[3], c[4]);
+        tma_load_5d(dsts[i] + panel, maps[i], bar, c[0] + 64, c[1], c[2], c[3], c[4]);
+      }
+      const uint32_t aq = smem_u32(sq), ak = smem_u32(sk), av = smem_u32(sv), ado = smem_u32(sdo);
+      const uint32_t ap = smem_u32(sp), ads = smem_u32(sds);
+      const uint32_t idesc_s = idesc_bf16(128, N, false);
+      bool ok = mbar_wait(&bars->load_qk, 0, ctl);
+      if (ok) {
+        tc_fence_after();
+        for (int kk = 0; kk < 8; ++kk)   // S = Q K^T -> [0, N)
+          umma_bf16_ss(tmem, kdesc(aq, kk, panel), kdesc(ak, kk, panel), idesc_s, kk > 0);
+        ok = mbar_wait(&bars->load_vd, 0, ctl);
+      }
+      if (ok) {
+        tc_fence_after();
+        for (int kk = 0; kk < 8; ++kk)   // dP = dO V^T -> [128, 128 + N)
+          umma_bf16_ss(tmem + 128, kdesc(ado, kk, panel), kdesc(av, kk, panel), idesc_s, kk > 0);
+        umma_commit(&bars->s_full);
+        ok = mbar_wait(&bars->p_full, 0, ctl);
+      }
+      if (ok) {
+        tc_fence_after();
+        const uint32_t idesc_q = idesc_bf16(128, 128, true);   // A K-major (dS), B MN-major (K)
+        const uint32_t idesc_t = idesc_bf16_a_mn(128, 128);    // A = P^T / dS^T, B = dO / Q
+        for (int kk = 0; kk < N / 16; ++kk)   // dQ = dS K -> [256, 384)
+          umma_bf16_ss(tmem + 256, kdesc(ads, kk, kPdsPanel), sw128_desc(ak + kk * 2048, panel, 1024), idesc_q,
+                       kk > 0);
+        for (int kk = 0; kk < N / 16; ++kk)   // dV = P^T dO -> [384, 512)
+          umma_bf16_ss(tmem + 384, sw128_desc(ap + kk * 2048, kPdsPanel, 1024), sw128_desc(ado + kk * 2048, panel, 1024),
+                       idesc_t, kk > 0);
+        for (int kk = 0; kk < N / 16; ++kk)   // dK = dS^T Q -> [0, 128)
+          umma_bf16_ss(tmem, sw128_desc(ads + kk * 2048, kPdsPanel, 1024), sw128_desc(aq + kk * 2048, panel, 1024),
+                       idesc_t, kk > 0);
+        umma_commit(&bars->o_full);
+      }
+      // every MMA issued has completed before the CTA frees tensor memory
+      umma_commit(&bars->drain);
+      mbar_wait_drain(&bars->drain, 0, 20000000ull);
+    }
+  } else {
+    // ------------------------------------------------------------------ row-owner warps
+    const int r = warp * 32 + lane;   // TMEM lane = query row = key row of this thread
+    const uint32_t t_row = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const float sl2 = a.scale_log2;
+    const int tok = r < s ? token_of(g, p, sigma, 0, r) : -1;
+    const size_t gi = static_cast<size_t>(bh) * g.n + (tok < 0 ? 0 : tok);
+    const float lse2 = tok >= 0 ? a.lse[gi] * kLog2e : 0.f;
+    uint4 orow[16];
+    {
+      const uint4* src = reinterpret_cast<const uint4*>(a.o + gi * 128);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) orow[i] = tok >= 0 ? src[i] : make_uint4(0, 0, 0, 0);
+    }
+    bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->load_vd, 0, ctl));
+    const float D = (ok && tok >= 0) ? row_dot_out(sdo, panel, r, orow) : 0.f;   // D_i = dO_i . O_i
+    if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->s_full, 0, ctl));
+    if (ok) {
+      tc_fence_after();
+      // P and dS = P o (dP - D) of this row, bf16, into shared memory (zero past the sequence, and on
+      // rows past it: those rows are K rows of dV and dK)
+      const uint32_t row_p = smem_u32(sp) + static_cast<uint32_t>(r) * 128u;
+      const uint32_t row_ds = smem_u32(sds) + static_cast<uint32_t>(r) * 128u;
+      const uint32_t sw = static_cast<uint32_t>(r & 7);
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t pp[16], pd[16];
+        if (32 * c < N) {
+          uint32_t sr[32], dr[32];
+          tmem_ld32(t_row + 32 * c, sr);
+          tmem_ld32(t_row + 128 + 32 * c, dr);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int j = 32 * c + 2 * i;
+            const bool v0 = tok >= 0 && j < s, v1 = tok >= 0 && j + 1 < s;
+            const float p0 = v0 ? ex2_approx(fmaf(__uint_as_float(sr[2 * i]), sl2, -lse2)) : 0.f;
+            const float p1 = v1 ? ex2_approx(fmaf(__uint_as_float(sr[2 * i + 1]), sl2, -lse2)) : 0.f;
+            const float s0 = v0 ? p0 * (__uint_as_float(dr[2 * i]) - D) : 0.f;
+            const float s1 = v1 ? p1 * (__uint_as_float(dr[2 * i + 1]) - D) : 0.f;
+            pp[i] = pack2_rn(p0, p1);
+            pd[i] = pack2_rn(s0, s1);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) pp[i] = pd[i] = 0u;
+        }
+        // keys [32 c, 32 c + 32): panel c / 2, 16-byte chunks 4 (c % 2) .. + 3 of the 128-byte row
+        const uint32_t pnl = static_cast<uint32_t>(c >> 1) * kPdsPanel;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint32_t off = pnl + (((static_cast<uint32_t>(4 * (c & 1) + q)) ^ sw) << 4);
+          st_shared_v4(row_p + off, pp[4 * q], pp[4 * q + 1], pp[4 * q + 2], pp[4 * q + 3]);
+          st_shared_v4(row_ds + off, pd[4 * q], pd[4 * q + 1], pd[4 * q + 2], pd[4 * q + 3]);
+        }
+      }
+      fence_proxy_async_smem();   // P and dS -> visible to the MMAs (async proxy)
+      tc_fence_before();
+      mbar_arrive(&bars->p_full);
+      ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->o_full, 0, ctl));
+    }
+    if (ok) {
+      tc_fence_after();
+      const size_t ro = gi * 128;
+      if (a.final_out)
+        write_row(t_row + 256, tok >= 0, a.scale, a.accumulate ? a.dq_acc + ro : nullptr, a.dq_out + ro, nullptr);
+      else
+        write_row(t_row + 256, tok >= 0, a.scale, a.accumulate ? a.dq_acc + ro : nullptr, nullptr, a.dq_acc + ro);
+      write_row(t_row + 384, tok >= 0, 1.f, nullptr, a.dv_out + ro, nullptr);
+      if (a.final_out)
+        write_row(t_row, tok >= 0, a.scale, a.accumulate ? a.dk_acc + ro : nullptr, a.dk_out + ro, nullptr);
+      else
+        write_row(t_row, tok >= 0, a.scale, a.accumulate ? a.dk_acc + ro : nullptr, nullptr, a.dk_acc + ro);
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 4) {
+    __syncwarp();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_bwd_tc(const BwdTcArgs& a, cudaStream_t stream) {
-  static std::atomic<unsigned long long> set{0};
-  const cudaError_t e = max_dyn_smem_once(bwd_tc_kernel, kBwdSmemLimit, set);
+  static std::atomic<unsigned long long> set{0}, set1{0};
+  cudaError_t e = max_dyn_smem_once(bwd_tc_kernel, kBwdSmemLimit, set);
+  if (e != cudaSuccess) return e;
+  e = max_dyn_smem_once(bwd_tc1_kernel, kBwdSmemLimit, set1);
   if (e != cudaSuccess) return e;
   const unsigned grid = static_cast<unsigned>(a.g.B * a.g.h * a.p.n_seq);
   if (grid == 0) return cudaSuccess;
-  bwd_tc_kernel<<<grid, kBwdThreads, a.smem_bytes, stream>>>(a);
+  if (a.single)
+    bwd_tc1_kernel<<<grid, kBwdThreads, a.smem_bytes, stream>>>(a);
+  else
+    bwd_tc_kernel<<<grid, kBwdThreads, a.smem_bytes, stream>>>(a);
   return cudaGetLastError();
 }
 
@@ -444,6 +655,10 @@ bool bwd_tc_plan(BwdTcArgs& a) {
   a.guard_bytes = (over + 1023u) & ~1023u;
   a.smem_bytes = 1024u + 8u * a.panel_bytes + a.guard_bytes + kBwdVecBytes + kBwdBarBytes;
   if (a.smem_bytes > kBwdSmemLimit) return false;
+  // One tile: P and dS in shared memory instead of the per-query vectors
+  const uint32_t single_bytes = 1024u + 8u * a.panel_bytes + a.guard_bytes + 4u * kPdsPanel + kBwdBarBytes;
+  a.single = (tiles == 1 && single_bytes <= kBwdSmemLimit) ? 1 : 0;
+  if (a.single) a.smem_bytes = single_bytes;
   if (a.smem_bytes < kBwdSmemMin) a.smem_bytes = kBwdSmemMin;
   return true;
 }

@@ -344,6 +344,10 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major)
          | (static_cast<uint32_t>(M >> 4) << 24);   // M / 16
 }
 
+// As idesc_bf16 with B MN-major, and A MN-major too (A read from shared memory with its M index
+// contiguous: the transpose of a K-major tile).
+__host__ __device__ constexpr uint32_t idesc_bf16_a_mn(int M, int N) { return idesc_bf16(M, N, true) | (1u << 15); }
+
 __device__ __forceinline__ void st_shared_v4(uint32_t saddr, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(saddr), "r"(x), "r"(y), "r"(z), "r"(w) : "memory");
 }
