@@ -27,6 +27,8 @@ struct BwdTcArgs {
   int final_out;              // write dq_out / dk_out (bf16) instead of the fp32 shares
   int accumulate;             // add the fp32 shares already in dq_acc / dk_acc (earlier passes') first
   int single;                 // sequences of at most 128 tokens: the one-tile kernel (no recomputation)
+  int pack;                   // sequences per CTA of the one-tile kernel (128 / seg_rows)
+  int seg_rows;               // rows of one sequence's band in its tiles (the length rounded up to 8)
   uint32_t panel_bytes;       // rows (rounded to 8) x 128 bytes
   uint32_t guard_bytes, smem_bytes;
   uint32_t* status;           // device status word (0 = ok, 4 = a wait timed out)

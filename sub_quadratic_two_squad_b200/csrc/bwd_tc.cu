@@ -419,35 +419,44 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
 }
 
 // ------------------------------------------------------------------------------------------------
-// Sequences of at most 128 tokens: one query tile and one key tile. S and dP are computed once; the
+// Sequences of at most 128 tokens: one query tile and one key tile. A CTA takes `pack` consecutive
+// sequences (of all B h n_seq), each in its own band of `seg` rows (the length rounded up to 8) of
+// every tile; S and dP are computed once over the whole tile, and a score counts only where query and
+// key lie in the same band (P = dS = 0 elsewhere, so the products stay block-diagonal). The
 // row-owner warps write P and dS (bf16) to shared memory, and dQ = dS K, dV = P^T dO and dK = dS^T Q
 // are three products read from there (P^T and dS^T as MN-major A operands of the same tiles).
 // ------------------------------------------------------------------------------------------------
 constexpr uint32_t kPdsPanel = 16384;   // 128 query rows x 64 keys (bf16), 128-byte swizzle
 
+// kPacked: several sequences per CTA (128-row operand tiles, a band per sequence). Otherwise one
+// sequence per CTA, its operand tiles as long as the sequence (rounded to 8 rows) with a zeroed guard
+// past the last one.
+template <bool kPacked>
 __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc1_kernel(const __grid_constant__ BwdTcArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const uint32_t panel = a.panel_bytes, alloc = 2u * panel;
+  const uint32_t panel = kPacked ? kPdsPanel : a.panel_bytes, alloc = 2u * panel;
   uint8_t* const sq = base;
   uint8_t* const sk = base + alloc;
   uint8_t* const sv = base + 2 * alloc;
   uint8_t* const sdo = base + 3 * alloc;
-  uint8_t* const sp = base + 4 * alloc + a.guard_bytes;   // P [query][key], two 64-key panels
-  uint8_t* const sds = sp + 2 * kPdsPanel;                 // dS, the same layout
+  uint8_t* const sp = base + 4 * alloc + (kPacked ? 0u : a.guard_bytes);   // P [query][key], two 64-key panels
+  uint8_t* const sds = sp + 2 * kPdsPanel;                                   // dS, the same layout
   BwdBars* const bars = reinterpret_cast<BwdBars*>(sds + 2 * kPdsPanel);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const Grid& g = a.g;
   const PassGeom& p = a.p;
   const int s = p.seq_len;
-  const int N = round16b(s);
-  const int bh = static_cast<int>(fdiv(blockIdx.x, p.f_per_bh));
-  const int sigma = static_cast<int>(blockIdx.x) - bh * p.n_seq;
+  const int seg = a.seg_rows;                                   // band of one sequence (s rounded to 8)
+  const int total = g.B * g.h * p.n_seq;                        // sequences of all (b, head)
+  const int first = static_cast<int>(blockIdx.x) * a.pack;      // this CTA's first sequence
+  const int nseq = min(a.pack, total - first);                  // sequences in this CTA
+  const int N = round16b(nseq * seg);                           // key (and query) rows in use
 
-  // Rows past the sequence in each allocation, and the guard past the last one, are read by the MMAs:
-  // zero them (the TMA boxes write exactly s rows per panel).
-  {
+  if constexpr (!kPacked) {
+    // Rows past the sequence in each tile, and the guard past the last one, are read by the MMAs:
+    // zero them (the TMA boxes write exactly s rows per panel).
     const uint32_t tail = panel - static_cast<uint32_t>(s) * 128u;   // bytes per panel
     const uint32_t tail16 = tail / 16u;
     for (uint32_t i = threadIdx.x; i < 8u * tail16; i += kBwdThreads) {
@@ -456,6 +465,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc1_kernel(const __grid_co
     }
     for (uint32_t i = threadIdx.x; i < a.guard_bytes / 16u; i += kBwdThreads)
       reinterpret_cast<uint4*>(base + 4 * alloc)[i] = make_uint4(0, 0, 0, 0);
+    fence_proxy_async_smem();   // zeroed rows -> visible to the MMAs (async proxy)
   }
   if (threadIdx.x == 128) {
     mbar_init(&bars->load_qk, 1);
@@ -472,7 +482,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc1_kernel(const __grid_co
     tmem_alloc(&bars->tmem_base, 512);
     tmem_relinquish();
   }
-  fence_proxy_async_smem();   // zeroed rows -> visible to the MMAs (async proxy)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -480,30 +489,53 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc1_kernel(const __grid_co
   WaitCtl ctl{&bars->abort, a.status, a.timeout_ns};
   const bool tmem_ok = tmem == 0u;   // all 512 columns requested: anything else is an error
   if (!tmem_ok && threadIdx.x == 0 && a.status != nullptr) atomicCAS(a.status, 0u, kStatusTimeout);
+  const uint32_t tx_half = static_cast<uint32_t>(nseq) * 4u * static_cast<uint32_t>(s) * 128u;
+  if (tmem_ok && threadIdx.x == 128) {
+    // the loads: each sequence's boxes into its band (a multiple of 8 rows, so the 128-byte swizzle
+    // phase is kept)
+    prefetch_tmap(&a.tm_q);
+    prefetch_tmap(&a.tm_k);
+    prefetch_tmap(&a.tm_v);
+    prefetch_tmap(&a.tm_do);
+    mbar_arrive_expect_tx(&bars->load_qk, tx_half);
+    mbar_arrive_expect_tx(&bars->load_vd, tx_half);
+    const CUtensorMap* maps[4] = {&a.tm_q, &a.tm_k, &a.tm_v, &a.tm_do};
+    uint8_t* dsts[4] = {sq, sk, sv, sdo};
+    for (int j = 0; j < nseq; ++j) {
+      const int gs = first + j;
+      const int bh = static_cast<int>(fdiv(static_cast<uint32_t>(gs), p.f_per_bh));
+      int c[5];
+      chunk_coords(g, p, a.variant, bh, gs - bh * p.n_seq, 0, 0, c);
+      const uint32_t row_off = static_cast<uint32_t>(j * seg) * 128u;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        uint64_t* bar = i < 2 ? &bars->load_qk : &bars->load_vd;
+        tma_load_5d(dsts[i] + row_off, maps[i], bar, c[0], c[1], c[2], c[3], c[4]);
+        tma_load_5d(dsts[i] + panel + row_off, maps[i], bar, c[0] + 64, c[1], c[2], c[3], c[4]);
+      }
+    }
+  }
+  if constexpr (kPacked) {
+    // Meanwhile, the rows of each tile that no box writes (the gap after each sequence in its band,
+    // and the rows past the last band) are zeroed: the MMAs read them.
+    for (uint32_t i = threadIdx.x; i < 8u * 128u; i += kBwdThreads) {   // (panel, row) pairs
+      const int row = static_cast<int>(i & 127u);
+      const int band = row / seg, pos = row - band * seg;
+      if (band < nseq && pos < s) continue;
+      uint4* dst = reinterpret_cast<uint4*>(base + (i >> 7) * panel + static_cast<uint32_t>(row) * 128u);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) dst[j] = make_uint4(0, 0, 0, 0);
+    }
+    fence_proxy_async_smem();   // zeroed rows -> visible to the MMAs (async proxy)
+    __syncthreads();
+  }
 
   // Tensor memory: S [0, N) then dK [0, 128); dP [128, 128 + N); dQ [256, 384); dV [384, 512).
   if (!tmem_ok) {
     // nothing issued: fall through to the release below
   } else if (warp == 4) {
     if (lane == 0) {
-      // ---------------------------------------------------------------- loads + MMA issue
-      prefetch_tmap(&a.tm_q);
-      prefetch_tmap(&a.tm_k);
-      prefetch_tmap(&a.tm_v);
-      prefetch_tmap(&a.tm_do);
-      const uint32_t tx_half = 4u * static_cast<uint32_t>(s) * 128u;   // two tensors, both panels
-      mbar_arrive_expect_tx(&bars->load_qk, tx_half);
-      mbar_arrive_expect_tx(&bars->load_vd, tx_half);
-      int c[5];
-      chunk_coords(g, p, a.variant, bh, sigma, 0, 0, c);
-      const CUtensorMap* maps[4] = {&a.tm_q, &a.tm_k, &a.tm_v, &a.tm_do};
-      uint8_t* dsts[4] = {sq, sk, sv, sdo};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        uint64_t* bar = i < 2 ? &bars->load_qk : &bars->load_vd;
-        tma_load_5d(dsts[i], maps[i], bar, c[0], c[1], c[2], c[3], c[4]);
-        tma_load_5d(dsts[i] + panel, maps[i], bar, c[0] + 64, c[1], c[2], c[3], c[4]);
-      }
+      // ---------------------------------------------------------------- MMA issue (loads above)
       const uint32_t aq = smem_u32(sq), ak = smem_u32(sk), av = smem_u32(sv), ado = smem_u32(sdo);
       const uint32_t ap = smem_u32(sp), ads = smem_u32(sds);
       const uint32_t idesc_s = idesc_bf16(128, N, false);
@@ -545,7 +577,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc1_kernel(const __grid_co
     const int r = warp * 32 + lane;   // TMEM lane = query row = key row of this thread
     const uint32_t t_row = tmem + (static_cast<uint32_t>(warp * 32) << 16);
     const float sl2 = a.scale_log2;
-    const int tok = r < s ? token_of(g, p, sigma, 0, r) : -1;
+    const int band = r / seg, pos = r - band * seg;   // this row's sequence within the CTA, and position
+    int tok = -1, bh = 0;
+    if (band < nseq && pos < s) {
+      const int gs = first + band;
+      bh = static_cast<int>(fdiv(static_cast<uint32_t>(gs), p.f_per_bh));
+      tok = token_of(g, p, gs - bh * p.n_seq, 0, pos);
+    }
+    const int k0 = band * seg;   // the row's own keys: columns [k0, k0 + s)
     const size_t gi = static_cast<size_t>(bh) * g.n + (tok < 0 ? 0 : tok);
     const float lse2 = tok >= 0 ? a.lse[gi] * kLog2e : 0.f;
     uint4 orow[16];
@@ -559,8 +598,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc1_kernel(const __grid_co
     if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->s_full, 0, ctl));
     if (ok) {
       tc_fence_after();
-      // P and dS = P o (dP - D) of this row, bf16, into shared memory (zero past the sequence, and on
-      // rows past it: those rows are K rows of dV and dK)
+      // P and dS = P o (dP - D) of this row, bf16, into shared memory (zero outside the row's own
+      // sequence, and on rows of no sequence: those rows are K rows of dV and dK)
       const uint32_t row_p = smem_u32(sp) + static_cast<uint32_t>(r) * 128u;
       const uint32_t row_ds = smem_u32(sds) + static_cast<uint32_t>(r) * 128u;
       const uint32_t sw = static_cast<uint32_t>(r & 7);
@@ -573,8 +612,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc1_kernel(const __grid_co
           tmem_ld32(t_row + 128 + 32 * c, dr);
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const int j = 32 * c + 2 * i;
-            const bool v0 = tok >= 0 && j < s, v1 = tok >= 0 && j + 1 < s;
+            const int j = 32 * c + 2 * i - k0;   // key position within the row's own sequence
+            const bool v0 = tok >= 0 && j >= 0 && j < s, v1 = tok >= 0 && j + 1 >= 0 && j + 1 < s;
             const float p0 = v0 ? ex2_approx(fmaf(__uint_as_float(sr[2 * i]), sl2, -lse2)) : 0.f;
             const float p1 = v1 ? ex2_approx(fmaf(__uint_as_float(sr[2 * i + 1]), sl2, -lse2)) : 0.f;
             const float s0 = v0 ? p0 * (__uint_as_float(dr[2 * i]) - D) : 0.f;
@@ -627,17 +666,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc1_kernel(const __grid_co
 }  // namespace
 
 cudaError_t launch_bwd_tc(const BwdTcArgs& a, cudaStream_t stream) {
-  static std::atomic<unsigned long long> set{0}, set1{0};
+  static std::atomic<unsigned long long> set{0}, set1{0}, set1p{0};
   cudaError_t e = max_dyn_smem_once(bwd_tc_kernel, kBwdSmemLimit, set);
   if (e != cudaSuccess) return e;
-  e = max_dyn_smem_once(bwd_tc1_kernel, kBwdSmemLimit, set1);
+  e = max_dyn_smem_once(bwd_tc1_kernel<false>, kBwdSmemLimit, set1);
   if (e != cudaSuccess) return e;
-  const unsigned grid = static_cast<unsigned>(a.g.B * a.g.h * a.p.n_seq);
-  if (grid == 0) return cudaSuccess;
-  if (a.single)
-    bwd_tc1_kernel<<<grid, kBwdThreads, a.smem_bytes, stream>>>(a);
+  e = max_dyn_smem_once(bwd_tc1_kernel<true>, kBwdSmemLimit, set1p);
+  if (e != cudaSuccess) return e;
+  const int seqs = a.g.B * a.g.h * a.p.n_seq;
+  if (seqs == 0) return cudaSuccess;
+  if (a.single && a.pack > 1)
+    bwd_tc1_kernel<true><<<static_cast<unsigned>((seqs + a.pack - 1) / a.pack), kBwdThreads, a.smem_bytes, stream>>>(a);
+  else if (a.single)
+    bwd_tc1_kernel<false><<<static_cast<unsigned>(seqs), kBwdThreads, a.smem_bytes, stream>>>(a);
   else
-    bwd_tc_kernel<<<grid, kBwdThreads, a.smem_bytes, stream>>>(a);
+    bwd_tc_kernel<<<static_cast<unsigned>(seqs), kBwdThreads, a.smem_bytes, stream>>>(a);
   return cudaGetLastError();
 }
 
@@ -655,10 +698,13 @@ bool bwd_tc_plan(BwdTcArgs& a) {
   a.guard_bytes = (over + 1023u) & ~1023u;
   a.smem_bytes = 1024u + 8u * a.panel_bytes + a.guard_bytes + kBwdVecBytes + kBwdBarBytes;
   if (a.smem_bytes > kBwdSmemLimit) return false;
-  // One tile: P and dS in shared memory instead of the per-query vectors
-  const uint32_t single_bytes = 1024u + 8u * a.panel_bytes + a.guard_bytes + 4u * kPdsPanel + kBwdBarBytes;
-  a.single = (tiles == 1 && single_bytes <= kBwdSmemLimit) ? 1 : 0;
-  if (a.single) a.smem_bytes = single_bytes;
+  // One tile: six 128-row tiles (Q, K, V, dO, P, dS), as many sequences per CTA as fit in 128 rows
+  a.single = tiles == 1 ? 1 : 0;
+  a.seg_rows = static_cast<int>(rows8);
+  a.pack = a.single ? 128 / a.seg_rows : 1;
+  if (a.single)
+    a.smem_bytes = a.pack > 1 ? 1024u + 12u * kPdsPanel + kBwdBarBytes
+                              : 1024u + 8u * a.panel_bytes + a.guard_bytes + 4u * kPdsPanel + kBwdBarBytes;
   if (a.smem_bytes < kBwdSmemMin) a.smem_bytes = kBwdSmemMin;
   return true;
 }
