@@ -17,6 +17,7 @@
 #include "kpass_plan.h"
 #include "bwd_pass.h"
 #include "bwd_stream.h"
+#include "pack_pass.h"
 #include "pad.h"
 #include "short_pass.h"
 #include "simt_pass.h"
@@ -292,6 +293,26 @@ squad_status_t launch_short_args(ShortArgs& a, float scale, uint32_t* status, ui
 squad_status_t run_pass(const squad_params_t* prm, const Grid& g, int kind, float scale, const void* q,
                         const void* k, const void* v, bool v_bf16, void* out, float* lse, uint32_t* status,
                         uint32_t* work, cudaStream_t stream) {
+  if (prm->dtype == SQUAD_BF16 && v_bf16) {
+    // sequences of at most 64 tokens: several per 128-row tile
+    PackFwdArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.g = g;
+    a.p = make_geom(g, kind, 256);
+    if (pack_eligible(g, a.p)) {
+      a.variant = kind == kGlobal ? kSlotBoxVariant : 0;
+      if (!encode_pass_map(&a.tm_q, q, g, a.p, a.variant) || !encode_pass_map(&a.tm_k, k, g, a.p, a.variant) ||
+          !encode_pass_map(&a.tm_v, v, g, a.p, a.variant))
+        return SQUAD_ERR_CUDA;
+      pack_plan(a);
+      a.out = static_cast<__nv_bfloat16*>(out);
+      a.lse = lse;
+      a.scale_log2 = scale * 1.4426950408889634f;
+      a.status = status;
+      a.timeout_ns = kWaitTimeoutNs;
+      return launch_pack_fwd(a, stream) == cudaSuccess ? SQUAD_OK : SQUAD_ERR_CUDA;
+    }
+  }
   if (short_eligible(prm, g, make_geom(g, kind, 256)) && v_bf16 && work != nullptr) {
     ShortArgs a;
     std::memset(&a, 0, sizeof(a));

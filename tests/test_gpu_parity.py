@@ -248,6 +248,14 @@ def test_single_pass_wan22_5b_shape(order):
     run_bwd(1, 2, 128, (21, 22, 40), (21, 2, 4), order, torch.bfloat16)
 
 
+@pytest.mark.parametrize("order", [LO, GO])
+def test_single_pass_short_sequences_packed(order):
+    """21-token windows (five per 128-row tile) and 8-token slot sequences (sixteen per tile), the last
+    tile of each launch partly filled, forward and backward."""
+    run_fwd(1, 3, 128, (3, 4, 14), (3, 1, 7), order, torch.bfloat16)
+    run_bwd(1, 3, 128, (3, 4, 14), (3, 1, 7), order, torch.bfloat16)
+
+
 # ------------------------------------------------------------------------------------------------
 # grids the window does not divide (reflect padding, both passes on the padded grid, crop)
 # ------------------------------------------------------------------------------------------------
