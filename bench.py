@@ -376,9 +376,11 @@ def run_ours(args, rank, world, local_rank):
         "single_pass": single,
         "backward": {"ms_per_block": bwd_ms,
                      "tflops_algorithmic": 2.0 * f / (bwd_ms * 1e-3) / 1e12,
-                     "flops_note": "algorithmic = 2x forward (dQ, dK, dV, dP products); the kernel executes 3.5x "
-                                   "forward (S and dP recomputed for the row and for the column products)",
-                     "kernels": "tcgen05 bwd_tc_kernel, one launch per pass (rows: dQ, D; columns: dK, dV)"},
+                     "flops_note": "algorithmic = 2x forward (dQ, dK, dV, dP products); executed: 3.5x forward "
+                                   "for the 168-token windows (S and dP recomputed for the row and for the column "
+                                   "products), 2.5x for the 110-token slot sequences (one tile, no recomputation)",
+                     "kernels": "tcgen05, one launch per pass: bwd_tc1_kernel (slot sequences) then bwd_tc_kernel "
+                                "(windows)"},
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
