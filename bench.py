@@ -31,8 +31,8 @@ E2E_GROUPS = 8             # runs of heads of the end-to-end host forward (copie
 # DRAM traffic of one launch of the forward kernel from an ncu capture of this workload
 # (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the kernel source it was measured on
 # (sha1 prefix below); otherwise reported as null.
-PROFILED_TRAFFIC_BYTES = (439.780864 + 193.515264) * 1e6
-PROFILED_KERNEL_SHA1 = "106eee5226f1020c"
+PROFILED_TRAFFIC_BYTES = (449.138688 + 193.413632) * 1e6
+PROFILED_KERNEL_SHA1 = "c050960863e2f152"
 PROFILED_KERNEL_SRC = os.path.join(ROOT, "sub_quadratic_two_squad_b200", "csrc", "attn_short.cu")
 
 
