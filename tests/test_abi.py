@@ -117,7 +117,7 @@ def test_single_pass_orders_accepted_and_counted(lib, cfg):
 
 
 @pytest.mark.parametrize("grid", [(21, 22, 40), (21, 30, 52), (21, 44, 80), (21, 60, 104), (13, 17, 29), (5, 8, 8),
-                                  (1, 1, 1), (3, 1, 50), (7, 31, 2)])
+                                  (1, 1, 1), (3, 1, 50), (7, 31, 2), (21, 23, 46), (5, 17, 17), (9, 31, 93), (21, 29, 29)])
 def test_window_solver_matches_the_oracle(lib, grid):
     tw, hw, ww = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
     assert lib.squad_window_solve(*grid, ctypes.byref(tw), ctypes.byref(hw), ctypes.byref(ww)) == _lib.SQUAD_OK

@@ -368,6 +368,26 @@ def test_window_solver_tracks_sqrt_n_and_is_locally_optimal(grid):
             assert cost(hw) <= cost(nb)
 
 
+@pytest.mark.parametrize("grid,r,pads", [((21, 23, 46), 2, True), ((5, 17, 17), 1, True), ((21, 45, 90), 2, False),
+                                         ((9, 31, 93), 3, True), ((21, 29, 29), 1, True)])
+def test_window_solver_is_the_brute_force_minimiser_on_exact_aspect_grids(grid, r, pads):
+    """Where W = r H exactly, following the aspect ratio fixes ww = r hw, so the solver must return the
+    hw of least cost over all of them. The cost is the pinned FLOP counter on the grid rounded up to
+    whole windows (reflect padding), computed here without the solver's own helpers; most grids are
+    chosen so that the minimiser pads (17, 23, 29 and 31 are prime)."""
+    T, H, W = grid
+    best = None
+    for hw in range(1, H + 1):
+        ww = r * hw
+        Hp, Wp = hw * -(-H // hw), ww * -(-W // ww)   # the least multiples of the window at least H, W
+        cost = orc.squad_flops(1, 1, 1, T * Hp * Wp, T * hw * ww)
+        if best is None or cost < best[0]:
+            best = (cost, hw, ww)
+    assert orc.window_solve(T, H, W) == (T, best[1], best[2])
+    _, hw, ww = orc.window_solve(T, H, W)
+    assert bool(H % hw or W % ww) == pads
+
+
 @pytest.mark.parametrize("grid,window", [((2, 5, 7), (2, 2, 3)), ((3, 7, 4), (3, 3, 3))])
 def test_reflect_pad_is_torch_reflect(grid, window):
     T, H, W = grid
