@@ -198,13 +198,13 @@ def test_backward_bf16_long_windows_chunked_tensor_cores(order):
     run_bwd(1, 1, 128, (21, 8, 8), (21, 4, 4), order, torch.bfloat16)
 
 
-@pytest.mark.parametrize("order", [GO, LG])
-def test_backward_bf16_long_slot_sequences_chunked(order):
+@pytest.mark.parametrize("order,B,h", [(GO, 1, 2), (LG, 1, 2), (GO, 2, 1)])
+def test_backward_bf16_long_slot_sequences_chunked(order, B, h):
     """576-token slot sequences (24 lines of 24 tokens: chunks of 5 lines, the last one 4) on the chunked
-    kernels, alone and after a 20-token local pass."""
-    ks = _bwd_kernels(2, (5, 48, 48), (5, 2, 2), order)
+    kernels, alone and after a 20-token local pass; two batches of one head."""
+    ks = _bwd_kernels(h, (5, 48, 48), (5, 2, 2), order)
     assert ks == (("tc_chunked", None) if order == GO else ("tc_whole", "tc_chunked"))
-    run_bwd(1, 2, 128, (5, 48, 48), (5, 2, 2), order, torch.bfloat16)
+    run_bwd(B, h, 128, (5, 48, 48), (5, 2, 2), order, torch.bfloat16)
 
 
 def test_backward_hires_5b_chunked():
@@ -248,12 +248,12 @@ def test_single_pass_wan22_5b_shape(order):
     run_bwd(1, 2, 128, (21, 22, 40), (21, 2, 4), order, torch.bfloat16)
 
 
-@pytest.mark.parametrize("order", [LO, GO])
-def test_single_pass_short_sequences_packed(order):
-    """21-token windows (five per 128-row tile) and 8-token slot sequences (sixteen per tile), the last
-    tile of each launch partly filled, forward and backward."""
-    run_fwd(1, 3, 128, (3, 4, 14), (3, 1, 7), order, torch.bfloat16)
-    run_bwd(1, 3, 128, (3, 4, 14), (3, 1, 7), order, torch.bfloat16)
+@pytest.mark.parametrize("order,B,h", [(LO, 1, 3), (GO, 1, 3), (LO, 2, 2)])
+def test_single_pass_short_sequences_packed(order, B, h):
+    """21-token windows (five per 128-row tile) and 8-token slot sequences (sixteen per tile), tiles that
+    span heads and batches, the last tile of each launch partly filled; forward and backward."""
+    run_fwd(B, h, 128, (3, 4, 14), (3, 1, 7), order, torch.bfloat16)
+    run_bwd(B, h, 128, (3, 4, 14), (3, 1, 7), order, torch.bfloat16)
 
 
 # ------------------------------------------------------------------------------------------------
