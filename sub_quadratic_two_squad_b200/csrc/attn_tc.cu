@@ -352,7 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pass_kernel(const __grid_const
                   for (int j = 0; j < 16; ++j) {
                     const float x0 = __uint_as_float(pw[j] << 16) * f;
                     const float x1 = __uint_as_float(pw[j] & 0xFFFF0000u) * f;
-                    pw[j] = __byte_perm(__float_as_uint(x0) + 0x8000u, __float_as_uint(x1) + 0x8000u, 0x7632);
+                    pw[j] = pack_bf16x2(x0, x1);
                   }
                   tmem_st16(t_s + 16 * cc, pw);
                 }
@@ -373,8 +373,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pass_kernel(const __grid_const
               l *= f;
               m_used = m_new;
             }
-            // P = 2^(x - m_used) (masked columns give 0), rounded to bf16 on the integer pipe (add half an
-            // ulp, keep the high half), packed two per 32-bit word over columns already read
+            // P = 2^(x - m_used) (masked columns give 0), rounded to bf16 pairs (one conversion per two
+            // values), packed two per 32-bit word over columns already read
             const float nm = -m_used;
             uint32_t pk[32];
 #pragma unroll
@@ -383,7 +383,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_pass_kernel(const __grid_const
               const float x1 = ex2_approx(fmaf(__uint_as_float(r[2 * j + 1]), sl2, nm));
               ls[(2 * j) & 3] += x0;
               ls[(2 * j + 1) & 3] += x1;
-              pk[j] = __byte_perm(__float_as_uint(x0) + 0x8000u, __float_as_uint(x1) + 0x8000u, 0x7632);
+              pk[j] = pack_bf16x2(x0, x1);
             }
             tmem_st32_nowait(t_s + 32 * c, pk);   // waited for before p_full
           }

@@ -139,6 +139,38 @@ def test_full_attention_small(n, dtype):
     np.testing.assert_allclose(lse.cpu().numpy(), ref_lse, rtol=0, atol=1e-3 if dtype == torch.bfloat16 else 1e-5)
 
 
+@pytest.mark.parametrize("case", ["short_kernel", "chunked_local", "full"])
+def test_late_large_keys_raise_the_softmax_reference(case):
+    """Keys late in each sequence scaled by 64 (a power of two, exact in bf16), so that later columns'
+    scores exceed the first chunk's maximum by far more than the kernels' headroom: the one-pass
+    softmax must raise its reference, rescale what it already wrote and take the chunk again.
+    168-token windows (short kernel, third chunk), 336-token windows (chunked kernel, second and third
+    key blocks) and full attention over 384 tokens (third key block, the output rescaled too)."""
+    if case == "full":
+        n = 384
+        x = make_inputs(1, 2, n, 128, dtype="bf16")
+        x["k"][:, :, 200:, :] *= 64.0
+        q, k, v = (_dev(x[s], torch.bfloat16) for s in "qkv")
+        lse = torch.empty((1, 2, n), dtype=torch.float32, device="cuda")
+        out = full_attn_fwd(q, k, v, lse=lse)
+        ref, ref_lse = orc.full_attn_fwd(x["q"], x["k"], x["v"])
+        check_bf16(_host(out), ref, "full")
+        np.testing.assert_allclose(lse.cpu().numpy(), ref_lse, rtol=1e-5, atol=1e-2)
+        return
+    grid, window, first_late = {"short_kernel": ((21, 4, 8), (21, 2, 4), 128),
+                                "chunked_local": ((21, 8, 8), (21, 4, 4), 192)}[case]
+    order = LG if case == "short_kernel" else LO
+    n = grid[0] * grid[1] * grid[2]
+    x = make_inputs(1, 2, n, 128, dtype="bf16")
+    late = orc.window_partition(*grid, *window)[:, first_late:].ravel()
+    x["k"][:, :, late, :] *= 64.0
+    q, k, v = (_dev(x[s], torch.bfloat16) for s in "qkv")
+    out, ws = squad_attn_fwd(q, k, v, grid, window, order)
+    assert squad_attn_fwd_status(ws, q, grid, window, order) == 0
+    ref = orc.squad_attn_fwd(x["q"], x["k"], x["v"], grid, window, ORC_ORDER[order])
+    check_bf16(_host(out), ref, case)
+
+
 @pytest.mark.parametrize("grid", [(21, 22, 40), (21, 44, 80)])
 def test_full_attention_wan_sizes_sampled_rows(grid):
     n = grid[0] * grid[1] * grid[2]
