@@ -387,7 +387,8 @@ __global__ void __launch_bounds__(kThreads, 1) short_kernel(const __grid_constan
           }
           float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-          for (int i = 0; i < 64; ++i) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(r[i]));
+          for (int i = 0; i < 32; ++i)
+            mx[i & 3] = fmax3(mx[i & 3], __uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
           const float cm = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;
           if (c == 0) {
             m = cm;   // chunk 0 holds at least one column of the sequence: finite
@@ -415,10 +416,10 @@ __global__ void __launch_bounds__(kThreads, 1) short_kernel(const __grid_constan
           uint32_t pk[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
-            const float x0 = ex2_approx(fmaf(__uint_as_float(r[2 * j]), sl2, nm));
-            const float x1 = ex2_approx(fmaf(__uint_as_float(r[2 * j + 1]), sl2, nm));
-            ls[(2 * j) & 3] += x0;
-            ls[(2 * j + 1) & 3] += x1;
+            float e0, e1;
+            ffma2(e0, e1, __uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]), sl2, sl2, nm, nm);
+            const float x0 = ex2_approx(e0), x1 = ex2_approx(e1);
+            fadd2(ls[2 * (j & 1)], ls[2 * (j & 1) + 1], x0, x1);
             pk[j] = pack_bf16x2(x0, x1);
           }
           tmem_st32_nowait(t_s + 32 * c, pk);   // over scores already read; waited for below
