@@ -14,6 +14,7 @@
 
 #include "squad_attn.h"
 #include "geometry.cuh"
+#include "host_util.h"
 #include "kpass_plan.h"
 #include "bwd_pass.h"
 #include "bwd_stream.h"
@@ -248,19 +249,6 @@ bool tc_eligible(const squad_params_t* prm, const Grid& g, const PassGeom& p) {
   return true;
 }
 
-int num_sms_current() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-  static std::atomic<int> cache[64];   // per device; 0 = not looked up yet (calls may come from many threads)
-  if (dev >= 0 && dev < 64) {
-    const int c = cache[dev].load(std::memory_order_relaxed);
-    if (c > 0) return c;
-  }
-  int sms = 0;
-  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-  if (dev >= 0 && dev < 64) cache[dev].store(sms, std::memory_order_relaxed);
-  return sms;
-}
 
 // Sequences of at most 256 tokens run whole (one TMA box, one K/V block) in the short-sequence kernel.
 bool short_eligible(const squad_params_t* prm, const Grid& g, const PassGeom& p) {

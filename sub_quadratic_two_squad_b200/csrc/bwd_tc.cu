@@ -8,9 +8,10 @@
 //   dP = dO V^T,  D_i = sum_j P_ij dP_ij = dO_i . O_i,  dS = P o (dP - D),
 //   dQ = scale dS K,  dK = scale dS^T Q,  dV = P^T dO.
 //
-// One kernel per pass, one CTA per sequence (160 threads): warps 0-3 own one TMEM lane (one row) per
-// thread, warp 4 loads the sequence's Q, K (first) and V, dO once as whole TMA boxes and issues the
-// tcgen05 MMAs.
+// One kernel per pass, persistent (one CTA per SM, 160 threads, sequences taken in turn): warps 0-3
+// own one TMEM lane (one row) per thread, warp 4 loads each sequence's Q, K (first) and V, dO once as
+// whole TMA boxes and issues the tcgen05 MMAs. A sequence's loads are issued once the previous
+// sequence's products have completed, so they land while its last gradients are written out.
 //   rows, per 128-query tile: each warp forms D from its rows of dO (shared memory) and O (global)
 //     while S = Q K^T and dP = dO V^T go into TMEM; then dS = P o (dP - D) in one pass over the
 //     scores (bf16, packed two per column over S); dQ = dS K (A from TMEM) is written out. Each row's
@@ -42,7 +43,7 @@ constexpr uint32_t kBwdSmemMin = 120u * 1024u;
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct BwdBars {
-  uint64_t load_qk, load_vd, s_full, p_full, o_full, o_free, drain;
+  uint64_t load_qk, load_vd, s_full, p_full, o_full, o_free, drain, rows_done;
   uint32_t tmem_base;
   uint32_t abort;
 };
@@ -138,11 +139,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
   const int s = p.seq_len;
   const int N = round16b(s);
   const int ntiles = (s + 127) / 128;
-  const int bh = static_cast<int>(fdiv(blockIdx.x, p.f_per_bh));
-  const int sigma = static_cast<int>(blockIdx.x) - bh * p.n_seq;
+  const int seqs = g.B * g.h * p.n_seq;
 
   // Rows past the sequence in each allocation, and the guard past the last one, are read by the MMAs:
-  // zero them (the TMA boxes write exactly s rows per panel).
+  // zero them once (the TMA boxes write exactly s rows per panel, sequence after sequence).
   {
     const uint32_t tail = panel - static_cast<uint32_t>(s) * 128u;   // bytes per panel
     const uint32_t tail16 = tail / 16u;
@@ -161,6 +161,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
     mbar_init(&bars->o_full, 1);
     mbar_init(&bars->o_free, 128);
     mbar_init(&bars->drain, 1);
+    mbar_init(&bars->rows_done, 128);
     bars->abort = 0;
     fence_mbar_init();
   }
@@ -191,22 +192,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
       prefetch_tmap(&a.tm_v);
       prefetch_tmap(&a.tm_do);
       const uint32_t tx_half = 4u * static_cast<uint32_t>(s) * 128u;   // two tensors, both panels
-      mbar_arrive_expect_tx(&bars->load_qk, tx_half);
-      mbar_arrive_expect_tx(&bars->load_vd, tx_half);
-      int c[5];
-      chunk_coords(g, p, a.variant, bh, sigma, 0, 0, c);
-      const CUtensorMap* maps[4] = {&a.tm_q, &a.tm_k, &a.tm_v, &a.tm_do};
-      uint8_t* dsts[4] = {sq, sk, sv, sdo};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        uint64_t* bar = i < 2 ? &bars->load_qk : &bars->load_vd;
-        tma_load_5d(dsts[i], maps[i], bar, c[0], c[1], c[2], c[3], c[4]);
-        tma_load_5d(dsts[i] + panel, maps[i], bar, c[0] + 64, c[1], c[2], c[3], c[4]);
-      }
-      bool ok = mbar_wait(&bars->load_qk, 0, ctl);
-      tc_fence_after();
       const uint32_t aq = smem_u32(sq), ak = smem_u32(sk), av = smem_u32(sv), ado = smem_u32(sdo);
-      uint32_t p_cnt = 0, f_cnt = 0;
+      uint32_t p_cnt = 0, f_cnt = 0, oc = 0, issued = 0;
       // the row owners have read the previous results (dQ, or dV and dK) out of tensor memory
       auto wait_free = [&]() -> bool {
         const bool r = mbar_wait(&bars->o_free, f_cnt & 1, ctl);
@@ -218,6 +205,34 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
       const uint32_t idesc_s = idesc_bf16(128, N, false);
       const bool own_dq = dq_own_columns(N);
       const uint32_t qcol = own_dq ? 384u : static_cast<uint32_t>(N);
+      bool ok = true;
+      bool pending = false;   // an o_full whose o_free has not been waited for
+      uint32_t it = 0;
+      for (int seq = static_cast<int>(blockIdx.x); ok && seq < seqs; seq += static_cast<int>(gridDim.x), ++it) {
+        if (it > 0) {
+          // the previous sequence's products have read all of its operand tiles
+          ok = mbar_wait(&bars->o_full, (oc - 1) & 1u, ctl);
+          if (!ok) break;
+        }
+        {
+          const int bh = static_cast<int>(fdiv(static_cast<uint32_t>(seq), p.f_per_bh));
+          int c[5];
+          chunk_coords(g, p, a.variant, bh, seq - bh * p.n_seq, 0, 0, c);
+          mbar_arrive_expect_tx(&bars->load_qk, tx_half);
+          mbar_arrive_expect_tx(&bars->load_vd, tx_half);
+          const CUtensorMap* maps[4] = {&a.tm_q, &a.tm_k, &a.tm_v, &a.tm_do};
+          uint8_t* dsts[4] = {sq, sk, sv, sdo};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            uint64_t* bar = i < 2 ? &bars->load_qk : &bars->load_vd;
+            tma_load_5d(dsts[i], maps[i], bar, c[0], c[1], c[2], c[3], c[4]);
+            tma_load_5d(dsts[i] + panel, maps[i], bar, c[0] + 64, c[1], c[2], c[3], c[4]);
+          }
+          ++issued;
+        }
+        ok = mbar_wait(&bars->load_qk, it & 1u, ctl);
+        if (!ok) break;
+        tc_fence_after();
       for (int t = 0; t < ntiles && ok; ++t) {
         // dQ over dP's columns: the previous tile's dQ must have been read before S and dP are written
         if (t > 0 && !own_dq && !(ok = wait_free())) break;
@@ -225,9 +240,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
         for (int kk = 0; kk < 8; ++kk)   // S = Q_t K^T -> [0, N)
           umma_bf16_ss(tmem, kdesc(aq + row_off, kk, panel), kdesc(ak, kk, panel), idesc_s, kk > 0);
         if (t == 0) {
-          ok = mbar_wait(&bars->load_vd, 0, ctl);
+          ok = mbar_wait(&bars->load_vd, it & 1u, ctl);
           if (!ok) break;
           tc_fence_after();
+          // dP (and dQ) reach the columns of the previous sequence's dV and dK: read out by now
+          if (pending) {
+            if (!(ok = wait_free())) break;
+            pending = false;
+          }
         }
         for (int kk = 0; kk < 8; ++kk)   // dP = dO_t V^T -> [N, 2N)
           umma_bf16_ss(tmem + N, kdesc(ado + row_off, kk, panel), kdesc(av, kk, panel), idesc_s, kk > 0);
@@ -241,11 +261,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
         for (int kk = 0; kk < N / 16; ++kk)   // dQ = dS K
           umma_bf16_ts(tmem + qcol, tmem + kk * 8, sw128_desc(ak + kk * 2048, panel, 1024), idesc_o, kk > 0);
         umma_commit(&bars->o_full);
+        ++oc;
       }
       // columns: per 128-key tile, over 128-query chunks, S^T and dP^T, then dV += P^T dO, dK += dS^T Q.
       // S^T and dP^T ([0, 256)) wait for the last dQ only where it overlaps them; dV and dK ([256, 512))
       // wait for the last dQ, or the previous key tile's dV and dK, to have been read.
-      bool pending = ok;   // an o_full whose o_free has not been waited for
+      pending = ok;
       for (int kt = 0; kt < ntiles && ok; ++kt) {
         if (kt == 0 && !own_dq) {
           if (!(ok = wait_free())) break;
@@ -280,12 +301,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
         }
         if (ok) {
           umma_commit(&bars->o_full);
+          ++oc;
           pending = true;
         }
       }
-      // every MMA issued has completed before the CTA frees tensor memory
+      }
+      // every MMA issued has completed before the CTA frees tensor memory, and every load issued has
+      // landed before it exits
       umma_commit(&bars->drain);
       mbar_wait_drain(&bars->drain, 0, 20000000ull);
+      if (issued > 0) {
+        mbar_wait_drain(&bars->load_qk, (issued - 1) & 1u, 20000000ull);
+        mbar_wait_drain(&bars->load_vd, (issued - 1) & 1u, 20000000ull);
+      }
     }
   } else {
     // ------------------------------------------------------------------ row-owner warps
@@ -294,8 +322,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
     const float sl2 = a.scale_log2;
     uint32_t s_cnt = 0, o_cnt = 0;
     bool ok = true;
-    // rows: D, dS, dQ; each row's LSE (log2 units) and D go to shared memory for the columns
     const uint32_t qcol = dq_own_columns(N) ? 384u : static_cast<uint32_t>(N);
+    uint32_t it = 0;
+    for (int seq = static_cast<int>(blockIdx.x); ok && seq < seqs; seq += static_cast<int>(gridDim.x), ++it) {
+    const int bh = static_cast<int>(fdiv(static_cast<uint32_t>(seq), p.f_per_bh));
+    const int sigma = seq - bh * p.n_seq;
+    // rows: D, dS, dQ; each row's LSE (log2 units) and D go to shared memory for the columns
     for (int t = 0; t < ntiles && ok; ++t) {
       const int r = 128 * t + rl;
       const int tok = r < s ? token_of(g, p, sigma, 0, r) : -1;
@@ -309,7 +341,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
         for (int i = 0; i < 16; ++i) orow[i] = tok >= 0 ? src[i] : make_uint4(0, 0, 0, 0);
       }
       if (t == 0) {
-        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->load_vd, 0, ctl));
+        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->load_vd, it & 1u, ctl));
         if (!ok) break;
       }
       const float D = tok >= 0 ? row_dot_out(sdo, panel, r, orow) : 0.f;
@@ -353,7 +385,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
       tc_fence_before();
       mbar_arrive(&bars->o_free);
     }
-    named_barrier_sync(1, 128);   // every row's LSE and D is in shared memory before the columns use them
+    if (!ok) break;
+    // every row's LSE and D is in shared memory before the columns use them (a bounded wait: a warp
+    // that gave up never arrives)
+    mbar_arrive(&bars->rows_done);
+    ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->rows_done, it & 1u, ctl));
     // columns: P^T, dS^T per 128-query chunk; dV and dK once the chunks are accumulated
     for (int kt = 0; kt < ntiles && ok; ++kt) {
       const int key = 128 * kt + rl;
@@ -406,6 +442,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
       tc_fence_before();
       mbar_arrive(&bars->o_free);
     }
+    }
   }
   // tcgen05.dealloc is warp-wide and aligned: reconverge warp 4 (lane 0 arrives from the issue loop)
   __syncwarp();
@@ -419,18 +456,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
 }
 
 // ------------------------------------------------------------------------------------------------
-// Sequences of at most 128 tokens: one query tile and one key tile. A CTA takes `pack` consecutive
+// Sequences of at most 128 tokens: one query tile and one key tile. A work item is `pack` consecutive
 // sequences (of all B h n_seq), each in its own band of `seg` rows (the length rounded up to 8) of
 // every tile; S and dP are computed once over the whole tile, and a score counts only where query and
 // key lie in the same band (P = dS = 0 elsewhere, so the products stay block-diagonal). The
 // row-owner warps write P and dS (bf16) to shared memory, and dQ = dS K, dV = P^T dO and dK = dS^T Q
 // are three products read from there (P^T and dS^T as MN-major A operands of the same tiles).
+//
+// Persistent: one CTA per SM takes items blockIdx.x, blockIdx.x + gridDim.x, ... Once the three
+// products of an item have completed, its operand tiles are dead, so the next item's loads are issued
+// while the owners write this item's gradients out; the next dP is computed meanwhile, and the next S
+// as soon as the owners have read dK out of the columns S reuses.
 // ------------------------------------------------------------------------------------------------
 constexpr uint32_t kPdsPanel = 16384;   // 128 query rows x 64 keys (bf16), 128-byte swizzle
 
-// kPacked: several sequences per CTA (128-row operand tiles, a band per sequence). Otherwise one
-// sequence per CTA, its operand tiles as long as the sequence (rounded to 8 rows) with a zeroed guard
-// past the last one.
+// kPacked: several sequences per item (128-row operand tiles, a band per sequence). Otherwise one
+// sequence per item, its operand tiles as long as the sequence (rounded to 8 rows) with a zeroed
+// guard past the last one.
 template <bool kPacked>
 __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc1_kernel(const __grid_constant__ BwdTcArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -450,13 +492,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc1_kernel(const __grid_co
   const int s = p.seq_len;
   const int seg = a.seg_rows;                                   // band of one sequence (s rounded to 8)
   const int total = g.B * g.h * p.n_seq;                        // sequences of all (b, head)
-  const int first = static_cast<int>(blockIdx.x) * a.pack;      // this CTA's first sequence
-  const int nseq = min(a.pack, total - first);                  // sequences in this CTA
-  const int N = round16b(nseq * seg);                           // key (and query) rows in use
+  const int n_items = (total + a.pack - 1) / a.pack;
 
   if constexpr (!kPacked) {
     // Rows past the sequence in each tile, and the guard past the last one, are read by the MMAs:
-    // zero them (the TMA boxes write exactly s rows per panel).
+    // zero them once (the TMA boxes write exactly s rows per panel, item after item).
     const uint32_t tail = panel - static_cast<uint32_t>(s) * 128u;   // bytes per panel
     const uint32_t tail16 = tail / 16u;
     for (uint32_t i = threadIdx.x; i < 8u * tail16; i += kBwdThreads) {
@@ -473,6 +513,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc1_kernel(const __grid_co
     mbar_init(&bars->s_full, 1);
     mbar_init(&bars->p_full, 128);
     mbar_init(&bars->o_full, 1);
+    mbar_init(&bars->o_free, 128);   // the owners have read dK: S of the next item may overwrite it
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
     fence_mbar_init();
@@ -489,14 +530,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc1_kernel(const __grid_co
   WaitCtl ctl{&bars->abort, a.status, a.timeout_ns};
   const bool tmem_ok = tmem == 0u;   // all 512 columns requested: anything else is an error
   if (!tmem_ok && threadIdx.x == 0 && a.status != nullptr) atomicCAS(a.status, 0u, kStatusTimeout);
-  const uint32_t tx_half = static_cast<uint32_t>(nseq) * 4u * static_cast<uint32_t>(s) * 128u;
-  if (tmem_ok && threadIdx.x == 128) {
-    // the loads: each sequence's boxes into its band (a multiple of 8 rows, so the 128-byte swizzle
-    // phase is kept)
-    prefetch_tmap(&a.tm_q);
-    prefetch_tmap(&a.tm_k);
-    prefetch_tmap(&a.tm_v);
-    prefetch_tmap(&a.tm_do);
+
+  // The loads of one item: each sequence's boxes into its band (a multiple of 8 rows, so the 128-byte
+  // swizzle phase is kept); Q and K on one barrier, V and dO on the other.
+  auto issue_loads = [&](int item) {
+    const int first = item * a.pack, nseq = min(a.pack, total - first);
+    const uint32_t tx_half = static_cast<uint32_t>(nseq) * 4u * static_cast<uint32_t>(s) * 128u;
     mbar_arrive_expect_tx(&bars->load_qk, tx_half);
     mbar_arrive_expect_tx(&bars->load_vd, tx_half);
     const CUtensorMap* maps[4] = {&a.tm_q, &a.tm_k, &a.tm_v, &a.tm_do};
@@ -514,14 +553,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc1_kernel(const __grid_co
         tma_load_5d(dsts[i] + panel + row_off, maps[i], bar, c[0] + 64, c[1], c[2], c[3], c[4]);
       }
     }
+  };
+  uint32_t issued = 0;   // items whose loads this CTA has issued (thread 128)
+  if (tmem_ok && threadIdx.x == 128 && static_cast<int>(blockIdx.x) < n_items) {
+    issued = 1;
+    prefetch_tmap(&a.tm_q);
+    prefetch_tmap(&a.tm_k);
+    prefetch_tmap(&a.tm_v);
+    prefetch_tmap(&a.tm_do);
+    issue_loads(static_cast<int>(blockIdx.x));
   }
   if constexpr (kPacked) {
     // Meanwhile, the rows of each tile that no box writes (the gap after each sequence in its band,
-    // and the rows past the last band) are zeroed: the MMAs read them.
+    // and the rows past the last band) are zeroed once: the MMAs read them. On an item with fewer
+    // sequences than bands, the unused bands hold an earlier item's (finite) rows, which only meet
+    // zero P and dS.
+    const int nseq0 = min(a.pack, total - static_cast<int>(blockIdx.x) * a.pack);   // this CTA's first item
     for (uint32_t i = threadIdx.x; i < 8u * 128u; i += kBwdThreads) {   // (panel, row) pairs
       const int row = static_cast<int>(i & 127u);
       const int band = row / seg, pos = row - band * seg;
-      if (band < nseq && pos < s) continue;
+      if (band < nseq0 && pos < s) continue;
       uint4* dst = reinterpret_cast<uint4*>(base + (i >> 7) * panel + static_cast<uint32_t>(row) * 128u);
 #pragma unroll
       for (int j = 0; j < 8; ++j) dst[j] = make_uint4(0, 0, 0, 0);
@@ -535,28 +586,40 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc1_kernel(const __grid_co
     // nothing issued: fall through to the release below
   } else if (warp == 4) {
     if (lane == 0) {
-      // ---------------------------------------------------------------- MMA issue (loads above)
+      // ---------------------------------------------------------------- loads and MMA issue
       const uint32_t aq = smem_u32(sq), ak = smem_u32(sk), av = smem_u32(sv), ado = smem_u32(sdo);
       const uint32_t ap = smem_u32(sp), ads = smem_u32(sds);
-      const uint32_t idesc_s = idesc_bf16(128, N, false);
-      bool ok = mbar_wait(&bars->load_qk, 0, ctl);
-      if (ok) {
+      const uint32_t idesc_q = idesc_bf16(128, 128, true);   // A K-major (dS), B MN-major (K)
+      const uint32_t idesc_t = idesc_bf16_a_mn(128, 128);    // A = P^T / dS^T, B = dO / Q
+      bool ok = true;
+      uint32_t it = 0;
+      for (int item = static_cast<int>(blockIdx.x); ok && item < n_items; item += static_cast<int>(gridDim.x), ++it) {
+        const uint32_t ph = it & 1u;
+        const int nseq = min(a.pack, total - item * a.pack);
+        const int N = round16b(nseq * seg);   // key (and query) rows in use
+        const uint32_t idesc_s = idesc_bf16(128, N, false);
+        if (it > 0) {
+          // the previous item's products have read all of its operand tiles: load this item's
+          ok = mbar_wait(&bars->o_full, ph ^ 1u, ctl);
+          if (!ok) break;
+          issue_loads(item);
+          ++issued;
+        }
+        ok = mbar_wait(&bars->load_qk, ph, ctl);
+        if (ok && it > 0) ok = mbar_wait(&bars->o_free, ph ^ 1u, ctl);   // dK of the previous item read
+        if (!ok) break;
         tc_fence_after();
         for (int kk = 0; kk < 8; ++kk)   // S = Q K^T -> [0, N)
           umma_bf16_ss(tmem, kdesc(aq, kk, panel), kdesc(ak, kk, panel), idesc_s, kk > 0);
-        ok = mbar_wait(&bars->load_vd, 0, ctl);
-      }
-      if (ok) {
+        ok = mbar_wait(&bars->load_vd, ph, ctl);
+        if (!ok) break;
         tc_fence_after();
         for (int kk = 0; kk < 8; ++kk)   // dP = dO V^T -> [128, 128 + N)
           umma_bf16_ss(tmem + 128, kdesc(ado, kk, panel), kdesc(av, kk, panel), idesc_s, kk > 0);
         umma_commit(&bars->s_full);
-        ok = mbar_wait(&bars->p_full, 0, ctl);
-      }
-      if (ok) {
+        ok = mbar_wait(&bars->p_full, ph, ctl);
+        if (!ok) break;
         tc_fence_after();
-        const uint32_t idesc_q = idesc_bf16(128, 128, true);   // A K-major (dS), B MN-major (K)
-        const uint32_t idesc_t = idesc_bf16_a_mn(128, 128);    // A = P^T / dS^T, B = dO / Q
         for (int kk = 0; kk < N / 16; ++kk)   // dQ = dS K -> [256, 384)
           umma_bf16_ss(tmem + 256, kdesc(ads, kk, kPdsPanel), sw128_desc(ak + kk * 2048, panel, 1024), idesc_q,
                        kk > 0);
@@ -568,41 +631,53 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc1_kernel(const __grid_co
                        idesc_t, kk > 0);
         umma_commit(&bars->o_full);
       }
-      // every MMA issued has completed before the CTA frees tensor memory
+      // every MMA issued has completed before the CTA frees tensor memory, and every load issued has
+      // landed before it exits
       umma_commit(&bars->drain);
       mbar_wait_drain(&bars->drain, 0, 20000000ull);
+      if (issued > 0) {
+        mbar_wait_drain(&bars->load_qk, (issued - 1) & 1u, 20000000ull);
+        mbar_wait_drain(&bars->load_vd, (issued - 1) & 1u, 20000000ull);
+      }
     }
   } else {
     // ------------------------------------------------------------------ row-owner warps
     const int r = warp * 32 + lane;   // TMEM lane = query row = key row of this thread
     const uint32_t t_row = tmem + (static_cast<uint32_t>(warp * 32) << 16);
     const float sl2 = a.scale_log2;
-    const int band = r / seg, pos = r - band * seg;   // this row's sequence within the CTA, and position
-    int tok = -1, bh = 0;
-    if (band < nseq && pos < s) {
-      const int gs = first + band;
-      bh = static_cast<int>(fdiv(static_cast<uint32_t>(gs), p.f_per_bh));
-      tok = token_of(g, p, gs - bh * p.n_seq, 0, pos);
-    }
-    const int k0 = band * seg;   // the row's own keys: columns [k0, k0 + s)
-    const size_t gi = static_cast<size_t>(bh) * g.n + (tok < 0 ? 0 : tok);
-    const float lse2 = tok >= 0 ? a.lse[gi] * kLog2e : 0.f;
-    uint4 orow[16];
-    {
-      const uint4* src = reinterpret_cast<const uint4*>(a.o + gi * 128);
+    const int band = r / seg, pos = r - band * seg;   // this row's sequence within the item, and position
+    const int k0 = band * seg;                        // the row's own keys: columns [k0, k0 + s)
+    const uint32_t row_p = smem_u32(sp) + static_cast<uint32_t>(r) * 128u;
+    const uint32_t row_ds = smem_u32(sds) + static_cast<uint32_t>(r) * 128u;
+    const uint32_t sw = static_cast<uint32_t>(r & 7);
+    bool ok = true;
+    uint32_t it = 0;
+    for (int item = static_cast<int>(blockIdx.x); ok && item < n_items; item += static_cast<int>(gridDim.x), ++it) {
+      const uint32_t ph = it & 1u;
+      const int first = item * a.pack;
+      const int nseq = min(a.pack, total - first);
+      const int N = round16b(nseq * seg);
+      int tok = -1, bh = 0;
+      if (band < nseq && pos < s) {
+        const int gs = first + band;
+        bh = static_cast<int>(fdiv(static_cast<uint32_t>(gs), p.f_per_bh));
+        tok = token_of(g, p, gs - bh * p.n_seq, 0, pos);
+      }
+      const size_t gi = static_cast<size_t>(bh) * g.n + (tok < 0 ? 0 : tok);
+      const float lse2 = tok >= 0 ? a.lse[gi] * kLog2e : 0.f;
+      uint4 orow[16];
+      {
+        const uint4* src = reinterpret_cast<const uint4*>(a.o + gi * 128);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) orow[i] = tok >= 0 ? src[i] : make_uint4(0, 0, 0, 0);
-    }
-    bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->load_vd, 0, ctl));
-    const float D = (ok && tok >= 0) ? row_dot_out(sdo, panel, r, orow) : 0.f;   // D_i = dO_i . O_i
-    if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->s_full, 0, ctl));
-    if (ok) {
+        for (int i = 0; i < 16; ++i) orow[i] = tok >= 0 ? src[i] : make_uint4(0, 0, 0, 0);
+      }
+      ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->load_vd, ph, ctl));
+      const float D = (ok && tok >= 0) ? row_dot_out(sdo, panel, r, orow) : 0.f;   // D_i = dO_i . O_i
+      if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->s_full, ph, ctl));
+      if (!ok) break;
       tc_fence_after();
       // P and dS = P o (dP - D) of this row, bf16, into shared memory (zero outside the row's own
       // sequence, and on rows of no sequence: those rows are K rows of dV and dK)
-      const uint32_t row_p = smem_u32(sp) + static_cast<uint32_t>(r) * 128u;
-      const uint32_t row_ds = smem_u32(sds) + static_cast<uint32_t>(r) * 128u;
-      const uint32_t sw = static_cast<uint32_t>(r & 7);
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         uint32_t pp[16], pd[16];
@@ -637,20 +712,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc1_kernel(const __grid_co
       fence_proxy_async_smem();   // P and dS -> visible to the MMAs (async proxy)
       tc_fence_before();
       mbar_arrive(&bars->p_full);
-      ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->o_full, 0, ctl));
-    }
-    if (ok) {
+      ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->o_full, ph, ctl));
+      if (!ok) break;
       tc_fence_after();
+      // dK first: its columns are where the next item's S goes
       const size_t ro = gi * 128;
+      if (a.final_out)
+        write_row(t_row, tok >= 0, a.scale, a.accumulate ? a.dk_acc + ro : nullptr, a.dk_out + ro, nullptr);
+      else
+        write_row(t_row, tok >= 0, a.scale, a.accumulate ? a.dk_acc + ro : nullptr, nullptr, a.dk_acc + ro);
+      tc_fence_before();
+      mbar_arrive(&bars->o_free);
       if (a.final_out)
         write_row(t_row + 256, tok >= 0, a.scale, a.accumulate ? a.dq_acc + ro : nullptr, a.dq_out + ro, nullptr);
       else
         write_row(t_row + 256, tok >= 0, a.scale, a.accumulate ? a.dq_acc + ro : nullptr, nullptr, a.dq_acc + ro);
       write_row(t_row + 384, tok >= 0, 1.f, nullptr, a.dv_out + ro, nullptr);
-      if (a.final_out)
-        write_row(t_row, tok >= 0, a.scale, a.accumulate ? a.dk_acc + ro : nullptr, a.dk_out + ro, nullptr);
-      else
-        write_row(t_row, tok >= 0, a.scale, a.accumulate ? a.dk_acc + ro : nullptr, nullptr, a.dk_acc + ro);
     }
   }
   __syncwarp();
@@ -675,12 +752,18 @@ cudaError_t launch_bwd_tc(const BwdTcArgs& a, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   const int seqs = a.g.B * a.g.h * a.p.n_seq;
   if (seqs == 0) return cudaSuccess;
-  if (a.single && a.pack > 1)
-    bwd_tc1_kernel<true><<<static_cast<unsigned>((seqs + a.pack - 1) / a.pack), kBwdThreads, a.smem_bytes, stream>>>(a);
-  else if (a.single)
-    bwd_tc1_kernel<false><<<static_cast<unsigned>(seqs), kBwdThreads, a.smem_bytes, stream>>>(a);
-  else
-    bwd_tc_kernel<<<static_cast<unsigned>(seqs), kBwdThreads, a.smem_bytes, stream>>>(a);
+  if (a.single) {
+    // persistent: one CTA per SM (each takes more than half of an SM's shared memory)
+    const int items = (seqs + a.pack - 1) / a.pack, sms = num_sms_current();
+    const unsigned grid = static_cast<unsigned>(sms > 0 && sms < items ? sms : items);
+    if (a.pack > 1)
+      bwd_tc1_kernel<true><<<grid, kBwdThreads, a.smem_bytes, stream>>>(a);
+    else
+      bwd_tc1_kernel<false><<<grid, kBwdThreads, a.smem_bytes, stream>>>(a);
+  } else {
+    const int sms = num_sms_current();
+    bwd_tc_kernel<<<static_cast<unsigned>(sms > 0 && sms < seqs ? sms : seqs), kBwdThreads, a.smem_bytes, stream>>>(a);
+  }
   return cudaGetLastError();
 }
 

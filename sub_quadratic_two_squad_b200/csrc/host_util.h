@@ -23,4 +23,19 @@ cudaError_t max_dyn_smem_once(Kernel kernel, int bytes, std::atomic<unsigned lon
   return e;
 }
 
+// Number of SMs of the current device (0 if it cannot be read), looked up once per device.
+inline int num_sms_current() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  static std::atomic<int> cache[64];   // per device; 0 = not looked up yet (calls may come from many threads)
+  if (dev >= 0 && dev < 64) {
+    const int c = cache[dev].load(std::memory_order_relaxed);
+    if (c > 0) return c;
+  }
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  if (dev >= 0 && dev < 64) cache[dev].store(sms, std::memory_order_relaxed);
+  return sms;
+}
+
 }  // namespace squad
