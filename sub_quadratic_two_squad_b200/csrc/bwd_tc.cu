@@ -35,7 +35,7 @@ namespace squad {
 
 namespace {
 
-constexpr int kBwdThreads = 160;
+constexpr int kBwdThreads = 288;   // 4 row-owner warps, 4 epilogue warps, 1 load/MMA warp
 constexpr uint32_t kBwdSmemLimit = 232448;
 // Each CTA takes all 512 TMEM columns, so it also takes more than half of an SM's shared memory:
 // no second CTA is ever resident beside it waiting for tensor memory.
@@ -43,7 +43,7 @@ constexpr uint32_t kBwdSmemMin = 120u * 1024u;
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct BwdBars {
-  uint64_t load_qk, load_vd, s_full, p_full, o_full, o_free, drain, rows_done;
+  uint64_t load_qk, load_vd, s_full, p_full, o_full, o_free, drain, rows_done, epi_free;
   uint32_t tmem_base;
   uint32_t abort;
 };
@@ -153,7 +153,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
     for (uint32_t i = threadIdx.x; i < a.guard_bytes / 16u; i += kBwdThreads)
       reinterpret_cast<uint4*>(base + 4 * alloc)[i] = make_uint4(0, 0, 0, 0);
   }
-  if (threadIdx.x == 128) {
+  if (threadIdx.x == 256) {
     mbar_init(&bars->load_qk, 1);
     mbar_init(&bars->load_vd, 1);
     mbar_init(&bars->s_full, 1);
@@ -165,7 +165,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
     bars->abort = 0;
     fence_mbar_init();
   }
-  if (warp == 4) {
+  if (warp == 8) {
     __syncwarp();
     tmem_alloc(&bars->tmem_base, 512);
     tmem_relinquish();
@@ -184,7 +184,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
 
   if (!tmem_ok) {
     // nothing issued: fall through to the release below
-  } else if (warp == 4) {
+  } else if (warp == 8) {
     if (lane == 0) {
       // ---------------------------------------------------------------- loads + MMA issue
       prefetch_tmap(&a.tm_q);
@@ -194,7 +194,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
       const uint32_t tx_half = 4u * static_cast<uint32_t>(s) * 128u;   // two tensors, both panels
       const uint32_t aq = smem_u32(sq), ak = smem_u32(sk), av = smem_u32(sv), ado = smem_u32(sdo);
       uint32_t p_cnt = 0, f_cnt = 0, oc = 0, issued = 0;
-      // the row owners have read the previous results (dQ, or dV and dK) out of tensor memory
+      // the epilogue warps have read the previous results (dQ, or dV and dK) out of tensor memory
       auto wait_free = [&]() -> bool {
         const bool r = mbar_wait(&bars->o_free, f_cnt & 1, ctl);
         ++f_cnt;
@@ -315,14 +315,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
         mbar_wait_drain(&bars->load_vd, (issued - 1) & 1u, 20000000ull);
       }
     }
-  } else {
+  } else if (warp < 4) {
     // ------------------------------------------------------------------ row-owner warps
     const int rl = warp * 32 + lane;   // TMEM lane of this thread
     const uint32_t t_row = tmem + (static_cast<uint32_t>(warp * 32) << 16);
     const float sl2 = a.scale_log2;
-    uint32_t s_cnt = 0, o_cnt = 0;
+    uint32_t s_cnt = 0;
     bool ok = true;
-    const uint32_t qcol = dq_own_columns(N) ? 384u : static_cast<uint32_t>(N);
     uint32_t it = 0;
     for (int seq = static_cast<int>(blockIdx.x); ok && seq < seqs; seq += static_cast<int>(gridDim.x), ++it) {
     const int bh = static_cast<int>(fdiv(static_cast<uint32_t>(seq), p.f_per_bh));
@@ -371,19 +370,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bars->p_full);
-      ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->o_full, o_cnt & 1, ctl));
-      ++o_cnt;
-      if (!ok) break;
-      tc_fence_after();
-      {
-        const size_t ro = gi * 128;
-        if (a.final_out)
-          write_row(t_row + qcol, tok >= 0, a.scale, a.accumulate ? a.dq_acc + ro : nullptr, a.dq_out + ro, nullptr);
-        else
-          write_row(t_row + qcol, tok >= 0, a.scale, a.accumulate ? a.dq_acc + ro : nullptr, nullptr, a.dq_acc + ro);
-      }
-      tc_fence_before();
-      mbar_arrive(&bars->o_free);
     }
     if (!ok) break;
     // every row's LSE and D is in shared memory before the columns use them (a bounded wait: a warp
@@ -392,9 +378,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
     ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->rows_done, it & 1u, ctl));
     // columns: P^T, dS^T per 128-query chunk; dV and dK once the chunks are accumulated
     for (int kt = 0; kt < ntiles && ok; ++kt) {
-      const int key = 128 * kt + rl;
-      const int tok = key < s ? token_of(g, p, sigma, 0, key) : -1;
-      const size_t gi = static_cast<size_t>(bh) * g.n + (tok < 0 ? 0 : tok);
       for (int qc = 0; qc < ntiles && ok; ++qc) {
         ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->s_full, s_cnt & 1, ctl));
         ++s_cnt;
@@ -426,30 +409,51 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
         tc_fence_before();
         mbar_arrive(&bars->p_full);
       }
-      if (!ok) break;
-      ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->o_full, o_cnt & 1, ctl));
-      ++o_cnt;
-      if (!ok) break;
-      tc_fence_after();
-      {
-        const size_t ro = gi * 128;
-        write_row(t_row + 256, tok >= 0, 1.f, nullptr, a.dv_out + ro, nullptr);
-        if (a.final_out)
-          write_row(t_row + 384, tok >= 0, a.scale, a.accumulate ? a.dk_acc + ro : nullptr, a.dk_out + ro, nullptr);
-        else
-          write_row(t_row + 384, tok >= 0, a.scale, a.accumulate ? a.dk_acc + ro : nullptr, nullptr, a.dk_acc + ro);
-      }
-      tc_fence_before();
-      mbar_arrive(&bars->o_free);
     }
+    }
+  } else {
+    // ------------------------------------------------------------------ epilogue warps
+    // dQ of each row tile, then dV and dK of each key tile, as the products complete; warp 4 + w reads
+    // the TMEM lanes of owner warp w.
+    const int rl = (warp - 4) * 32 + lane;
+    const uint32_t t_row = tmem + (static_cast<uint32_t>((warp - 4) * 32) << 16);
+    const uint32_t qcol = dq_own_columns(N) ? 384u : static_cast<uint32_t>(N);
+    uint32_t o_cnt = 0;
+    bool ok = true;
+    for (int seq = static_cast<int>(blockIdx.x); ok && seq < seqs; seq += static_cast<int>(gridDim.x)) {
+      const int bh = static_cast<int>(fdiv(static_cast<uint32_t>(seq), p.f_per_bh));
+      const int sigma = seq - bh * p.n_seq;
+      for (int t = 0; t < 2 * ntiles && ok; ++t) {   // row tiles, then key tiles
+        const int r = 128 * (t < ntiles ? t : t - ntiles) + rl;
+        const int tok = r < s ? token_of(g, p, sigma, 0, r) : -1;
+        const size_t ro = (static_cast<size_t>(bh) * g.n + (tok < 0 ? 0 : tok)) * 128;
+        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->o_full, o_cnt & 1, ctl));
+        ++o_cnt;
+        if (!ok) break;
+        tc_fence_after();
+        if (t < ntiles) {
+          if (a.final_out)
+            write_row(t_row + qcol, tok >= 0, a.scale, a.accumulate ? a.dq_acc + ro : nullptr, a.dq_out + ro, nullptr);
+          else
+            write_row(t_row + qcol, tok >= 0, a.scale, a.accumulate ? a.dq_acc + ro : nullptr, nullptr, a.dq_acc + ro);
+        } else {
+          write_row(t_row + 256, tok >= 0, 1.f, nullptr, a.dv_out + ro, nullptr);
+          if (a.final_out)
+            write_row(t_row + 384, tok >= 0, a.scale, a.accumulate ? a.dk_acc + ro : nullptr, a.dk_out + ro, nullptr);
+          else
+            write_row(t_row + 384, tok >= 0, a.scale, a.accumulate ? a.dk_acc + ro : nullptr, nullptr, a.dk_acc + ro);
+        }
+        tc_fence_before();
+        mbar_arrive(&bars->o_free);
+      }
     }
   }
-  // tcgen05.dealloc is warp-wide and aligned: reconverge warp 4 (lane 0 arrives from the issue loop)
+  // tcgen05.dealloc is warp-wide and aligned: reconverge warp 8 (lane 0 arrives from the issue loop)
   __syncwarp();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 4) {
+  if (warp == 8) {
     __syncwarp();
     tmem_dealloc(tmem, 512);
   }
@@ -463,10 +467,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
 // row-owner warps write P and dS (bf16) to shared memory, and dQ = dS K, dV = P^T dO and dK = dS^T Q
 // are three products read from there (P^T and dS^T as MN-major A operands of the same tiles).
 //
-// Persistent: one CTA per SM takes items blockIdx.x, blockIdx.x + gridDim.x, ... Once the three
-// products of an item have completed, its operand tiles are dead, so the next item's loads are issued
-// while the owners write this item's gradients out; the next dP is computed meanwhile, and the next S
-// as soon as the owners have read dK out of the columns S reuses.
+// Persistent: one CTA per SM takes items blockIdx.x, blockIdx.x + gridDim.x, ... 288 threads: warps
+// 0-3 own the rows (D, P and dS), warps 4-7 write the gradients out (a thread per row again: warp
+// 4 + w reads the TMEM lanes of warp w), warp 8 loads and issues the MMAs. Once the three products of
+// an item have completed its operand tiles are dead, so the next item's loads are issued while the
+// epilogue warps write this item's gradients out; the next dP is computed meanwhile, the next S as
+// soon as dK has been read out of the columns S reuses, and the owners form the next P and dS while
+// dQ and dV are still being written.
 // ------------------------------------------------------------------------------------------------
 constexpr uint32_t kPdsPanel = 16384;   // 128 query rows x 64 keys (bf16), 128-byte swizzle
 
@@ -507,18 +514,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc1_kernel(const __grid_co
       reinterpret_cast<uint4*>(base + 4 * alloc)[i] = make_uint4(0, 0, 0, 0);
     fence_proxy_async_smem();   // zeroed rows -> visible to the MMAs (async proxy)
   }
-  if (threadIdx.x == 128) {
+  if (threadIdx.x == 256) {
     mbar_init(&bars->load_qk, 1);
     mbar_init(&bars->load_vd, 1);
     mbar_init(&bars->s_full, 1);
     mbar_init(&bars->p_full, 128);
     mbar_init(&bars->o_full, 1);
-    mbar_init(&bars->o_free, 128);   // the owners have read dK: S of the next item may overwrite it
+    mbar_init(&bars->o_free, 128);     // dK read out: S of the next item may overwrite it
+    mbar_init(&bars->epi_free, 128);   // dQ and dV read out: the next item's products may overwrite them
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
     fence_mbar_init();
   }
-  if (warp == 4) {
+  if (warp == 8) {
     __syncwarp();
     tmem_alloc(&bars->tmem_base, 512);
     tmem_relinquish();
@@ -554,8 +562,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc1_kernel(const __grid_co
       }
     }
   };
-  uint32_t issued = 0;   // items whose loads this CTA has issued (thread 128)
-  if (tmem_ok && threadIdx.x == 128 && static_cast<int>(blockIdx.x) < n_items) {
+  uint32_t issued = 0;   // items whose loads this CTA has issued (thread 256)
+  if (tmem_ok && threadIdx.x == 256 && static_cast<int>(blockIdx.x) < n_items) {
     issued = 1;
     prefetch_tmap(&a.tm_q);
     prefetch_tmap(&a.tm_k);
@@ -584,7 +592,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc1_kernel(const __grid_co
   // Tensor memory: S [0, N) then dK [0, 128); dP [128, 128 + N); dQ [256, 384); dV [384, 512).
   if (!tmem_ok) {
     // nothing issued: fall through to the release below
-  } else if (warp == 4) {
+  } else if (warp == 8) {
     if (lane == 0) {
       // ---------------------------------------------------------------- loads and MMA issue
       const uint32_t aq = smem_u32(sq), ak = smem_u32(sk), av = smem_u32(sv), ado = smem_u32(sdo);
@@ -618,6 +626,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc1_kernel(const __grid_co
           umma_bf16_ss(tmem + 128, kdesc(ado, kk, panel), kdesc(av, kk, panel), idesc_s, kk > 0);
         umma_commit(&bars->s_full);
         ok = mbar_wait(&bars->p_full, ph, ctl);
+        if (ok && it > 0) ok = mbar_wait(&bars->epi_free, ph ^ 1u, ctl);   // dQ, dV of the previous item read
         if (!ok) break;
         tc_fence_after();
         for (int kk = 0; kk < N / 16; ++kk)   // dQ = dS K -> [256, 384)
@@ -640,7 +649,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc1_kernel(const __grid_co
         mbar_wait_drain(&bars->load_vd, (issued - 1) & 1u, 20000000ull);
       }
     }
-  } else {
+  } else if (warp < 4) {
     // ------------------------------------------------------------------ row-owner warps
     const int r = warp * 32 + lane;   // TMEM lane = query row = key row of this thread
     const uint32_t t_row = tmem + (static_cast<uint32_t>(warp * 32) << 16);
@@ -712,11 +721,28 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc1_kernel(const __grid_co
       fence_proxy_async_smem();   // P and dS -> visible to the MMAs (async proxy)
       tc_fence_before();
       mbar_arrive(&bars->p_full);
-      ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->o_full, ph, ctl));
+    }
+  } else {
+    // ------------------------------------------------------------------ epilogue warps
+    const int r = (warp - 4) * 32 + lane;   // the row of owner warp (warp - 4), lane `lane`
+    const uint32_t t_row = tmem + (static_cast<uint32_t>((warp - 4) * 32) << 16);
+    const int band = r / seg, pos = r - band * seg;
+    bool ok = true;
+    uint32_t it = 0;
+    for (int item = static_cast<int>(blockIdx.x); ok && item < n_items; item += static_cast<int>(gridDim.x), ++it) {
+      const int first = item * a.pack;
+      const int nseq = min(a.pack, total - first);
+      int tok = -1, bh = 0;
+      if (band < nseq && pos < s) {
+        const int gs = first + band;
+        bh = static_cast<int>(fdiv(static_cast<uint32_t>(gs), p.f_per_bh));
+        tok = token_of(g, p, gs - bh * p.n_seq, 0, pos);
+      }
+      const size_t ro = (static_cast<size_t>(bh) * g.n + (tok < 0 ? 0 : tok)) * 128;
+      ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->o_full, it & 1u, ctl));
       if (!ok) break;
       tc_fence_after();
       // dK first: its columns are where the next item's S goes
-      const size_t ro = gi * 128;
       if (a.final_out)
         write_row(t_row, tok >= 0, a.scale, a.accumulate ? a.dk_acc + ro : nullptr, a.dk_out + ro, nullptr);
       else
@@ -728,13 +754,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc1_kernel(const __grid_co
       else
         write_row(t_row + 256, tok >= 0, a.scale, a.accumulate ? a.dq_acc + ro : nullptr, nullptr, a.dq_acc + ro);
       write_row(t_row + 384, tok >= 0, 1.f, nullptr, a.dv_out + ro, nullptr);
+      tc_fence_before();
+      mbar_arrive(&bars->epi_free);
     }
   }
   __syncwarp();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 4) {
+  if (warp == 8) {
     __syncwarp();
     tmem_dealloc(tmem, 512);
   }
