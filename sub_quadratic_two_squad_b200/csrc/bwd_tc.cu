@@ -359,11 +359,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int j = 32 * c + 2 * i;
-          const float p0 = j < s ? ex2_approx(fmaf(__uint_as_float(sr[2 * i]), sl2, -lse2)) : 0.f;
-          const float p1 = j + 1 < s ? ex2_approx(fmaf(__uint_as_float(sr[2 * i + 1]), sl2, -lse2)) : 0.f;
-          const float s0 = j < s ? p0 * (__uint_as_float(dr[2 * i]) - D) : 0.f;
-          const float s1 = j + 1 < s ? p1 * (__uint_as_float(dr[2 * i + 1]) - D) : 0.f;
-          pk[i] = pack2_rn(s0, s1);
+          float e0, e1, d0, d1, s0, s1;
+          ffma2(e0, e1, __uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1]), sl2, sl2, -lse2, -lse2);
+          ffma2(d0, d1, __uint_as_float(dr[2 * i]), __uint_as_float(dr[2 * i + 1]), 1.f, 1.f, -D, -D);
+          fmul2(s0, s1, ex2_approx(e0), ex2_approx(e1), d0, d1);
+          pk[i] = pack2_rn(j < s ? s0 : 0.f, j + 1 < s ? s1 : 0.f);
         }
         tmem_st16_nowait(t_row + 16 * c, pk);   // waited for below, before the MMA reads dS
       }
@@ -395,12 +395,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
             const int j0 = 128 * qc + 32 * c + 2 * i;   // query index of the column pair
             const int jl = 32 * c + 2 * i;               // within this chunk
             const bool v0 = jl < nq, v1 = jl + 1 < nq;
-            const float p0 = v0 ? ex2_approx(fmaf(__uint_as_float(sr[2 * i]), sl2, -lse_s[j0])) : 0.f;
-            const float p1 = v1 ? ex2_approx(fmaf(__uint_as_float(sr[2 * i + 1]), sl2, -lse_s[j0 + 1])) : 0.f;
-            const float s0 = v0 ? p0 * (__uint_as_float(dr[2 * i]) - d_s[j0]) : 0.f;
-            const float s1 = v1 ? p1 * (__uint_as_float(dr[2 * i + 1]) - d_s[j0 + 1]) : 0.f;
+            float e0, e1, d0, d1, s0, s1;
+            ffma2(e0, e1, __uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1]), sl2, sl2, -lse_s[j0],
+                  -lse_s[j0 + 1]);
+            ffma2(d0, d1, __uint_as_float(dr[2 * i]), __uint_as_float(dr[2 * i + 1]), 1.f, 1.f, -d_s[j0], -d_s[j0 + 1]);
+            const float p0 = v0 ? ex2_approx(e0) : 0.f, p1 = v1 ? ex2_approx(e1) : 0.f;
+            fmul2(s0, s1, p0, p1, d0, d1);
             pp[i] = pack2_rn(p0, p1);
-            ps[i] = pack2_rn(s0, s1);
+            ps[i] = pack2_rn(v0 ? s0 : 0.f, v1 ? s1 : 0.f);
           }
           tmem_st16_nowait(t_row + 16 * c, pp);
           tmem_st16_nowait(t_row + 128 + 16 * c, ps);
@@ -698,12 +700,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc1_kernel(const __grid_co
           for (int i = 0; i < 16; ++i) {
             const int j = 32 * c + 2 * i - k0;   // key position within the row's own sequence
             const bool v0 = tok >= 0 && j >= 0 && j < s, v1 = tok >= 0 && j + 1 >= 0 && j + 1 < s;
-            const float p0 = v0 ? ex2_approx(fmaf(__uint_as_float(sr[2 * i]), sl2, -lse2)) : 0.f;
-            const float p1 = v1 ? ex2_approx(fmaf(__uint_as_float(sr[2 * i + 1]), sl2, -lse2)) : 0.f;
-            const float s0 = v0 ? p0 * (__uint_as_float(dr[2 * i]) - D) : 0.f;
-            const float s1 = v1 ? p1 * (__uint_as_float(dr[2 * i + 1]) - D) : 0.f;
+            float e0, e1, d0, d1, s0, s1;
+            ffma2(e0, e1, __uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1]), sl2, sl2, -lse2, -lse2);
+            ffma2(d0, d1, __uint_as_float(dr[2 * i]), __uint_as_float(dr[2 * i + 1]), 1.f, 1.f, -D, -D);
+            const float p0 = v0 ? ex2_approx(e0) : 0.f, p1 = v1 ? ex2_approx(e1) : 0.f;
+            fmul2(s0, s1, p0, p1, d0, d1);
             pp[i] = pack2_rn(p0, p1);
-            pd[i] = pack2_rn(s0, s1);
+            pd[i] = pack2_rn(v0 ? s0 : 0.f, v1 ? s1 : 0.f);
           }
         } else {
 #pragma unroll
