@@ -294,12 +294,12 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_rows_kernel(const __grid_cons
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int k0 = 32 * c + 2 * i;
-          const float p0 = k0 < nk ? ex2_approx(fmaf(__uint_as_float(sr[2 * i]), sl2, -lse2)) : 0.f;
-          const float p1 = k0 + 1 < nk ? ex2_approx(fmaf(__uint_as_float(sr[2 * i + 1]), sl2, -lse2)) : 0.f;
-          // columns past the chunk hold unwritten tensor memory: zero them without reading
-          const float s0 = k0 < nk ? p0 * (__uint_as_float(dr[2 * i]) - D) : 0.f;
-          const float s1 = k0 + 1 < nk ? p1 * (__uint_as_float(dr[2 * i + 1]) - D) : 0.f;
-          pk[i] = pack_bf16x2(s0, s1);
+          float e0, e1, d0, d1, s0, s1;
+          ffma2(e0, e1, __uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1]), sl2, sl2, -lse2, -lse2);
+          ffma2(d0, d1, __uint_as_float(dr[2 * i]), __uint_as_float(dr[2 * i + 1]), 1.f, 1.f, -D, -D);
+          fmul2(s0, s1, ex2_approx(e0), ex2_approx(e1), d0, d1);
+          // columns past the chunk hold unwritten tensor memory: whatever was formed there is dropped
+          pk[i] = pack_bf16x2(k0 < nk ? s0 : 0.f, k0 + 1 < nk ? s1 : 0.f);
         }
         tmem_st16_nowait(t_row + 16 * c, pk);   // over scores already read; waited for below
       }
@@ -433,12 +433,13 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_cols_kernel(const __grid_cons
         for (int q = 0; q < 16; ++q) {
           const int j0 = 32 * c + 2 * q;   // query column within the chunk
           const bool v0 = j0 < nq, v1 = j0 + 1 < nq;
-          const float p0 = v0 ? ex2_approx(fmaf(__uint_as_float(sr[2 * q]), sl2, -ls[j0])) : 0.f;
-          const float p1 = v1 ? ex2_approx(fmaf(__uint_as_float(sr[2 * q + 1]), sl2, -ls[j0 + 1])) : 0.f;
-          const float s0 = v0 ? p0 * (__uint_as_float(dr[2 * q]) - dd[j0]) : 0.f;
-          const float s1 = v1 ? p1 * (__uint_as_float(dr[2 * q + 1]) - dd[j0 + 1]) : 0.f;
+          float e0, e1, d0, d1, s0, s1;
+          ffma2(e0, e1, __uint_as_float(sr[2 * q]), __uint_as_float(sr[2 * q + 1]), sl2, sl2, -ls[j0], -ls[j0 + 1]);
+          ffma2(d0, d1, __uint_as_float(dr[2 * q]), __uint_as_float(dr[2 * q + 1]), 1.f, 1.f, -dd[j0], -dd[j0 + 1]);
+          const float p0 = v0 ? ex2_approx(e0) : 0.f, p1 = v1 ? ex2_approx(e1) : 0.f;
+          fmul2(s0, s1, p0, p1, d0, d1);
           pp[q] = pack_bf16x2(p0, p1);
-          ps[q] = pack_bf16x2(s0, s1);
+          ps[q] = pack_bf16x2(v0 ? s0 : 0.f, v1 ? s1 : 0.f);
         }
         tmem_st16_nowait(t_row + 16 * c, pp);
         tmem_st16_nowait(t_row + 128 + 16 * c, ps);
