@@ -1,5 +1,6 @@
 // Arguments and launcher of the chunked tensor-core backward (bwd_stream.cu): one SQuad pass's
-// gradients for sequences of any length, cut into chunks of at most 128 rows, one CTA per chunk.
+// gradients for sequences of any length, cut into chunks of at most 128 rows, persistent CTAs taking
+// the chunks in turn.
 #pragma once
 
 #include <cuda.h>
