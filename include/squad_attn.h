@@ -113,7 +113,9 @@ SQUAD_API squad_status_t squad_attn_fwd_status(const squad_params_t* p, const vo
 
 /* Bytes of backward workspace: fp32 partial dQ and dK, the gradient of the pass-1 output, the per-row
  * softmax-Jacobian terms of each pass, and a control block (for a padded grid: sized for the padded n,
- * plus the zero-padded dout and the gradients on the padded grid). Returns 0 for invalid params. */
+ * plus the zero-padded dout and the gradients on the padded grid); when a pass has sequences of 129 to
+ * 208 tokens, also the bf16 P and dS of one sequence per resident CTA (160 slots of at most 208 KB,
+ * independent of n). Returns 0 for invalid params. */
 SQUAD_API size_t squad_attn_bwd_workspace_bytes(const squad_params_t* p);
 
 /* SQuad-Attention backward (the pages print no formula; it is the chain rule through both passes).

@@ -154,12 +154,15 @@ struct BwdWorkspace {
   float* do1;
   float* drow;
   void *dop, *dqp, *dkp, *dvp;   // padded grids only: dout zero-padded, gradients on the padded grid
+  uint8_t* pds;                  // the whole-sequence kernel's P/dS scratch slots (last; may be empty)
 };
 
 size_t bwd_ws_bytes(const Grid& g, size_t eb, bool padded) {
   const size_t bhn = static_cast<size_t>(g.B) * g.h * g.n;
   return ctrl_bytes(g) + 3 * align256(bhn * g.d * 4) + align256(bhn * 4) + (padded ? 4 * align256(bhn * g.d * eb) : 0);
 }
+
+size_t pds_bytes(const squad_params_t* sp, const Grid& g);
 
 BwdWorkspace carve_bwd(void* ws, const Grid& g, size_t eb, bool padded) {
   uint8_t* b = static_cast<uint8_t*>(ws);
@@ -182,7 +185,9 @@ BwdWorkspace carve_bwd(void* ws, const Grid& g, size_t eb, bool padded) {
     w.dqp = b + t;
     w.dkp = b + 2 * t;
     w.dvp = b + 3 * t;
+    b += 4 * t;
   }
+  w.pds = b;
   return w;
 }
 
@@ -419,7 +424,7 @@ size_t squad_attn_bwd_workspace_bytes(const squad_params_t* p) {
   float sc;
   PadDims pd;
   if (validate(p, true, &g, &sc, &pd) != SQUAD_OK) return 0;
-  return bwd_ws_bytes(g, elem_bytes(p), pd.padded);
+  return bwd_ws_bytes(g, elem_bytes(p), pd.padded) + pds_bytes(p, g);
 }
 
 }  // extern "C"
@@ -517,6 +522,22 @@ int bwd_kernel_of(const squad_params_t* sp, const Grid& g, int kind) {
   return SQUAD_BWD_CUDA_CORE;
 }
 
+// Bytes of P/dS scratch the whole-sequence backward kernel needs for either pass of this problem (0
+// when no pass of more than 128 tokens runs on it).
+size_t pds_bytes(const squad_params_t* sp, const Grid& g) {
+  size_t m = 0;
+  if (sp->dtype != SQUAD_BF16) return 0;
+  for (const int kind : {kLocal, kGlobal}) {
+    BwdTcArgs b;
+    std::memset(&b, 0, sizeof(b));
+    b.g = g;
+    b.p = make_geom(g, kind, 256);
+    if (short_eligible(sp, g, b.p) && bwd_tc_plan(b) && !b.single)
+      m = std::max(m, static_cast<size_t>(kBwdPdsSlots) * b.pds_slot_bytes);
+  }
+  return align256(m);
+}
+
 // One pass's backward inside a chain of passes. accumulate: add the fp32 dQ/dK shares already in the
 // accumulators; final_out: write dq, dk (input dtype) instead of the accumulators. dv_out receives the
 // gradient of this pass's values in the input dtype; out is this pass's forward output (the chunked
@@ -524,7 +545,7 @@ int bwd_kernel_of(const squad_params_t* sp, const Grid& g, int kind) {
 squad_status_t bwd_one_pass(const squad_params_t* sp, const Grid& g, int kind, float scale, const void* q,
                             const void* k, const void* values, const void* out, const void* dout, const float* lse,
                             uint32_t* status, float* dq_acc, float* dk_acc, float* drow, void* dq, void* dk,
-                            void* dv_out, bool accumulate, bool final_out, cudaStream_t stream) {
+                            void* dv_out, bool accumulate, bool final_out, uint8_t* pds, cudaStream_t stream) {
   const bool bf16 = sp->dtype == SQUAD_BF16;
   const int kernel = bwd_kernel_of(sp, g, kind);
   if (kernel == SQUAD_BWD_TC_WHOLE) {
@@ -550,6 +571,7 @@ squad_status_t bwd_one_pass(const squad_params_t* sp, const Grid& g, int kind, f
       b.scale_log2 = scale * 1.4426950408889634f;
       b.status = status;
       b.timeout_ns = kWaitTimeoutNs;
+      b.pds = pds;
       return launch_bwd_tc(b, stream) == cudaSuccess ? SQUAD_OK : SQUAD_ERR_CUDA;
     }
   }
@@ -613,7 +635,7 @@ squad_status_t bwd_core(const squad_params_t* p, const Grid& g, float scale, con
     // One pass: values v, upstream dout, the pass's LSE in the first slot; no share to add.
     const int kind = p->order == SQUAD_LOCAL_ONLY ? kLocal : kGlobal;
     return bwd_one_pass(p, g, kind, scale, q, k, v, o, dout, fw.lse1, bw.status, bw.dq_acc, bw.dk_acc, bw.drow,
-                        dq, dk, dv, /*accumulate=*/false, /*final_out=*/true, stream);
+                        dq, dk, dv, /*accumulate=*/false, /*final_out=*/true, bw.pds, stream);
   }
   const int first = p->order == SQUAD_LOCAL_THEN_GLOBAL ? kLocal : kGlobal;
   const int second = p->order == SQUAD_LOCAL_THEN_GLOBAL ? kGlobal : kLocal;
@@ -645,6 +667,7 @@ squad_status_t bwd_core(const squad_params_t* p, const Grid& g, float scale, con
         b->scale_log2 = scale * 1.4426950408889634f;
         b->status = bw.status;
         b->timeout_ns = kWaitTimeoutNs;
+        b->pds = bw.pds;
       }
       b2.lse = fw.lse2;
       b2.o = static_cast<const __nv_bfloat16*>(o);
@@ -666,10 +689,10 @@ squad_status_t bwd_core(const squad_params_t* p, const Grid& g, float scale, con
       // cores); dO1 is bf16 as in the fused pair.
       squad_status_t st = bwd_one_pass(p, g, second, scale, q, k, fw.o1, o, dout, fw.lse2, bw.status, bw.dq_acc,
                                        bw.dk_acc, bw.drow, dq, dk, bw.do1, /*accumulate=*/false,
-                                       /*final_out=*/false, stream);
+                                       /*final_out=*/false, bw.pds, stream);
       if (st != SQUAD_OK) return st;
       return bwd_one_pass(p, g, first, scale, q, k, v, fw.o1, bw.do1, fw.lse1, bw.status, bw.dq_acc, bw.dk_acc,
-                          bw.drow, dq, dk, dv, /*accumulate=*/true, /*final_out=*/true, stream);
+                          bw.drow, dq, dk, dv, /*accumulate=*/true, /*final_out=*/true, bw.pds, stream);
     }
   }
 
@@ -846,12 +869,20 @@ struct KpassBwdWs {
   float* dk_acc;
   float* drow;      // [B, h, n] per-row softmax-Jacobian terms (CUDA-core kernels)
   void* gbuf[2];    // value gradients passed between consecutive passes (input dtype)
+  uint8_t* pds;     // the whole-sequence kernel's P/dS scratch slots (last; may be empty)
 };
+
+// P/dS scratch of the largest whole-sequence level of the chain (0 if none runs on that kernel).
+size_t kpass_pds_bytes(const KpassPlan& pl) {
+  size_t m = 0;
+  for (int l = 0; l < pl.k; ++l) m = std::max(m, pds_bytes(&pl.sub[l], pl.g[l]));
+  return m;
+}
 
 size_t kpass_bwd_bytes(const KpassPlan& pl) {
   const size_t d = static_cast<size_t>(pl.sub[0].d);
   const size_t t = align256(pl.bhn * d * pl.eb), f = align256(pl.bhn * d * 4), l = align256(pl.bhn * 4);
-  return kKpassCtrlBytes + 2 * f + l + static_cast<size_t>(kpass_n_gbuf(pl.k)) * t;
+  return kKpassCtrlBytes + 2 * f + l + static_cast<size_t>(kpass_n_gbuf(pl.k)) * t + kpass_pds_bytes(pl);
 }
 
 KpassBwdWs carve_kpass_bwd(void* ws, const KpassPlan& pl) {
@@ -869,6 +900,7 @@ KpassBwdWs carve_kpass_bwd(void* ws, const KpassPlan& pl) {
   b += l;
   w.gbuf[0] = kpass_n_gbuf(pl.k) > 0 ? b : nullptr;
   w.gbuf[1] = kpass_n_gbuf(pl.k) > 1 ? b + t : nullptr;
+  w.pds = b + static_cast<size_t>(kpass_n_gbuf(pl.k)) * t;
   return w;
 }
 
@@ -959,7 +991,7 @@ squad_status_t squad_kpass_bwd(const squad_kpass_params_t* p, const void* q, con
     const void* out = e + 1 == p->k ? o : fw.inter[e];   // this pass's output: the next pass's values
     const squad_status_t ps = bwd_one_pass(&pl.sub[l], pl.g[l], pl.kind[l], pl.scale, q, k, values, out, g_in,
                                            fw.lse[st.lse], bw.ctrl, bw.dq_acc, bw.dk_acc, bw.drow, dq, dk, g_out,
-                                           st.accumulate, st.final_out, stream);
+                                           st.accumulate, st.final_out, bw.pds, stream);
     if (ps != SQUAD_OK) return ps;
   }
   return SQUAD_OK;

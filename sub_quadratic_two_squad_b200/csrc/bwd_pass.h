@@ -33,11 +33,21 @@ struct BwdTcArgs {
   uint32_t guard_bytes, smem_bytes;
   uint32_t* status;           // device status word (0 = ok, 4 = a wait timed out)
   unsigned long long timeout_ns;
+  uint8_t* pds;               // whole-sequence kernel: kBwdPdsSlots slots of pds_slot_bytes (P and dS of
+                              // one sequence, bf16, written in the row phase, read by the column phase)
+  uint32_t pds_slot_bytes;
 };
+
+// Scratch of the whole-sequence backward: one slot per resident CTA, each holding a sequence's P and dS
+// (bf16) in the layout of two 128-key operand tiles (two 64-key panels of at most 208 rows, 128-byte
+// swizzle): 8 panels of at most 208 x 128 bytes.
+constexpr int kBwdPdsSlots = 160;
+constexpr size_t kBwdPdsSlotMaxBytes = 8u * 208u * 128u;
+constexpr size_t kBwdPdsScratchBytes = static_cast<size_t>(kBwdPdsSlots) * kBwdPdsSlotMaxBytes;
 
 // Fills the shared-memory plan of `a` (p and g set); false if the sequences do not fit.
 bool bwd_tc_plan(BwdTcArgs& a);
-// One pass's gradients: dQ, then dK and dV, in one launch (one CTA per sequence).
+// One pass's gradients: dQ, then dK and dV, in one persistent launch (the two-tile kernel needs `pds`).
 cudaError_t launch_bwd_tc(const BwdTcArgs& a, cudaStream_t stream);
 
 }  // namespace squad

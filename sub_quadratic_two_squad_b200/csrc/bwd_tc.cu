@@ -8,19 +8,23 @@
 //   dP = dO V^T,  D_i = sum_j P_ij dP_ij = dO_i . O_i,  dS = P o (dP - D),
 //   dQ = scale dS K,  dK = scale dS^T Q,  dV = P^T dO.
 //
-// One kernel per pass, persistent (one CTA per SM, 160 threads, sequences taken in turn): warps 0-3
-// own one TMEM lane (one row) per thread, warp 4 loads each sequence's Q, K (first) and V, dO once as
-// whole TMA boxes and issues the tcgen05 MMAs. A sequence's loads are issued once the previous
-// sequence's products have completed, so they land while its last gradients are written out.
+// One kernel per pass, persistent (one CTA per SM, sequences taken in turn), 288 threads: warps 0-3 own
+// one TMEM lane (one row) per thread, warps 4-7 write the gradients out (warp 4 + w reads the lanes of
+// warp w), warp 8 loads each sequence's Q, K (first) and V, dO once as whole TMA boxes and issues the
+// tcgen05 MMAs. A sequence's loads are issued once the previous sequence's products have completed,
+// so they land while its last gradients are written out.
+// Sequences of 129-208 tokens (bwd_tc_kernel):
 //   rows, per 128-query tile: each warp forms D from its rows of dO (shared memory) and O (global)
-//     while S = Q K^T and dP = dO V^T go into TMEM; then dS = P o (dP - D) in one pass over the
-//     scores (bf16, packed two per column over S); dQ = dS K (A from TMEM) is written out. Each row's
-//     LSE and D stay in shared memory. Where tensor memory has room, dQ has columns of its own, so the
-//     next tile's S and dP (or the first S^T and dP^T) are computed while it is written out.
-//   columns, per 128-key tile and 128-query chunk: S^T = K Q^T and dP^T = V dO^T into TMEM; with the
-//     per-query LSE and D the warps form P^T and dS^T (packed over S^T and dP^T); dV += P^T dO and
-//     dK += dS^T Q accumulate in TMEM over the chunks and are written out (the next key tile's S^T
-//     and dP^T are computed meanwhile).
+//     while S = Q K^T and dP = dO V^T go into TMEM; then P and dS = P o (dP - D) in one pass over the
+//     scores (bf16): dS packed two per column over S for dQ = dS K (A from TMEM), and P and dS of the
+//     row written to the CTA's scratch slot in global memory, in the layout of 128-key operand
+//     tiles. Where tensor memory has room, dQ has columns of its own, so the next tile's S and dP are
+//     computed while it is written out.
+//   columns, per 128-key tile: that tile's P and dS come back from the slot (L2) into the K and V
+//     allocations, free once the row products are done, by bulk copies, and dV = P^T dO and
+//     dK = dS^T Q are two products over all queries (P^T and dS^T as MN-major A operands). No score
+//     is computed twice.
+// Sequences of at most 128 tokens (bwd_tc1_kernel): one tile each way, P and dS through shared memory.
 // Rows past the sequence are computed and dropped; columns past it are masked to P = dS = 0, and the
 // shared-memory rows past each box are zeroed so every MMA operand is finite.
 #include <cuda_runtime.h>
@@ -43,7 +47,8 @@ constexpr uint32_t kBwdSmemMin = 120u * 1024u;
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct BwdBars {
-  uint64_t load_qk, load_vd, s_full, p_full, o_full, o_free, drain, rows_done, epi_free;
+  uint64_t load_qk, load_vd, s_full, p_full, o_full, o_free, drain, epi_free;
+  uint64_t pds_ready, pds_full, pds_empty;   // whole-sequence kernel: P and dS through the scratch slot
   uint32_t tmem_base;
   uint32_t abort;
 };
@@ -129,9 +134,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
   uint8_t* const sk = base + alloc;
   uint8_t* const sv = base + 2 * alloc;
   uint8_t* const sdo = base + 3 * alloc;
-  float* const lse_s = reinterpret_cast<float*>(base + 4 * alloc + a.guard_bytes);   // per query, log2 units
-  float* const d_s = lse_s + 256;                                                     // per query D
-  BwdBars* const bars = reinterpret_cast<BwdBars*>(d_s + 256);
+  BwdBars* const bars = reinterpret_cast<BwdBars*>(base + 4 * alloc + a.guard_bytes + kBwdVecBytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const Grid& g = a.g;
@@ -153,6 +156,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
     for (uint32_t i = threadIdx.x; i < a.guard_bytes / 16u; i += kBwdThreads)
       reinterpret_cast<uint4*>(base + 4 * alloc)[i] = make_uint4(0, 0, 0, 0);
   }
+  // This CTA's scratch slot starts zeroed: its parts that no row writes (keys past the last column
+  // chunk) are read by the column products.
+  uint8_t* const pds = a.pds + static_cast<size_t>(blockIdx.x) * a.pds_slot_bytes;
+  for (uint32_t i = threadIdx.x; i < a.pds_slot_bytes / 16u; i += kBwdThreads)
+    reinterpret_cast<uint4*>(pds)[i] = make_uint4(0, 0, 0, 0);
+  fence_proxy_async_global();   // ... visible to the bulk copies (async proxy)
   if (threadIdx.x == 256) {
     mbar_init(&bars->load_qk, 1);
     mbar_init(&bars->load_vd, 1);
@@ -161,7 +170,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
     mbar_init(&bars->o_full, 1);
     mbar_init(&bars->o_free, 128);
     mbar_init(&bars->drain, 1);
-    mbar_init(&bars->rows_done, 128);
+    mbar_init(&bars->pds_ready, 128);   // the owners' P and dS rows of the sequence are in the slot
+    mbar_init(&bars->pds_full, 1);      // a key tile's P and dS landed in the K and V allocations
+    mbar_init(&bars->pds_empty, 1);     // ... and the products that read them are done
     bars->abort = 0;
     fence_mbar_init();
   }
@@ -193,7 +204,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
       prefetch_tmap(&a.tm_do);
       const uint32_t tx_half = 4u * static_cast<uint32_t>(s) * 128u;   // two tensors, both panels
       const uint32_t aq = smem_u32(sq), ak = smem_u32(sk), av = smem_u32(sv), ado = smem_u32(sdo);
-      uint32_t p_cnt = 0, f_cnt = 0, oc = 0, issued = 0;
+      uint32_t p_cnt = 0, f_cnt = 0, oc = 0, issued = 0, pf = 0, pe = 0;
       // the epilogue warps have read the previous results (dQ, or dV and dK) out of tensor memory
       auto wait_free = [&]() -> bool {
         const bool r = mbar_wait(&bars->o_free, f_cnt & 1, ctl);
@@ -263,47 +274,40 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
         umma_commit(&bars->o_full);
         ++oc;
       }
-      // columns: per 128-key tile, over 128-query chunks, S^T and dP^T, then dV += P^T dO, dK += dS^T Q.
-      // S^T and dP^T ([0, 256)) wait for the last dQ only where it overlaps them; dV and dK ([256, 512))
-      // wait for the last dQ, or the previous key tile's dV and dK, to have been read.
+      // columns, per 128-key tile kt: the owners' P and dS of the whole sequence (bf16, in this CTA's
+      // scratch slot) come into the K and V allocations, which the row phase's last products free, and
+      // dV += P^T dO and dK += dS^T Q run over all queries (P^T and dS^T as MN-major A operands) into
+      // [256, 384) and [384, 512), once the epilogue has read the last dQ, or the previous key tile's dV
+      // and dK, out of those columns. No scores are recomputed.
       pending = ok;
+      if (ok) ok = mbar_wait(&bars->pds_ready, it & 1u, ctl);
+      if (ok) ok = mbar_wait(&bars->o_full, (oc - 1) & 1u, ctl);   // the last dQ product has read K
+      const int Ns = round16b(s);
       for (int kt = 0; kt < ntiles && ok; ++kt) {
-        if (kt == 0 && !own_dq) {
+        if (kt > 0 && !(ok = mbar_wait(&bars->pds_empty, (pe - 1) & 1u, ctl))) break;
+        mbar_arrive_expect_tx(&bars->pds_full, 4u * panel);
+        bulk_load(sk, pds + static_cast<size_t>(4 * kt) * panel, 2u * panel, &bars->pds_full);       // P, keys of kt
+        bulk_load(sv, pds + static_cast<size_t>(4 * kt + 2) * panel, 2u * panel, &bars->pds_full);   // dS
+        ok = mbar_wait(&bars->pds_full, pf & 1u, ctl);
+        ++pf;
+        if (!ok) break;
+        if (pending) {
           if (!(ok = wait_free())) break;
           pending = false;
         }
-        const uint32_t key_off = static_cast<uint32_t>(kt) * 16384u;
-        for (int qc = 0; qc < ntiles && ok; ++qc) {
-          const int nq = min(128, s - 128 * qc);
-          const int Nq = round16b(nq);
-          const uint32_t q_off = static_cast<uint32_t>(qc) * 16384u;
-          const uint32_t idesc_c = idesc_bf16(128, Nq, false);
-          for (int kk = 0; kk < 8; ++kk)   // S^T = K_kt Q_qc^T -> [0, Nq)
-            umma_bf16_ss(tmem, kdesc(ak + key_off, kk, panel), kdesc(aq + q_off, kk, panel), idesc_c, kk > 0);
-          for (int kk = 0; kk < 8; ++kk)   // dP^T = V_kt dO_qc^T -> [128, 128 + Nq)
-            umma_bf16_ss(tmem + 128, kdesc(av + key_off, kk, panel), kdesc(ado + q_off, kk, panel), idesc_c,
-                         kk > 0);
-          umma_commit(&bars->s_full);
-          ok = mbar_wait(&bars->p_full, p_cnt & 1, ctl);
-          ++p_cnt;
-          if (!ok) break;
-          tc_fence_after();
-          if (qc == 0 && pending) {
-            if (!(ok = wait_free())) break;
-            pending = false;
-          }
-          for (int kk = 0; kk < Nq / 16; ++kk)   // dV += P^T dO_qc -> [256, 384)
-            umma_bf16_ts(tmem + 256, tmem + kk * 8, sw128_desc(ado + q_off + kk * 2048, panel, 1024), idesc_o,
-                         qc > 0 || kk > 0);
-          for (int kk = 0; kk < Nq / 16; ++kk)   // dK += dS^T Q_qc -> [384, 512)
-            umma_bf16_ts(tmem + 384, tmem + 128 + kk * 8, sw128_desc(aq + q_off + kk * 2048, panel, 1024), idesc_o,
-                         qc > 0 || kk > 0);
-        }
-        if (ok) {
-          umma_commit(&bars->o_full);
-          ++oc;
-          pending = true;
-        }
+        tc_fence_after();
+        const uint32_t idesc_t = idesc_bf16_a_mn(128, 128);   // A = P^T / dS^T, B = dO / Q (MN-major)
+        for (int kk = 0; kk < Ns / 16; ++kk)   // dV = P^T dO -> [256, 384)
+          umma_bf16_ss(tmem + 256, sw128_desc(ak + kk * 2048, panel, 1024), sw128_desc(ado + kk * 2048, panel, 1024),
+                       idesc_t, kk > 0);
+        for (int kk = 0; kk < Ns / 16; ++kk)   // dK = dS^T Q -> [384, 512)
+          umma_bf16_ss(tmem + 384, sw128_desc(av + kk * 2048, panel, 1024), sw128_desc(aq + kk * 2048, panel, 1024),
+                       idesc_t, kk > 0);
+        umma_commit(&bars->pds_empty);
+        ++pe;
+        umma_commit(&bars->o_full);
+        ++oc;
+        pending = true;
       }
       }
       // every MMA issued has completed before the CTA frees tensor memory, and every load issued has
@@ -326,7 +330,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
     for (int seq = static_cast<int>(blockIdx.x); ok && seq < seqs; seq += static_cast<int>(gridDim.x), ++it) {
     const int bh = static_cast<int>(fdiv(static_cast<uint32_t>(seq), p.f_per_bh));
     const int sigma = seq - bh * p.n_seq;
-    // rows: D, dS, dQ; each row's LSE (log2 units) and D go to shared memory for the columns
+    // rows: D, then P and dS of each 128-query tile; dS packed over S for dQ = dS K, and P and dS of
+    // every row also written to this CTA's scratch slot for the column products
+    const int rows = static_cast<int>(panel / 128u);   // rows of a scratch panel (the sequence rounded to 16)
     for (int t = 0; t < ntiles && ok; ++t) {
       const int r = 128 * t + rl;
       const int tok = r < s ? token_of(g, p, sigma, 0, r) : -1;
@@ -344,74 +350,54 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
         if (!ok) break;
       }
       const float D = tok >= 0 ? row_dot_out(sdo, panel, r, orow) : 0.f;
-      lse_s[r] = tok >= 0 ? lse2 : INFINITY;   // +inf past the sequence: P = 0 in those columns
-      d_s[r] = D;
       ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->s_full, s_cnt & 1, ctl));   // warp-uniform exit
       ++s_cnt;
       if (!ok) break;
       tc_fence_after();
-      // dS = P o (dP - D), P recomputed from S and the LSE; bf16, packed over the S columns already read
+      const bool put = r < rows;   // this row is one of the scratch tiles' rows
+      uint8_t* const row_p = pds + static_cast<size_t>(r) * 128u;
+      const uint32_t sw = static_cast<uint32_t>(r & 7);
+      // P = 2^(S scale log2e - LSE log2e) recomputed from S and the LSE, dS = P o (dP - D); both bf16,
+      // zero outside the sequence
 #pragma unroll 1
       for (int c = 0; c < (N + 31) / 32; ++c) {
-        uint32_t sr[32], dr[32], pk[16];
+        uint32_t sr[32], dr[32], pp[16], pk[16];
         tmem_ld32(t_row + 32 * c, sr);
         tmem_ld32(t_row + N + 32 * c, dr);
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int j = 32 * c + 2 * i;
+          const bool v0 = tok >= 0 && j < s, v1 = tok >= 0 && j + 1 < s;
           float e0, e1, d0, d1, s0, s1;
           ffma2(e0, e1, __uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1]), sl2, sl2, -lse2, -lse2);
           ffma2(d0, d1, __uint_as_float(dr[2 * i]), __uint_as_float(dr[2 * i + 1]), 1.f, 1.f, -D, -D);
-          fmul2(s0, s1, ex2_approx(e0), ex2_approx(e1), d0, d1);
-          pk[i] = pack2_rn(j < s ? s0 : 0.f, j + 1 < s ? s1 : 0.f);
+          const float p0 = v0 ? ex2_approx(e0) : 0.f, p1 = v1 ? ex2_approx(e1) : 0.f;
+          fmul2(s0, s1, p0, p1, d0, d1);
+          pp[i] = pack2_rn(p0, p1);
+          pk[i] = pack2_rn(v0 ? s0 : 0.f, v1 ? s1 : 0.f);
         }
         tmem_st16_nowait(t_row + 16 * c, pk);   // waited for below, before the MMA reads dS
+        if (put) {
+          // keys [32 c, 32 c + 32): key tile c / 4, its 64-key panel (c / 2) % 2, 16-byte chunks
+          // 4 (c % 2) .. + 3 of the row (128-byte swizzle)
+          const size_t pnl = static_cast<size_t>(4 * (c >> 2) + ((c >> 1) & 1)) * panel;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const uint32_t off = ((static_cast<uint32_t>(4 * (c & 1) + q)) ^ sw) << 4;
+            *reinterpret_cast<uint4*>(row_p + pnl + off) = make_uint4(pp[4 * q], pp[4 * q + 1], pp[4 * q + 2], pp[4 * q + 3]);
+            *reinterpret_cast<uint4*>(row_p + pnl + 2 * static_cast<size_t>(panel) + off) =
+                make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+          }
+        }
       }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bars->p_full);
     }
     if (!ok) break;
-    // every row's LSE and D is in shared memory before the columns use them (a bounded wait: a warp
-    // that gave up never arrives)
-    mbar_arrive(&bars->rows_done);
-    ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->rows_done, it & 1u, ctl));
-    // columns: P^T, dS^T per 128-query chunk; dV and dK once the chunks are accumulated
-    for (int kt = 0; kt < ntiles && ok; ++kt) {
-      for (int qc = 0; qc < ntiles && ok; ++qc) {
-        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->s_full, s_cnt & 1, ctl));
-        ++s_cnt;
-        if (!ok) break;
-        tc_fence_after();
-        const int nq = min(128, s - 128 * qc);
-        // P^T over S^T and dS^T over dP^T, both bf16 packed two per column
-#pragma unroll 1
-        for (int c = 0; c < (nq + 31) / 32; ++c) {
-          uint32_t sr[32], dr[32], pp[16], ps[16];
-          tmem_ld32(t_row + 32 * c, sr);
-          tmem_ld32(t_row + 128 + 32 * c, dr);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int j0 = 128 * qc + 32 * c + 2 * i;   // query index of the column pair
-            const int jl = 32 * c + 2 * i;               // within this chunk
-            const bool v0 = jl < nq, v1 = jl + 1 < nq;
-            float e0, e1, d0, d1, s0, s1;
-            ffma2(e0, e1, __uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1]), sl2, sl2, -lse_s[j0],
-                  -lse_s[j0 + 1]);
-            ffma2(d0, d1, __uint_as_float(dr[2 * i]), __uint_as_float(dr[2 * i + 1]), 1.f, 1.f, -d_s[j0], -d_s[j0 + 1]);
-            const float p0 = v0 ? ex2_approx(e0) : 0.f, p1 = v1 ? ex2_approx(e1) : 0.f;
-            fmul2(s0, s1, p0, p1, d0, d1);
-            pp[i] = pack2_rn(p0, p1);
-            ps[i] = pack2_rn(v0 ? s0 : 0.f, v1 ? s1 : 0.f);
-          }
-          tmem_st16_nowait(t_row + 16 * c, pp);
-          tmem_st16_nowait(t_row + 128 + 16 * c, ps);
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(&bars->p_full);
-      }
-    }
+    // the sequence's P and dS rows are in the slot: visible to the bulk copies of the column phase
+    fence_proxy_async_global();
+    mbar_arrive(&bars->pds_ready);
     }
   } else {
     // ------------------------------------------------------------------ epilogue warps
@@ -792,8 +778,11 @@ cudaError_t launch_bwd_tc(const BwdTcArgs& a, cudaStream_t stream) {
     else
       bwd_tc1_kernel<false><<<grid, kBwdThreads, a.smem_bytes, stream>>>(a);
   } else {
-    const int sms = num_sms_current();
-    bwd_tc_kernel<<<static_cast<unsigned>(sms > 0 && sms < seqs ? sms : seqs), kBwdThreads, a.smem_bytes, stream>>>(a);
+    if (a.pds == nullptr) return cudaErrorInvalidValue;
+    int grid = num_sms_current();
+    if (grid <= 0 || grid > kBwdPdsSlots) grid = kBwdPdsSlots;   // one scratch slot per CTA
+    if (grid > seqs) grid = seqs;
+    bwd_tc_kernel<<<static_cast<unsigned>(grid), kBwdThreads, a.smem_bytes, stream>>>(a);
   }
   return cudaGetLastError();
 }
@@ -803,7 +792,12 @@ bool bwd_tc_plan(BwdTcArgs& a) {
   const int s = a.p.seq_len;
   if (s < 1 || s > 256) return false;
   const uint32_t rows8 = static_cast<uint32_t>((s + 7) & ~7);
-  a.panel_bytes = rows8 * 128u;
+  const uint32_t rows16 = static_cast<uint32_t>((s + 15) & ~15);
+  // Two tiles: operand tiles of the sequence rounded to 16 rows (the column products contract over
+  // it in steps of 16), and the P/dS scratch slot in the same panels.
+  if (s > 128 && 8u * rows16 * 128u > kBwdPdsSlotMaxBytes) return false;
+  a.panel_bytes = (s > 128 ? rows16 : rows8) * 128u;
+  a.pds_slot_bytes = s > 128 ? 8u * a.panel_bytes : 0u;
   // Past the last allocation's second panel the MMAs read up to the last 128-row tile's end (A
   // operands) and the sequence rounded to 16 rows (B operands).
   const uint32_t tiles = static_cast<uint32_t>((s + 127) / 128);
