@@ -118,7 +118,9 @@ __device__ __forceinline__ float row_dot(const uint8_t* a, const uint8_t* b, int
 }
 
 // The 128 fp32 values of this thread's row in TMEM columns [col, col + 128), written to global memory
-// when `store`: times `mul`, plus `acc` (fp32 row) if given, as bf16 to `out16` or as fp32 to `out32`.
+// when `store`: times `mul`, plus `acc` (fp32 row) if given, as bf16 to `out16` or as fp32 to `out32`
+// (acc and out32 rows are 32-byte aligned: workspace rows of 512 bytes, read and written 32 bytes at a
+// time).
 // Every thread of the warp calls it (tcgen05.ld is warp-wide); only the stores depend on `store`.
 __device__ __forceinline__ void write_row(uint32_t taddr, bool store, float mul, const float* acc,
                                           __nv_bfloat16* out16, float* out32) {
@@ -131,14 +133,12 @@ __device__ __forceinline__ void write_row(uint32_t taddr, bool store, float mul,
 #pragma unroll
     for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]) * mul;
     if (acc != nullptr) {
-      const float4* a4 = reinterpret_cast<const float4*>(acc + 64 * h);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const float4 x = a4[i];
-        v[4 * i] += x.x;
-        v[4 * i + 1] += x.y;
-        v[4 * i + 2] += x.z;
-        v[4 * i + 3] += x.w;
+      for (int i = 0; i < 8; ++i) {
+        float x[8];
+        ldg_v8(acc + 64 * h + 8 * i, x);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[8 * i + j] += x[j];
       }
     }
     if (out16 != nullptr) {
@@ -148,9 +148,8 @@ __device__ __forceinline__ void write_row(uint32_t taddr, bool store, float mul,
         o4[i] = make_uint4(pack_bf16x2(v[8 * i], v[8 * i + 1]), pack_bf16x2(v[8 * i + 2], v[8 * i + 3]),
                            pack_bf16x2(v[8 * i + 4], v[8 * i + 5]), pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
     } else {
-      float4* o4 = reinterpret_cast<float4*>(out32 + 64 * h);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) o4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+      for (int i = 0; i < 8; ++i) stg_v8(out32 + 64 * h + 8 * i, &v[8 * i]);
     }
   }
 }
@@ -366,6 +365,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_rows_kernel(const __grid_cons
       const int nq = chunk_valid_rows(p, qc);
       const int tok = rl < nq ? token_of(g, p, sigma, qc, rl) : -1;
       const size_t ro = (static_cast<size_t>(bh) * g.n + (tok < 0 ? 0 : tok)) * 128;
+      if (a.accumulate && tok >= 0) prefetch_l2(a.dq_acc + ro, 512u);   // the earlier passes' share: into L2
       ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->o_full[k & 1], (k >> 1) & 1, ctl));
       if (!ok) break;
       tc_fence_after();
@@ -558,6 +558,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_cols_kernel(const __grid_cons
       const int nk = chunk_valid_rows(p, kc);
       const int tok = rl < nk ? token_of(g, p, sigma, kc, rl) : -1;
       const size_t ro = (static_cast<size_t>(bh) * g.n + (tok < 0 ? 0 : tok)) * 128;
+      if (a.accumulate && tok >= 0) prefetch_l2(a.dk_acc + ro, 512u);   // the earlier passes' share: into L2
       ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->o_full[0], k & 1, ctl));
       if (!ok) break;
       tc_fence_after();

@@ -89,7 +89,9 @@ __device__ __forceinline__ uint64_t kdesc(uint32_t addr, int kk, uint32_t panel)
 }
 
 // The 128 fp32 values of this thread's row in TMEM columns [col, col + 128), written to global memory
-// when `store`: times `mul`, plus `acc` (fp32 row) if given, as bf16 to `out16` or as fp32 to `out32`.
+// when `store`: times `mul`, plus `acc` (fp32 row) if given, as bf16 to `out16` or as fp32 to `out32`
+// (acc and out32 rows are 32-byte aligned: workspace rows of 512 bytes, read and written 32 bytes at a
+// time).
 // Every thread of the warp calls it (tcgen05.ld is warp-wide); only the stores depend on `store`.
 __device__ __forceinline__ void write_row(uint32_t taddr, bool store, float mul, const float* acc,
                                           __nv_bfloat16* out16, float* out32) {
@@ -102,14 +104,12 @@ __device__ __forceinline__ void write_row(uint32_t taddr, bool store, float mul,
 #pragma unroll
     for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]) * mul;
     if (acc != nullptr) {
-      const float4* a4 = reinterpret_cast<const float4*>(acc + 64 * h);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const float4 x = a4[i];
-        v[4 * i] += x.x;
-        v[4 * i + 1] += x.y;
-        v[4 * i + 2] += x.z;
-        v[4 * i + 3] += x.w;
+      for (int i = 0; i < 8; ++i) {
+        float x[8];
+        ldg_v8(acc + 64 * h + 8 * i, x);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[8 * i + j] += x[j];
       }
     }
     if (out16 != nullptr) {
@@ -119,9 +119,8 @@ __device__ __forceinline__ void write_row(uint32_t taddr, bool store, float mul,
         o4[i] = make_uint4(pack2_rn(v[8 * i], v[8 * i + 1]), pack2_rn(v[8 * i + 2], v[8 * i + 3]),
                            pack2_rn(v[8 * i + 4], v[8 * i + 5]), pack2_rn(v[8 * i + 6], v[8 * i + 7]));
     } else {
-      float4* o4 = reinterpret_cast<float4*>(out32 + 64 * h);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) o4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+      for (int i = 0; i < 8; ++i) stg_v8(out32 + 64 * h + 8 * i, &v[8 * i]);
     }
   }
 }
@@ -333,6 +332,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
     // rows: D, then P and dS of each 128-query tile; dS packed over S for dQ = dS K, and P and dS of
     // every row also written to this CTA's scratch slot for the column products
     const int rows = static_cast<int>(panel / 128u);   // rows of a scratch panel (the sequence rounded to 16)
+    for (int t = 1; t < ntiles; ++t) {   // the output rows of the later tiles (for D): into L2 now
+      const int r = 128 * t + rl;
+      const int tok = r < s ? token_of(g, p, sigma, 0, r) : -1;
+      if (tok >= 0) prefetch_l2(a.o + (static_cast<size_t>(bh) * g.n + tok) * 128, 256u);
+    }
     for (int t = 0; t < ntiles && ok; ++t) {
       const int r = 128 * t + rl;
       const int tok = r < s ? token_of(g, p, sigma, 0, r) : -1;
@@ -411,6 +415,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc_kernel(const __grid_con
     for (int seq = static_cast<int>(blockIdx.x); ok && seq < seqs; seq += static_cast<int>(gridDim.x)) {
       const int bh = static_cast<int>(fdiv(static_cast<uint32_t>(seq), p.f_per_bh));
       const int sigma = seq - bh * p.n_seq;
+      if (a.accumulate) {
+        // the earlier passes' fp32 shares of this sequence's rows, added below: into L2 now
+        for (int t = 0; t < ntiles; ++t) {
+          const int r = 128 * t + rl;
+          const int tok = r < s ? token_of(g, p, sigma, 0, r) : -1;
+          if (tok >= 0) {
+            const size_t ro = (static_cast<size_t>(bh) * g.n + tok) * 128;
+            prefetch_l2(a.dq_acc + ro, 512u);
+            prefetch_l2(a.dk_acc + ro, 512u);
+          }
+        }
+      }
       for (int t = 0; t < 2 * ntiles && ok; ++t) {   // row tiles, then key tiles
         const int r = 128 * (t < ntiles ? t : t - ntiles) + rl;
         const int tok = r < s ? token_of(g, p, sigma, 0, r) : -1;
@@ -728,6 +744,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_tc1_kernel(const __grid_co
         tok = token_of(g, p, gs - bh * p.n_seq, 0, pos);
       }
       const size_t ro = (static_cast<size_t>(bh) * g.n + (tok < 0 ? 0 : tok)) * 128;
+      if (a.accumulate && tok >= 0) {   // the earlier passes' fp32 shares of this row: into L2 now
+        prefetch_l2(a.dq_acc + ro, 512u);
+        prefetch_l2(a.dk_acc + ro, 512u);
+      }
       ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->o_full, it & 1u, ctl));
       if (!ok) break;
       tc_fence_after();
