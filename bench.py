@@ -376,9 +376,9 @@ def run_ours(args, rank, world, local_rank):
         "single_pass": single,
         "backward": {"ms_per_block": bwd_ms,
                      "tflops_algorithmic": 2.0 * f / (bwd_ms * 1e-3) / 1e12,
-                     "flops_note": "algorithmic = 2x forward (dQ, dK, dV, dP products); executed: 3.5x forward "
-                                   "for the 168-token windows (S and dP recomputed for the row and for the column "
-                                   "products), 2.5x for the 110-token slot sequences (one tile, no recomputation)",
+                     "flops_note": "algorithmic = 2x forward (dQ, dK, dV, dP products); executed: 2.5x forward "
+                                   "(S and dP once; the 168-token windows' P and dS pass through an L2 scratch "
+                                   "to the column products, the 110-token slot sequences through shared memory)",
                      "kernels": "tcgen05, one persistent launch per pass (one CTA per SM; row-owner, epilogue "
                                 "and load/MMA warps): bwd_tc1_kernel (slot sequences) then bwd_tc_kernel (windows)"},
     }
