@@ -528,6 +528,8 @@ size_t pds_bytes(const squad_params_t* sp, const Grid& g) {
   size_t m = 0;
   if (sp->dtype != SQUAD_BF16) return 0;
   for (const int kind : {kLocal, kGlobal}) {
+    if ((kind == kLocal && sp->order == SQUAD_GLOBAL_ONLY) || (kind == kGlobal && sp->order == SQUAD_LOCAL_ONLY))
+      continue;   // a pass this order does not run
     BwdTcArgs b;
     std::memset(&b, 0, sizeof(b));
     b.g = g;

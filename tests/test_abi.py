@@ -5,6 +5,7 @@ import os
 import re
 
 import pytest
+import torch
 
 from oracle import squad_oracle as orc
 from sub_quadratic_two_squad_b200 import _lib, make_params
@@ -223,3 +224,21 @@ def test_backward_kernel_selection(lib, grid, window, order, dtype, d, expect):
     assert (ks[0], ks[1]) == expect
     assert lib.squad_attn_bwd_kernels(ctypes.byref(prm), None) == _lib.SQUAD_ERR_INVALID_ARG
     assert lib.squad_attn_bwd_kernels(ctypes.byref(make_params(1, 2, d, grid, (4, 2, 4), order, dtype)), ks) != 0
+
+
+def test_bwd_workspace_carries_pds_scratch_only_where_the_whole_sequence_kernel_needs_it():
+    """The whole-sequence backward (129-208 tokens) keeps each sequence's P and dS in one scratch slot per
+    resident CTA (160 slots of 8 panels of the sequence rounded to 16 rows x 128 bytes); other passes
+    need none. Same n, so the rest of the workspace is the same size."""
+    lib = _lib.load()
+
+    def ws(window, order="local_then_global", dtype=torch.bfloat16):
+        prm = make_params(1, 24, 128, (21, 22, 40), window, order, dtype)
+        return lib.squad_attn_bwd_workspace_bytes(ctypes.byref(prm))
+
+    slot = 8 * 176 * 128                                   # 168-token windows: 176-row panels
+    base = ws((21, 1, 4))                                  # 84-token windows, 220-token slots: no scratch
+    assert ws((21, 2, 4)) == base + 160 * slot             # local pass of 168 tokens
+    assert ws((21, 2, 4), "local_only") == base + 160 * slot
+    assert ws((21, 2, 4), "global_only") == base           # 110-token slots: the one-tile kernel
+    assert ws((21, 2, 4), dtype=torch.float32) == ws((21, 1, 4), dtype=torch.float32)   # CUDA-core kernels
