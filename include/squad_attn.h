@@ -278,7 +278,9 @@ SQUAD_API squad_status_t squad_kpass_fwd(const squad_kpass_params_t* p, const vo
                                          const void* v, void* o, void* workspace, squad_stream_t stream);
 
 /* Bytes of backward workspace: a control block, fp32 dQ and dK shares, per-row softmax-Jacobian terms
- * and up to two intermediate value gradients (input dtype). 0 for invalid parameters. */
+ * and up to two intermediate value gradients (input dtype), plus, when a level has sequences of 129 to
+ * 208 tokens, the bf16 P and dS of one sequence per resident CTA (as for squad_attn_bwd). 0 for
+ * invalid parameters. */
 SQUAD_API size_t squad_kpass_bwd_workspace_bytes(const squad_kpass_params_t* p);
 
 /* Backward (the chain rule through the k passes, last executed first): gradients of <dout, o> with
