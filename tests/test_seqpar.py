@@ -1,4 +1,4 @@
-"""Sequence-parallel SQuad (one all-to-all between the passes), world size 2 over gloo on the CPU.
+"""Sequence-parallel SQuad (one all-to-all between the passes), world sizes 2, 3 and 4 over gloo on the CPU.
 
 Each rank holds a band of window rows; the per-rank compute is the fp64 oracle's single-pass functions
 (test doubles for the library calls), so this checks the exchange and the composition of the passes
@@ -64,9 +64,17 @@ def _assemble(bands, grid):
     return np.concatenate(parts, axis=3).reshape(B, h, T * H * W, d)
 
 
+SPLITS = [
+    # (world, grid, window): T % R == 0 and (H / hw) % R == 0
+    (2, (4, 8, 6), (4, 2, 3)),     # two row bands of two window rows, two frames per group
+    (3, (3, 6, 6), (3, 2, 3)),     # a world size that is not a power of two: one window row per band
+    (4, (4, 8, 6), (4, 2, 3)),     # one frame per group: the global pass's window is one frame deep
+]
+
+
+@pytest.mark.parametrize("world,grid,window", SPLITS)
 @pytest.mark.parametrize("order", ["local_then_global", "global_then_local"])
-def test_sequence_parallel_matches_whole_grid(order):
-    grid, window, world = (4, 8, 6), (4, 2, 3), 2
+def test_sequence_parallel_matches_whole_grid(order, world, grid, window):
     with mp.get_context("spawn").Manager() as m:
         result = m.dict()
         mp.spawn(_rank_main, args=(world, _free_port(), grid, window, order, result), nprocs=world, join=True)
