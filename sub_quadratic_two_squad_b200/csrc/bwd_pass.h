@@ -1,5 +1,5 @@
 // Arguments and launchers of the tensor-core backward kernels (bwd_tc.cu): one SQuad pass's gradients
-// over sequences of at most 256 tokens, each sequence loaded whole (Q, K, V, dO) as TMA boxes.
+// over sequences of at most 208 tokens, each sequence loaded whole (Q, K, V, dO) as TMA boxes.
 #pragma once
 
 #include <cuda.h>

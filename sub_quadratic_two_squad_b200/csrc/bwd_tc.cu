@@ -1,4 +1,4 @@
-// Tensor-core backward of one SQuad pass over sequences of at most 256 tokens, sm_100a.
+// Tensor-core backward of one SQuad pass over sequences of at most 208 tokens, sm_100a.
 //
 // Each pass of SQuad-Attention is ordinary softmax attention inside each sequence (a window for the
 // local pass, a slot across windows for the global pass; SQuad paper §3.2), so its gradients are those
