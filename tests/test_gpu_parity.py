@@ -221,6 +221,23 @@ def _bwd_kernels(h, grid, window, order):
     return squad_attn_bwd_kernels(1, h, 128, grid, window, order, torch.bfloat16)
 
 
+@pytest.mark.parametrize("B,h,grid,window", [
+    (1, 2, (3, 2, 43), (3, 1, 43)),     # local 129 = 128 + 1 rows (scratch panels of 144 rows); global 2
+    (2, 1, (2, 43, 6), (2, 1, 2)),      # global 129 (43 x 3 slot boxes); local 4
+    (1, 2, (3, 30, 52), (3, 2, 4)),     # global 195: 13 rows past the sequence in 208-row panels
+    (1, 2, (13, 4, 32), (13, 2, 8)),    # local 208 = 13 x 16: no padding row, dQ over dP's columns
+    (2, 1, (2, 13, 32), (2, 1, 2)),     # global 208
+    (1, 2, (11, 4, 6), (11, 3, 6)),     # local 198 on a reflect-padded grid (H 4 -> 6)
+])
+@pytest.mark.parametrize("order", [LG, GL])
+def test_backward_whole_sequence_kernel_length_range(B, h, grid, window, order):
+    """The whole-sequence backward at the ends of its two-tile range (129-208 tokens): a one-row second
+    tile, rows past the sequence up to the 16-row rounding, and sequences long enough (over 192 tokens)
+    that dQ shares tensor-memory columns with dP instead of having its own."""
+    assert _bwd_kernels(h, grid, window, order) == ("tc_whole", "tc_whole")
+    run_bwd(B, h, 128, grid, window, order, torch.bfloat16)
+
+
 @pytest.mark.parametrize("order", [LG, GL])
 def test_backward_bf16_long_windows_chunked_tensor_cores(order):
     """336-token windows (3 chunks of 8, 8 and 5 lines of 16 tokens) on the chunked tensor-core kernels;
