@@ -238,6 +238,21 @@ def test_backward_whole_sequence_kernel_length_range(B, h, grid, window, order):
     run_bwd(B, h, 128, grid, window, order, torch.bfloat16)
 
 
+@pytest.mark.parametrize("grid,window,long_pass", [
+    ((2, 64, 32), (2, 4, 2), "global"),    # slot sequences of 256 tokens (O over the second half of S); windows of 16
+    ((15, 8, 16), (15, 4, 4), "local"),    # windows of 240 = 128 + 112 rows; slot sequences of 8
+])
+@pytest.mark.parametrize("order", [LG, GL])
+def test_fused_forward_longest_short_sequences(grid, window, long_pass, order):
+    """The fused two-pass forward at the top of the short kernel's range (221-256 tokens; heavy-tailed
+    keys for the forward), and its backward, whose long pass runs on the chunked kernels."""
+    run_fwd(1, 2, 128, grid, window, order, torch.bfloat16, heavy_tail=True)
+    ks = _bwd_kernels(2, grid, window, order)
+    first_is_long = (order == LG) == (long_pass == "local")
+    assert ks == (("tc_chunked", "tc_whole") if first_is_long else ("tc_whole", "tc_chunked"))
+    run_bwd(1, 2, 128, grid, window, order, torch.bfloat16)
+
+
 @pytest.mark.parametrize("order", [LG, GL])
 def test_backward_bf16_long_windows_chunked_tensor_cores(order):
     """336-token windows (3 chunks of 8, 8 and 5 lines of 16 tokens) on the chunked tensor-core kernels;
