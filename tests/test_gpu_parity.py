@@ -238,6 +238,25 @@ def test_backward_whole_sequence_kernel_length_range(B, h, grid, window, order):
     run_bwd(B, h, 128, grid, window, order, torch.bfloat16)
 
 
+@pytest.mark.parametrize("B,h,grid,window", [
+    (1, 2, (4, 3, 22), (4, 1, 11)),     # local 44: two 48-row bands per packed tile; global 6
+    (1, 2, (4, 8, 8), (4, 4, 4)),       # local 64: two 64-row bands; global 4
+    (1, 2, (5, 2, 26), (5, 1, 13)),     # local 65: one 72-row band, products over 80 rows; global 4
+    (1, 2, (3, 2, 80), (3, 1, 40)),     # local 120: products read 8 rows past the 120-row panels
+    (1, 2, (2, 16, 16), (2, 2, 2)),     # global 64; local 8
+    (2, 1, (2, 16, 18), (2, 2, 2)),     # global 72; local 8
+    (1, 2, (3, 20, 20), (3, 2, 2)),     # global 100 (a 104-row band); local 12
+    (1, 1, (1, 120, 2), (1, 1, 2)),     # global 120; local 2
+])
+@pytest.mark.parametrize("order", [LG, GL, LO, GO])
+def test_one_tile_sequence_lengths(B, h, grid, window, order):
+    """Sequences of 44-120 tokens: the packed one-tile backward (and the packed single-pass forward) with
+    two sequences per tile, and the unpacked one where the band (the length rounded to 8 rows) is not a
+    multiple of 16, so its products read 8 rows past the panel, which meet only zero P and dS."""
+    assert all(k == "tc_whole" for k in _bwd_kernels(h, grid, window, order) if k is not None)
+    run_bwd(B, h, 128, grid, window, order, torch.bfloat16)
+
+
 @pytest.mark.parametrize("grid,window,long_pass", [
     ((2, 64, 32), (2, 4, 2), "global"),    # slot sequences of 256 tokens (O over the second half of S); windows of 16
     ((15, 8, 16), (15, 4, 4), "local"),    # windows of 240 = 128 + 112 rows; slot sequences of 8
