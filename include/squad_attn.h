@@ -130,8 +130,9 @@ SQUAD_API squad_status_t squad_attn_bwd(const squad_params_t* p, const void* q, 
 /* The kernel each pass of squad_attn_bwd(p, ...) runs on, in execution order of the forward:
  * kernels[0] for the first pass, kernels[1] for the second (0 when the order has one pass). The
  * choice depends only on p (on the padded grid where the window does not divide it):
- *   SQUAD_BWD_TC_WHOLE    tensor cores, whole sequences, one at a time per CTA (bf16, d = 128,
- *                         sequences of at most 208 tokens, whatever fits its shared-memory plan);
+ *   SQUAD_BWD_TC_WHOLE    tensor cores, whole sequences, one per work item (several per 128-row
+ *                         tile when they have at most 64 tokens) (bf16, d = 128, sequences of at
+ *                         most 208 tokens, whatever fits its shared-memory plan);
  *   SQUAD_BWD_TC_CHUNKED  tensor cores, sequences cut into chunks of whole lines of at most 128 rows
  *                         (bf16, d = 128, lines of at most 128 tokens): any sequence length;
  *   SQUAD_BWD_CUDA_CORE   the fp32 CUDA-core kernels (fp32 inputs, other d).
