@@ -168,9 +168,9 @@ SQUAD_API squad_status_t full_attn_fwd(const squad_params_t* p, const void* q, c
  * zero. Every call looks up the array's device address on the current device (a host-side query
  * with no stream work); make the first call on a device before any stream capture on it. q, k, v
  * and o must be device memory of the current device (SQUAD_ERR_INVALID_ARG otherwise: the scratch
- * used is the current device's). The LSEs and the device status word of this entry point stay inside the scratch
- * and are not exposed: a bounded device-side wait that gives up leaves o incomplete and is not
- * reported to the caller (the workspace entry point reports it through squad_attn_fwd_status).
+ * used is the current device's). The LSEs and the device status word of this entry point stay inside
+ * the scratch and are not exposed: a bounded device-side wait that gives up leaves o incomplete and
+ * is not reported to the caller (the workspace entry point reports it through squad_attn_fwd_status).
  * Returns SQUAD_ERR_UNSUPPORTED, before launching anything, when squad_attn_fwd_workspace_bytes(p)
  * exceeds SQUAD_NOALLOC_MAX_WORKSPACE_BYTES. It allocates nothing (no cudaMalloc or cudaFree). */
 SQUAD_API squad_status_t squad_attn_fwd_noalloc(const squad_params_t* p, const void* q, const void* k,
