@@ -300,6 +300,31 @@ SQUAD_API squad_status_t squad_kpass_status(const squad_kpass_params_t* p, const
 /* FLOPs of one k-pass forward: 4 B h d n (m_1 + ... + m_k); 0 for invalid parameters. */
 SQUAD_API double squad_kpass_flops(const squad_kpass_params_t* p);
 
+/* ------------------------------------------------------------------------------------------------
+ * Sequence split over R ranks: the reorderings around its all-to-all exchanges
+ *
+ * Each pass folds the axis it does not attend over into the batch of heads (agihunt.info digest, the
+ * paragraph that defines the operator), so the tokens of a block can be split over R ranks with one
+ * exchange between the passes: a rank holds a band of latent rows of every frame for the local pass,
+ * and a group of frames with every row for the global pass. A tensor of the split is a stack of
+ * blocks of Hb*W*d contiguous elements (Hb = H/R rows of one frame of one head), indexed by
+ * (b, head, r, tg) with r < R and tg < Tg = T/R, in one of three layouts:
+ *   SQUAD_SP_BAND    [B, h, R, Tg]  a rank's band: its Hb rows of frame t = r*Tg + tg ([B,h,T*Hb*W,d])
+ *   SQUAD_SP_FRAMES  [B, h, Tg, R]  a rank's frame group: row band r of its frame tg ([B,h,Tg*H*W,d])
+ *   SQUAD_SP_CHUNKS  [R, B, h, Tg]  an all-to-all buffer: chunk r goes to, or came from, rank r
+ * squad_seqpar_reorder writes y (layout `to`) from x (layout `from`), moving whole blocks; with add
+ * (layout `to`) not NULL, each element of y is the moved value plus add's element, summed in fp32 and
+ * rounded once to the dtype (the two passes' shares of dq and dk). p gives B, h, d, T, H, W and dtype
+ * (window fields and order are ignored); T and H must be multiples of R. x, add, y: device buffers
+ * of one rank's share, B*h*T*(H/R)*W*d elements, 16-byte aligned, caller-owned; y must not overlap
+ * x or add. Asynchronous on `stream`; argument errors return SQUAD_ERR_INVALID_ARG before anything is
+ * launched, a failed launch SQUAD_ERR_CUDA. */
+#define SQUAD_SP_BAND 0
+#define SQUAD_SP_FRAMES 1
+#define SQUAD_SP_CHUNKS 2
+SQUAD_API squad_status_t squad_seqpar_reorder(const squad_params_t* p, int R, int from, int to, const void* x,
+                                              const void* add, void* y, squad_stream_t stream);
+
 /* Static string for a status code (never NULL). */
 SQUAD_API const char* squad_status_string(squad_status_t s);
 

@@ -28,4 +28,5 @@ from .api import (  # noqa: F401
     squad_kpass_fwd,
     squad_kpass_pass_params,
     squad_kpass_status,
+    squad_seqpar_reorder,
 )

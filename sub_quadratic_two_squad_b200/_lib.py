@@ -9,6 +9,7 @@ LIB_PATH = os.path.join(PKG_DIR, "libsquad_attn.so")
 
 SQUAD_OK, SQUAD_ERR_INVALID_ARG, SQUAD_ERR_UNSUPPORTED, SQUAD_ERR_CUDA, SQUAD_ERR_TIMEOUT = range(5)
 SQUAD_BWD_TC_WHOLE, SQUAD_BWD_TC_CHUNKED, SQUAD_BWD_CUDA_CORE = 1, 2, 3
+SQUAD_SP_BAND, SQUAD_SP_FRAMES, SQUAD_SP_CHUNKS = 0, 1, 2
 SQUAD_BF16, SQUAD_FP32 = 0, 1
 SQUAD_LOCAL_THEN_GLOBAL, SQUAD_GLOBAL_THEN_LOCAL, SQUAD_LOCAL_ONLY, SQUAD_GLOBAL_ONLY = 0, 1, 2, 3
 SQUAD_NOALLOC_MAX_WORKSPACE_BYTES = 128 * 1024 * 1024
@@ -62,6 +63,7 @@ SIGNATURES = {
     "squad_kpass_bwd": (ctypes.c_int, [_KP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
     "squad_kpass_status": (ctypes.c_int, [_KP, _VP, _VP]),
     "squad_kpass_flops": (ctypes.c_double, [_KP]),
+    "squad_seqpar_reorder": (ctypes.c_int, [_PP, ctypes.c_int, ctypes.c_int, ctypes.c_int, _VP, _VP, _VP, _VP]),
     "squad_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "squad_attn_abi_version": (ctypes.c_int, []),
 }

@@ -179,6 +179,36 @@ def full_attn_fwd(q, k, v, grid=None, scale=None, out=None, lse=None, stream=Non
     return out
 
 
+SP_LAYOUTS = {"band": _lib.SQUAD_SP_BAND, "frames": _lib.SQUAD_SP_FRAMES, "chunks": _lib.SQUAD_SP_CHUNKS}
+
+
+def squad_seqpar_reorder(x, grid, R, src, dst, add=None, out=None, stream=None):
+    """The sequence split's block reordering (squad_seqpar_reorder): x in layout `src` ("band",
+    "frames" or "chunks") -> a new tensor in layout `dst`, plus `add` (layout `dst`) if given.
+    band and frames tensors are [B, h, n/R, d]; chunks tensors are [R, B, h, n/R^2, d] (the all-to-all
+    splits their first dimension)."""
+    T, H, W = grid
+    if x.dim() not in (4, 5) or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("x must be a contiguous CUDA tensor [B, h, n/R, d] or [R, B, h, n/R^2, d]")
+    B, h = (x.shape[1], x.shape[2]) if x.dim() == 5 else (x.shape[0], x.shape[1])
+    d = x.shape[-1]
+    if R < 1 or T % R or H % R or x.numel() * R != B * h * T * H * W * d or (x.dim() == 5) != (src == "chunks"):
+        raise ValueError(f"x does not hold one rank's {src} tensor of the {T}x{H}x{W} grid split {R} ways")
+    shape = (R, B, h, T * H * W // (R * R), d) if dst == "chunks" else (B, h, T * H * W // R, d)
+    out = torch.empty(shape, dtype=x.dtype, device=x.device) if out is None else out
+    for t in (add, out):
+        if t is not None and (not t.is_cuda or not t.is_contiguous() or t.dtype != x.dtype or t.device != x.device
+                              or tuple(t.shape) != shape):
+            raise ValueError(f"add and out must be contiguous CUDA tensors of x's dtype and device, shape {shape}")
+    prm = make_params(B, h, d, grid, (T, 1, 1), "local_then_global", x.dtype)
+    with torch.cuda.device(x.device):
+        st = _lib.load().squad_seqpar_reorder(ctypes.byref(prm), int(R), SP_LAYOUTS[src], SP_LAYOUTS[dst], _ptr(x),
+                                              _ptr(add), _ptr(out), _stream(stream))
+    if st != _lib.SQUAD_OK:
+        raise SquadError(st, "squad_seqpar_reorder")
+    return out
+
+
 def squad_attn_flops(B, h, d, grid, window, order="local_then_global") -> float:
     return float(_lib.load().squad_attn_flops(ctypes.byref(make_params(B, h, d, grid, window, order))))
 

@@ -14,11 +14,14 @@ block can be split over R ranks with one exchange between the passes:
 The global-then-local order runs the same steps the other way round, and the backward retraces them.
 Requirements: T % R == 0, H % hw == W % ww == 0 and (H / hw) % R == 0.
 
-Compute is the library's single-pass forward and backward (`local_only` / `global_only`); the exchange
-is torch.distributed.all_to_all_single on contiguous buffers, so on GPUs it is NCCL over NVLink. The
-per-rank compute can be replaced (`fwd`, `bwd` arguments) for testing the exchange without a GPU.
-With one rank both exchanges are the identity and the band is the whole grid, so the library's fused
-two-pass forward and its backward run directly (no exchange buffers, no single-pass split).
+Compute is the library's single-pass forward and backward (`local_only` / `global_only`). Around each
+exchange the library's squad_seqpar_reorder moves the blocks between the band, frame-group and
+all-to-all layouts, and adds the two passes' dQ and dK shares while moving the second one back; the
+exchange itself is torch.distributed.all_to_all_single on those buffers, so on GPUs it is NCCL over
+NVLink. The per-rank compute and the reordering can be replaced (`fwd`, `bwd`, `reorder` arguments) for
+testing the composition without a GPU. With one rank both exchanges are the identity and the band is
+the whole grid, so the library's fused two-pass forward and its backward run directly (no exchange
+buffers, no single-pass split).
 """
 from __future__ import annotations
 
@@ -27,7 +30,7 @@ import torch.distributed as dist
 
 
 class SeqParallelSquad:
-    def __init__(self, grid, window, group=None, fwd=None, bwd=None):
+    def __init__(self, grid, window, group=None, fwd=None, bwd=None, reorder=None):
         self.group = group
         self.R = dist.get_world_size(group)
         self.rank = dist.get_rank(group)
@@ -42,11 +45,12 @@ class SeqParallelSquad:
         self.frame_window = (self.Tg, hw, ww)
         # one rank with the library's own compute: the fused launch, no exchange
         self.whole = self.R == 1 and fwd is None and bwd is None
-        if fwd is None or bwd is None:
-            from .api import squad_attn_bwd, squad_attn_fwd
+        if fwd is None or bwd is None or reorder is None:
+            from .api import squad_attn_bwd, squad_attn_fwd, squad_seqpar_reorder
             fwd = fwd or (lambda q, k, v, g, w, o: squad_attn_fwd(q, k, v, g, w, o))
             bwd = bwd or (lambda q, k, v, out, do, ws, g, w, o: squad_attn_bwd(q, k, v, out, do, ws, g, w, o))
-        self._fwd, self._bwd = fwd, bwd
+            reorder = reorder or squad_seqpar_reorder
+        self._fwd, self._bwd, self._reorder = fwd, bwd, reorder
 
     # -------------------------------------------------------------------------------- exchange
     def _a2a(self, send):
@@ -56,21 +60,16 @@ class SeqParallelSquad:
 
     def band_to_frames(self, x):
         """[B, h, T*Hb*W, d] (this rank's rows, all frames) -> [B, h, Tg*H*W, d] (its frames, all rows)."""
-        B, h, _, d = x.shape
-        T, _, W = self.grid
-        R, Hb, Tg = self.R, self.Hb, self.Tg
-        send = x.reshape(B, h, R, Tg, Hb, W, d).permute(2, 0, 1, 3, 4, 5, 6).contiguous()   # chunk per frame group
-        recv = self._a2a(send)                                                              # chunk per row band
-        return recv.permute(1, 2, 3, 0, 4, 5, 6).reshape(B, h, Tg * R * Hb * W, d)
+        send = self._reorder(x, self.grid, self.R, "band", "chunks")       # a chunk per frame group
+        recv = self._a2a(send)                                             # a chunk per row band
+        return self._reorder(recv, self.grid, self.R, "chunks", "frames")
 
-    def frames_to_band(self, x):
-        """[B, h, Tg*H*W, d] -> [B, h, T*Hb*W, d], the inverse of band_to_frames."""
-        B, h, _, d = x.shape
-        T, _, W = self.grid
-        R, Hb, Tg = self.R, self.Hb, self.Tg
-        send = x.reshape(B, h, Tg, R, Hb, W, d).permute(3, 0, 1, 2, 4, 5, 6).contiguous()   # chunk per row band
-        recv = self._a2a(send)                                                              # chunk per frame group
-        return recv.permute(1, 2, 0, 3, 4, 5, 6).reshape(B, h, R * Tg * Hb * W, d)
+    def frames_to_band(self, x, add=None):
+        """[B, h, Tg*H*W, d] -> [B, h, T*Hb*W, d], the inverse of band_to_frames; plus `add` (a band
+        tensor) if given."""
+        send = self._reorder(x, self.grid, self.R, "frames", "chunks")     # a chunk per row band
+        recv = self._a2a(send)                                             # a chunk per frame group
+        return self._reorder(recv, self.grid, self.R, "chunks", "band", add=add)
 
     # -------------------------------------------------------------------------------- passes
     def _local(self, q, k, v):
@@ -109,14 +108,14 @@ class SeqParallelSquad:
             _, q, k, v, o1, ws1, qf, kf, o1f, of, ws2 = ctx
             dqf, dkf, do1f = self._bwd(qf, kf, o1f, of, self.band_to_frames(dout), ws2, self.frame_grid,
                                        self.frame_window, "global_only")
-            dq_g, dk_g, do1 = self.frames_to_band(dqf), self.frames_to_band(dkf), self.frames_to_band(do1f)
+            do1 = self.frames_to_band(do1f)
             dq_l, dk_l, dv = self._bwd(q, k, v, o1, do1, ws1, self.band_grid, self.window, "local_only")
-            return dq_l + dq_g, dk_l + dk_g, dv
+            return self.frames_to_band(dqf, add=dq_l), self.frames_to_band(dkf, add=dk_l), dv
         _, q, k, v, o1, o, ws2, qf, kf, vf, o1f, ws1 = ctx
         dq_l, dk_l, do1 = self._bwd(q, k, o1, o, dout, ws2, self.band_grid, self.window, "local_only")
         dqf, dkf, dvf = self._bwd(qf, kf, vf, o1f, self.band_to_frames(do1), ws1, self.frame_grid,
                                   self.frame_window, "global_only")
-        return dq_l + self.frames_to_band(dqf), dk_l + self.frames_to_band(dkf), self.frames_to_band(dvf)
+        return self.frames_to_band(dqf, add=dq_l), self.frames_to_band(dkf, add=dk_l), self.frames_to_band(dvf)
 
 
 def band_of(x, grid, rank, R):

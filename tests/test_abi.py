@@ -242,3 +242,24 @@ def test_bwd_workspace_carries_pds_scratch_only_where_the_whole_sequence_kernel_
     assert ws((21, 2, 4), "local_only") == base + 160 * slot
     assert ws((21, 2, 4), "global_only") == base           # 110-token slots: the one-tile kernel
     assert ws((21, 2, 4), dtype=torch.float32) == ws((21, 1, 4), dtype=torch.float32)   # CUDA-core kernels
+
+
+def test_seqpar_reorder_rejects_bad_arguments(lib):
+    """Argument errors come back before anything is launched (no GPU needed)."""
+    prm = make_params(1, 2, 128, (4, 6, 5), (4, 1, 1))
+    a, b, c = ctypes.c_void_p(4096), ctypes.c_void_p(8192), ctypes.c_void_p(12288)
+    bad = ctypes.c_void_p(4104)   # 8-byte aligned only
+    reorder = lib.squad_seqpar_reorder
+    assert reorder(None, 2, 0, 2, a, None, b, None) == _lib.SQUAD_ERR_INVALID_ARG
+    assert reorder(ctypes.byref(prm), 0, 0, 2, a, None, b, None) == _lib.SQUAD_ERR_INVALID_ARG     # R < 1
+    assert reorder(ctypes.byref(prm), 3, 0, 2, a, None, b, None) == _lib.SQUAD_ERR_INVALID_ARG     # H % R (T = 4)
+    assert reorder(ctypes.byref(prm), 4, 0, 2, a, None, b, None) == _lib.SQUAD_ERR_INVALID_ARG     # T % R ok, H % R
+    assert reorder(ctypes.byref(prm), 2, 0, 3, a, None, b, None) == _lib.SQUAD_ERR_INVALID_ARG     # layout
+    assert reorder(ctypes.byref(prm), 2, -1, 2, a, None, b, None) == _lib.SQUAD_ERR_INVALID_ARG
+    assert reorder(ctypes.byref(prm), 2, 0, 2, a, None, a, None) == _lib.SQUAD_ERR_INVALID_ARG     # y == x
+    assert reorder(ctypes.byref(prm), 2, 0, 2, a, b, b, None) == _lib.SQUAD_ERR_INVALID_ARG        # y == add
+    assert reorder(ctypes.byref(prm), 2, 0, 2, bad, None, b, None) == _lib.SQUAD_ERR_INVALID_ARG   # alignment
+    assert reorder(ctypes.byref(prm), 2, 0, 2, a, bad, c, None) == _lib.SQUAD_ERR_INVALID_ARG
+    assert reorder(ctypes.byref(prm), 2, 0, 2, a, None, None, None) == _lib.SQUAD_ERR_INVALID_ARG
+    odd = make_params(1, 2, 96, (4, 6, 5), (4, 1, 1))
+    assert reorder(ctypes.byref(odd), 2, 0, 2, a, None, b, None) == _lib.SQUAD_ERR_INVALID_ARG     # d

@@ -1,8 +1,10 @@
 """Sequence-parallel SQuad (one all-to-all between the passes), world sizes 2, 3 and 4 over gloo on the CPU.
 
-Each rank holds a band of window rows; the per-rank compute is the fp64 oracle's single-pass functions
-(test doubles for the library calls), so this checks the exchange and the composition of the passes
-against the oracle's whole-grid result, forward and backward, in both orders."""
+Each rank holds a band of window rows; the per-rank compute is the fp64 oracle's single-pass functions and
+the block reordering around the exchanges a plain torch statement of it (test doubles for the library
+calls, which tests/test_gpu_seqpar.py checks against the same statement), so this checks the exchange and
+the composition of the passes against the oracle's whole-grid result, forward and backward, in both
+orders."""
 import os
 import socket
 
@@ -28,6 +30,23 @@ def _bwd(q, k, v, o, do, ws, grid, window, order):
     return tuple(torch.from_numpy(x) for x in g)
 
 
+# Axis order of the block index (b, head, r, tg) in each layout of the split (a block is Hb*W*d contiguous
+# elements): the library's squad_seqpar_reorder moves blocks between these layouts.
+AXES = {"band": "bhrt", "frames": "bhtr", "chunks": "rbht"}
+
+
+def torch_reorder(x, grid, R, src, dst, add=None):
+    """Plain torch statement of the split's block reordering (the test double of squad_seqpar_reorder)."""
+    T, H, W = grid
+    d = x.shape[-1]
+    B, h = (x.shape[1], x.shape[2]) if src == "chunks" else (x.shape[0], x.shape[1])
+    size = {"b": B, "h": h, "r": R, "t": T // R}
+    blocks = x.reshape(*(size[a] for a in AXES[src]), (H // R) * W * d)
+    y = blocks.permute(*(AXES[src].index(a) for a in AXES[dst]), 4).contiguous()
+    y = y.reshape((R, B, h, -1, d) if dst == "chunks" else (B, h, -1, d))
+    return y if add is None else y + add
+
+
 def _free_port():
     with socket.socket() as s:
         s.bind(("127.0.0.1", 0))
@@ -41,7 +60,7 @@ def _rank_main(rank, world, port, grid, window, order, result):
         T, H, W = grid
         rng = np.random.default_rng(5)
         q, k, v, do = (torch.from_numpy(rng.standard_normal((1, 2, T * H * W, 4))) for _ in range(4))
-        sp = SeqParallelSquad(grid, window, fwd=_fwd, bwd=_bwd)
+        sp = SeqParallelSquad(grid, window, fwd=_fwd, bwd=_bwd, reorder=torch_reorder)
         o_b, ctx = sp.forward(band_of(q, grid, rank, world), band_of(k, grid, rank, world),
                               band_of(v, grid, rank, world), order)
         grads = sp.backward(ctx, band_of(do, grid, rank, world))
@@ -94,6 +113,6 @@ def test_sequence_parallel_rejects_bad_splits():
     import unittest.mock as um
     with um.patch.object(dist, "get_world_size", return_value=2), um.patch.object(dist, "get_rank", return_value=0):
         with pytest.raises(ValueError):
-            SeqParallelSquad((3, 8, 6), (3, 2, 3), group=G(), fwd=_fwd, bwd=_bwd)     # T % R
+            SeqParallelSquad((3, 8, 6), (3, 2, 3), group=G(), fwd=_fwd, bwd=_bwd, reorder=torch_reorder)  # T % R
         with pytest.raises(ValueError):
-            SeqParallelSquad((4, 6, 6), (4, 2, 3), group=G(), fwd=_fwd, bwd=_bwd)     # (H / hw) % R
+            SeqParallelSquad((4, 6, 6), (4, 2, 3), group=G(), fwd=_fwd, bwd=_bwd, reorder=torch_reorder)  # (H / hw) % R
