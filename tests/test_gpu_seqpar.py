@@ -69,7 +69,7 @@ def _layout_shape(layout, B, h, n, d, R):
     (2, 3, 128, (4, 6, 5), 2, torch.bfloat16),
     (2, 3, 64, (6, 9, 5), 3, torch.float32),
     (1, 2, 128, (8, 8, 6), 4, torch.float32),
-    (1, 12, 128, (21, 30, 52), 3, torch.bfloat16),   # the 1.3B grid over 3 ranks: 756 blocks of 10x52 tokens
+    (1, 12, 128, (21, 30, 52), 3, torch.bfloat16),   # the 1.3B grid over 3 ranks: 252 blocks of 10x52 tokens
 ])
 def test_seqpar_reorder_matches_torch(B, h, d, grid, R, dtype):
     """squad_seqpar_reorder bit for bit against the torch statement of the block reordering, for every
