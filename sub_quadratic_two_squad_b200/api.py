@@ -186,7 +186,8 @@ def squad_seqpar_reorder(x, grid, R, src, dst, add=None, out=None, stream=None):
     """The sequence split's block reordering (squad_seqpar_reorder): x in layout `src` ("band",
     "frames" or "chunks") -> a new tensor in layout `dst`, plus `add` (layout `dst`) if given.
     band and frames tensors are [B, h, n/R, d]; chunks tensors are [R, B, h, n/R^2, d] (the all-to-all
-    splits their first dimension)."""
+    splits their first dimension). With one rank, or src == dst, and neither add nor out given, the
+    layouts order the blocks alike and x itself is returned, reshaped."""
     T, H, W = grid
     if x.dim() not in (4, 5) or not x.is_cuda or not x.is_contiguous():
         raise ValueError("x must be a contiguous CUDA tensor [B, h, n/R, d] or [R, B, h, n/R^2, d]")
@@ -195,6 +196,8 @@ def squad_seqpar_reorder(x, grid, R, src, dst, add=None, out=None, stream=None):
     if R < 1 or T % R or H % R or x.numel() * R != B * h * T * H * W * d or (x.dim() == 5) != (src == "chunks"):
         raise ValueError(f"x does not hold one rank's {src} tensor of the {T}x{H}x{W} grid split {R} ways")
     shape = (R, B, h, T * H * W // (R * R), d) if dst == "chunks" else (B, h, T * H * W // R, d)
+    if add is None and out is None and (R == 1 or src == dst):
+        return x.view(shape)   # the two layouts order the blocks alike: nothing moves
     out = torch.empty(shape, dtype=x.dtype, device=x.device) if out is None else out
     for t in (add, out):
         if t is not None and (not t.is_cuda or not t.is_contiguous() or t.dtype != x.dtype or t.device != x.device
