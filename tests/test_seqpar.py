@@ -116,3 +116,19 @@ def test_sequence_parallel_rejects_bad_splits():
             SeqParallelSquad((3, 8, 6), (3, 2, 3), group=G(), fwd=_fwd, bwd=_bwd, reorder=torch_reorder)  # T % R
         with pytest.raises(ValueError):
             SeqParallelSquad((4, 6, 6), (4, 2, 3), group=G(), fwd=_fwd, bwd=_bwd, reorder=torch_reorder)  # (H / hw) % R
+
+
+def test_reorder_moves_nothing_when_the_layouts_order_blocks_alike():
+    """The premise of the library's shortcut (a view instead of a copy): with one rank every pair of
+    layouts, and with any R a layout and itself, order the blocks alike."""
+    B, h, d = 2, 3, 4
+    for R, grid in ((1, (4, 6, 5)), (2, (4, 6, 5)), (3, (6, 9, 5))):
+        n = grid[0] * grid[1] * grid[2]
+        pairs = [(a, b) for a in AXES for b in AXES] if R == 1 else [(a, a) for a in AXES]
+        for src, dst in pairs:
+            shape = (R, B, h, n // (R * R), d) if src == "chunks" else (B, h, n // R, d)
+            x = torch.arange(B * h * n // R * d, dtype=torch.float64).reshape(shape)
+            assert torch.equal(torch_reorder(x, grid, R, src, dst).flatten(), x.flatten()), (R, src, dst)
+    # and with more than one rank, different layouts do move blocks
+    x = torch.arange(B * h * 120 // 2 * d, dtype=torch.float64).reshape(B, h, 60, d)
+    assert not torch.equal(torch_reorder(x, (4, 6, 5), 2, "band", "frames").flatten(), x.flatten())
